@@ -1,0 +1,455 @@
+/*
+ * oracle.c -- plain, slow, fp64 CPU oracle for confidence-scheduled
+ * speculative verification.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file: only the tests, the smoke check and the benchmark's CPU
+ * baseline use it.  It shares no source, header, table or constant with the
+ * CUDA library; the two meet only through the seeded synthetic inputs.
+ *
+ * Sources (cited as page title + section):
+ *  [P1] umans.ai, "DeepSeek V4 Pro DSpark: the model isn't ready, the
+ *       architecture is": sections "Speculative decoding, briefly" and
+ *       "What DSpark adds" (item "2. Verify smarter").
+ *  [P2] en.5iter.com DSpark news article: sections "Guess first, then test"
+ *       and "What DSpark changed is how to generate a draft".
+ *  [P3] zhichai.net DSpark topic: sections "Why LLMs speak so slowly" and
+ *       "Under the hood: why parallel drafts get weirder".
+ *  [P4] techvisionai, "DeepSeek-V4: Breaking the Efficiency Barrier",
+ *       Chapter 7 "DSpark", subsections "Confidence-Scheduled Verification"
+ *       and "Deployment with vLLM".
+ *  [P5] aiweekly.co, "DeepSeek DSpark accelerates V4 per-user generation
+ *       60-85%".
+ *  [SC11] J. Salmon, M. Moraes, R. Dror, D. Shaw, "Parallel Random Numbers:
+ *       As Easy as 1, 2, 3", SC'11 -- the Philox-4x32 bijection.
+ *
+ * The pages state the rule in words only: the target accepts the prefix it
+ * agrees with plus one token of its own [P1 "Speculative decoding, briefly"],
+ * by rejection sampling on the target/draft probability ratio [P3 "Why LLMs
+ * speak so slowly"], so that accepted tokens follow the target distribution
+ * exactly [P1]; a rejected token is replaced by one the target would produce
+ * [P1].  Written out in symbols (the standard speculative-sampling rule):
+ *   accept x_i with probability min(1, p_i(x_i) / q_i(x_i)); at the first
+ *   rejection j emit a draw from norm(max(0, p_j - q_j)); if all L drafts
+ *   survive emit a bonus draw from p_L.
+ * The verify length L comes from prefix survival S_i = prod_{j<=i} c_j
+ * [P1 "Verify smarter"; P5] cut at a load threshold tau [P2; P4 Ch.7].
+ *
+ * Readings where the pages are silent (each is listed in the design notes):
+ *  - accept iff u < min(1, ratio), u in [0,1);
+ *  - inverse CDF in token order, y = smallest v with C(v) > t, t = u * R;
+ *  - one temperature T per row for both models; T == 0 means greedy
+ *    (argmax, lowest index wins ties); 0 < T < 1e-6 is a data error;
+ *  - the bonus is drawn from target position L (not K);
+ *  - uniforms: Philox4x32-10 [SC11], key = (seed_lo, seed_hi), counter =
+ *    (row_lo, pos, draw, row_hi), u = (word0 >> 8) * 2^-24; draw 0 is the
+ *    accept test at position pos, draw 1 the resample/bonus at pos;
+ *  - residual mass R == 0 after a rejection (only reachable through
+ *    rounding): draw from p_j instead (flagged in the diagnostics);
+ *  - a NULL draft array means a greedy drafter: q_i is one-hot at x_i
+ *    ([P4 Ch.7 "Deployment with vLLM", draft_sample_method greedy]).
+ *
+ * Pins (tests/test_oracle_*.py): exact interval enumeration against the
+ * target distribution, chi-square of Philox-keyed draws, greedy reduction to
+ * a brute-force longest matching prefix, closed-form E[accept length],
+ * schedule invariants and a hand-worked example, and Philox agreement with
+ * Triton's independent Philox implementation run on the CPU.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { OR_F32 = 0, OR_BF16 = 1, OR_F64 = 2 };
+
+/* ---------------------------------------------------------------------------
+ * Philox4x32-10 [SC11].  One round: two 32x32->64 multiplications of the
+ * even words by the round multipliers; the high halves are XORed with the
+ * odd words and the key, the low halves pass through; the words are then
+ * permuted.  The key is bumped by the Weyl constants between rounds.
+ * ------------------------------------------------------------------------- */
+#define PHILOX_M0 0xD2511F53u
+#define PHILOX_M1 0xCD9E8D57u
+#define PHILOX_W0 0x9E3779B9u
+#define PHILOX_W1 0xBB67AE85u
+
+void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+{
+    uint32_t x0 = ctr[0], x1 = ctr[1], x2 = ctr[2], x3 = ctr[3];
+    uint32_t k0 = key[0], k1 = key[1];
+    for (int r = 0; r < 10; ++r) {
+        uint64_t p0 = (uint64_t)PHILOX_M0 * (uint64_t)x0;
+        uint64_t p1 = (uint64_t)PHILOX_M1 * (uint64_t)x2;
+        uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+        uint32_t y0 = hi1 ^ x1 ^ k0;
+        uint32_t y1 = lo1;
+        uint32_t y2 = hi0 ^ x3 ^ k1;
+        uint32_t y3 = lo0;
+        x0 = y0; x1 = y1; x2 = y2; x3 = y3;
+        k0 += PHILOX_W0;
+        k1 += PHILOX_W1;
+    }
+    out[0] = x0; out[1] = x1; out[2] = x2; out[3] = x3;
+}
+
+/* u(seed, row, pos, draw) in [0,1): the top 24 bits of word 0, scaled by
+ * 2^-24, so the value is exact in both fp32 and fp64. */
+double oracle_uniform(uint64_t seed, uint64_t row, uint32_t pos, uint32_t draw)
+{
+    uint32_t ctr[4] = { (uint32_t)row, pos, draw, (uint32_t)(row >> 32) };
+    uint32_t key[2] = { (uint32_t)seed, (uint32_t)(seed >> 32) };
+    uint32_t out[4];
+    oracle_philox4x32_10(ctr, key, out);
+    return (double)(out[0] >> 8) * (1.0 / 16777216.0);
+}
+
+/* Uniforms for n (row, pos, draw) triples; used by the statistical pins. */
+void oracle_uniform_batch(uint64_t seed, const uint64_t *row, const uint32_t *pos,
+                          const uint32_t *draw, int64_t n, double *out)
+{
+    for (int64_t k = 0; k < n; ++k) out[k] = oracle_uniform(seed, row[k], pos[k], draw[k]);
+}
+
+/* ---------------------------------------------------------------------------
+ * Logit access.  bf16 is widened by placing its 16 bits in the top half of
+ * an IEEE single, which is exact.
+ * ------------------------------------------------------------------------- */
+typedef struct { const void *p; int dtype; } vec_t;
+
+static double zval(vec_t z, int64_t v)
+{
+    if (z.dtype == OR_F64) return ((const double *)z.p)[v];
+    if (z.dtype == OR_F32) return (double)((const float *)z.p)[v];
+    uint32_t bits = (uint32_t)((const uint16_t *)z.p)[v] << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+static size_t elt_size(int dtype) { return dtype == OR_F64 ? 8 : dtype == OR_F32 ? 4 : 2; }
+
+static vec_t vec_at(const void *base, int dtype, int64_t index, int V)
+{
+    vec_t r = { (const char *)base + (size_t)index * (size_t)V * elt_size(dtype), dtype };
+    return r;
+}
+
+/* Temperature-scaled softmax statistics of one logit vector:
+ * m = max_v z_v and Sigma = sum_v exp((z_v - m) / T), so that
+ * p(v) = exp((z_v - m) / T) / Sigma. */
+static void softmax_stats(vec_t z, int V, double T, double *m_out, double *sum_out)
+{
+    double m = -INFINITY;
+    for (int v = 0; v < V; ++v) {
+        double x = zval(z, v);
+        if (x > m) m = x;
+    }
+    double s = 0.0;
+    for (int v = 0; v < V; ++v) s += exp((zval(z, v) - m) / T);
+    *m_out = m;
+    *sum_out = s;
+}
+
+/* Index of the largest logit; ties go to the lowest index. */
+static int argmax_first(vec_t z, int V)
+{
+    int best = 0;
+    double bv = zval(z, 0);
+    for (int v = 1; v < V; ++v) {
+        double x = zval(z, v);
+        if (x > bv) { bv = x; best = v; }
+    }
+    return best;
+}
+
+void oracle_vector_stats(const void *z, int dtype, int V, double T,
+                         double *m, double *sum, int32_t *amax)
+{
+    vec_t zz = { z, dtype };
+    if (T > 0.0) softmax_stats(zz, V, T, m, sum);
+    else { *m = zval(zz, argmax_first(zz, V)); *sum = 1.0; }
+    if (amax) *amax = argmax_first(zz, V);
+}
+
+/* Inverse-CDF draw in token order 0..V-1 from the unnormalised weights r:
+ * R = sum_v r(v), t = u * R, y = the smallest v with C(v) = sum_{w<=v} r(w)
+ * strictly greater than t.  margin = distance from t to the nearer CDF
+ * boundary of the chosen token, relative to R.  If no v qualifies (R == 0,
+ * or rounding put t at the total) the last v with r(v) > 0 is returned and
+ * *fallback is set; -1 if every weight is zero. */
+static int inverse_cdf(const double *r, int V, double u, double *margin, int *fallback)
+{
+    double R = 0.0;
+    for (int v = 0; v < V; ++v) R += r[v];
+    double t = u * R;
+    double C = 0.0;
+    for (int v = 0; v < V; ++v) {
+        double prev = C;
+        C += r[v];
+        if (C > t) {
+            double a = t - prev, b = C - t;
+            *margin = (a < b ? a : b) / R;
+            *fallback = 0;
+            return v;
+        }
+    }
+    *fallback = 1;
+    *margin = 0.0;
+    for (int v = V - 1; v >= 0; --v)
+        if (r[v] > 0.0) return v;
+    return -1;
+}
+
+/* Diagnostics written per row (double[OR_NDIAG]):
+ *  [0] smallest |u_i - min(1, ratio_i)| over the tested positions 0..j
+ *      (+inf when none were tested, or for greedy rows);
+ *  [1] inverse-CDF margin of the correction/bonus draw, relative to R
+ *      (+inf for greedy rows);
+ *  [2] flags: 1 = residual mass was zero (drew from p_j), 2 = inverse-CDF
+ *      fallback taken;
+ *  [3] j: first rejected position, or L when every draft survived;
+ *  [4] R: total mass of the distribution the final token was drawn from. */
+#define OR_NDIAG 5
+
+/*
+ * One row, uniforms injected.
+ *   zt: target logits [K+1, V]; zd: draft logits [K, V] or NULL (greedy
+ *   drafter, q_i one-hot at x_i); x: draft tokens [K]; L: verify length;
+ *   T: temperature (0 = greedy verification); u_acc[i]: accept uniform of
+ *   position i; u_res[i]: resample/bonus uniform used if the final token is
+ *   drawn at position i.  Writes out_tokens[0..K] (x_0..x_{a-1}, y, then -1)
+ *   and returns a, the accepted length.
+ */
+static int verify_row(vec_t zt_row, const void *zd_base, int dtype, int K, int V,
+                      const int32_t *x, int L, double T,
+                      const double *u_acc, const double *u_res,
+                      int32_t *out_tokens, double *diag, double *work)
+{
+    double d0 = INFINITY, d1 = INFINITY, flags = 0.0, Rfinal = 0.0;
+    int j = L;
+    int y;
+
+    if (T == 0.0) {
+        /* Greedy verification: keep x_i while it equals the target argmax;
+         * the final token is the target argmax at the first mismatch (or at
+         * L).  No uniforms are drawn and draft logits are not read. */
+        j = L;
+        for (int i = 0; i < L; ++i) {
+            vec_t zt = vec_at(zt_row.p, dtype, i, V);
+            if (x[i] != argmax_first(zt, V)) { j = i; break; }
+        }
+        y = argmax_first(vec_at(zt_row.p, dtype, j, V), V);
+        Rfinal = 1.0;
+    } else {
+        double *r = work; /* V doubles */
+        int rejected = 0;
+        double mt = 0, st = 0, md = 0, sd = 0;
+        for (int i = 0; i < L; ++i) {
+            vec_t zt = vec_at(zt_row.p, dtype, i, V);
+            softmax_stats(zt, V, T, &mt, &st);
+            double logp = (zval(zt, x[i]) - mt) / T - log(st);
+            double logq;
+            if (zd_base) {
+                vec_t zd = vec_at(zd_base, dtype, i, V);
+                softmax_stats(zd, V, T, &md, &sd);
+                logq = (zval(zd, x[i]) - md) / T - log(sd);
+            } else {
+                logq = 0.0; /* q_i(x_i) = 1 */
+            }
+            /* min(1, p/q) in the log domain; p == 0 rejects, q == 0 accepts. */
+            double acc;
+            if (logp == -INFINITY) acc = 0.0;
+            else if (logq == -INFINITY) acc = 1.0;
+            else acc = logp >= logq ? 1.0 : exp(logp - logq);
+            double mg = fabs(u_acc[i] - acc);
+            if (mg < d0) d0 = mg;
+            if (u_acc[i] < acc) continue; /* accepted */
+            /* First rejection at i: residual r = max(0, p_i - q_i). */
+            j = i;
+            rejected = 1;
+            for (int v = 0; v < V; ++v) {
+                double p = exp((zval(zt, v) - mt) / T) / st;
+                double q;
+                if (zd_base) {
+                    vec_t zd = vec_at(zd_base, dtype, i, V);
+                    q = exp((zval(zd, v) - md) / T) / sd;
+                } else {
+                    q = (v == x[i]) ? 1.0 : 0.0;
+                }
+                r[v] = p - q > 0.0 ? p - q : 0.0;
+            }
+            break;
+        }
+        int fb = 0;
+        double mg = 0.0;
+        if (rejected) {
+            double R = 0.0;
+            for (int v = 0; v < V; ++v) R += r[v];
+            if (R == 0.0) {
+                /* p_j == q_j to rounding: the rejection had probability ~0.
+                 * Draw from p_j instead. */
+                vec_t zt = vec_at(zt_row.p, dtype, j, V);
+                for (int v = 0; v < V; ++v) r[v] = exp((zval(zt, v) - mt) / T) / st;
+                flags += 1.0;
+            }
+        } else {
+            /* Every draft survived: bonus draw from p_L. */
+            vec_t zt = vec_at(zt_row.p, dtype, L, V);
+            softmax_stats(zt, V, T, &mt, &st);
+            for (int v = 0; v < V; ++v) r[v] = exp((zval(zt, v) - mt) / T) / st;
+        }
+        Rfinal = 0.0;
+        for (int v = 0; v < V; ++v) Rfinal += r[v];
+        y = inverse_cdf(r, V, u_res[j], &mg, &fb);
+        if (fb) flags += 2.0;
+        d1 = mg;
+    }
+
+    for (int i = 0; i < j; ++i) out_tokens[i] = x[i];
+    out_tokens[j] = y;
+    for (int i = j + 1; i <= K; ++i) out_tokens[i] = -1;
+    if (diag) {
+        diag[0] = d0; diag[1] = d1; diag[2] = flags; diag[3] = (double)j; diag[4] = Rfinal;
+    }
+    return j;
+}
+
+/* Single row with fp64 logits and injected uniforms (for exact enumeration).
+ * zd may be NULL (greedy drafter).  Returns a; -1 on bad arguments. */
+int oracle_verify_row_u(const double *zt, const double *zd, int K, int V,
+                        const int32_t *x, int L, double T,
+                        const double *u_acc, const double *u_res,
+                        int32_t *out_tokens, double *diag)
+{
+    if (K < 0 || V <= 0 || L < 0 || L > K || !(T >= 0.0)) return -1;
+    for (int i = 0; i < L; ++i) if (x[i] < 0 || x[i] >= V) return -1;
+    double *work = (double *)malloc(sizeof(double) * (size_t)V);
+    if (!work) return -1;
+    vec_t zr = { zt, OR_F64 };
+    int a = verify_row(zr, zd, OR_F64, K, V, x, L, T, u_acc, u_res, out_tokens, diag, work);
+    free(work);
+    return a;
+}
+
+/* Data checks shared by the batch entry point: a row is invalid when its
+ * length is outside [0,K], its temperature is negative, NaN, infinite or in
+ * (0, 1e-6), or a draft token it verifies lies outside [0,V).  Returns the
+ * status bits (1 token, 2 length, 4 temperature). */
+static int row_errors(int K, int V, const int32_t *x, int L, float T)
+{
+    int bits = 0;
+    if (L < 0 || L > K) bits |= 2;
+    if (!(T >= 0.0f) || isinf(T) || (T > 0.0f && T < 1e-6f)) bits |= 4;
+    if (!(bits & 2))
+        for (int i = 0; i < L; ++i)
+            if (x[i] < 0 || x[i] >= V) { bits |= 1; break; }
+    return bits;
+}
+
+/*
+ * Batch verification with Philox-keyed uniforms.
+ *   zt [B, K+1, V], zd [B, K, V] (or NULL: greedy drafter), dtype OR_F32 or
+ *   OR_BF16; tokens [B, K]; lengths [B]; temperature [B]; the Philox row id
+ *   of local row b is row_ids[b] if row_ids is non-NULL, else row_base + b.
+ *   Outputs out_tokens [B, K+1], out_accept [B] (-1 and a row of -1 for an
+ *   invalid row), diag [B, OR_NDIAG] (nullable).  Returns the OR of the
+ *   status bits of all rows.  nthreads <= 0 uses the OpenMP default.
+ */
+int oracle_verify(const void *zt, const void *zd, int dtype, int64_t B, int K, int V,
+                  const int32_t *tokens, const int32_t *lengths, const float *temperature,
+                  uint64_t seed, int64_t row_base, const int64_t *row_ids,
+                  int32_t *out_tokens, int32_t *out_accept, double *diag, int nthreads)
+{
+    int status = 0;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+#pragma omp parallel reduction(| : status)
+    {
+        double *work = (double *)malloc(sizeof(double) * (size_t)V);
+        double *u_acc = (double *)malloc(sizeof(double) * (size_t)(K + 1));
+        double *u_res = (double *)malloc(sizeof(double) * (size_t)(K + 1));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t b = 0; b < B; ++b) {
+            const int32_t *x = tokens + b * K;
+            int L = lengths[b];
+            float T = temperature[b];
+            int32_t *ot = out_tokens + b * (K + 1);
+            double *dg = diag ? diag + b * OR_NDIAG : NULL;
+            int bits = row_errors(K, V, x, L, T);
+            if (bits) {
+                status |= bits;
+                out_accept[b] = -1;
+                for (int i = 0; i <= K; ++i) ot[i] = -1;
+                if (dg) for (int q = 0; q < OR_NDIAG; ++q) dg[q] = NAN;
+                continue;
+            }
+            uint64_t row = row_ids ? (uint64_t)row_ids[b] : (uint64_t)(row_base + b);
+            for (int i = 0; i <= K; ++i) {
+                u_acc[i] = oracle_uniform(seed, row, (uint32_t)i, 0);
+                u_res[i] = oracle_uniform(seed, row, (uint32_t)i, 1);
+            }
+            vec_t zr = vec_at(zt, dtype, b * (K + 1), V);
+            const void *zdr = zd ? vec_at(zd, dtype, b * K, V).p : NULL;
+            out_accept[b] = verify_row(zr, zdr, dtype, K, V, x, L, (double)T,
+                                       u_acc, u_res, ot, dg, work);
+        }
+        free(work); free(u_acc); free(u_res);
+    }
+    return status;
+}
+
+/* Normaliser export: for every vector of a [n, V] array, m and Sigma at the
+ * given per-vector temperature (T == 0: m only, Sigma = 1) and the argmax. */
+void oracle_stats_batch(const void *z, int dtype, int64_t n, int V, const float *T,
+                        double *m, double *sum, int32_t *amax, int nthreads)
+{
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t k = 0; k < n; ++k)
+        oracle_vector_stats(vec_at(z, dtype, k, V).p, dtype, V, (double)T[k],
+                            &m[k], &sum[k], &amax[k]);
+}
+
+/* ---------------------------------------------------------------------------
+ * Schedule [P1 "Verify smarter"; P2; P4 Ch.7 "Confidence-Scheduled
+ * Verification"; P5]: prefix survival S_i = prod_{j<=i} c_j along the block,
+ * verify length L = the largest i with S_i >= tau (S_0 = 1, so L = 0 when
+ * even the first draft falls below tau).  A NaN confidence counts as 0 and
+ * confidences are clamped to [0,1], which keeps S non-increasing.
+ * S_out [B,K] (nullable) receives S_1..S_K; the return value is the
+ * smallest |S_i - tau| over the block (for tie accounting).
+ * ------------------------------------------------------------------------- */
+double oracle_schedule(const float *conf, int64_t B, int K, double tau,
+                       int32_t *lengths, double *S_out)
+{
+    double closest = INFINITY;
+    for (int64_t b = 0; b < B; ++b) {
+        double S = 1.0;
+        int L = 0;
+        for (int i = 1; i <= K; ++i) {
+            double c = (double)conf[b * K + (i - 1)];
+            if (isnan(c)) c = 0.0;
+            if (c < 0.0) c = 0.0;
+            if (c > 1.0) c = 1.0;
+            S = S * c;
+            if (S_out) S_out[b * K + (i - 1)] = S;
+            if (fabs(S - tau) < closest) closest = fabs(S - tau);
+            if (S >= tau) L = i;
+        }
+        lengths[b] = L;
+    }
+    return closest;
+}
+
+int oracle_ndiag(void) { return OR_NDIAG; }
