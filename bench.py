@@ -1,0 +1,423 @@
+"""Benchmark: confidence-scheduled speculative verification on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload c2]
+
+One step = one pass of the whole hot path over one batch: the schedule
+(prefix survival -> verify lengths) and the verification (softmax statistics,
+accept test, correction/bonus draw), through the library's C ABI.  The
+default workload is the 256-row, 8-draft, 129280-token bf16 batch (per-row
+temperature from {0, 0.6, 1.0}, lengths from the schedule with
+conf ~ Beta(8,2), tau = 0.3).  Inputs are synthetic and seeded.
+
+Prints one JSON line (rank 0).  `value` is verified draft positions per
+second over all ranks (sum of the scheduled lengths per step / device time,
+max over ranks); `roofline` is the main verification kernel's algorithmic
+logit bytes per launch over its CUDA-event duration; `e2e` repeats the
+measurement with the inputs in pinned host memory and the host<->device
+copies inside the timed region; `cpu_baseline` is the fp64 CPU oracle on a
+bounded sample of the same workload.  `--impl reference` times the oracle
+alone (rank 0; other ranks exit).
+
+Multi-GPU (torchrun): rows are independent, so every rank verifies its own
+batch of B rows (Philox rows offset by rank * B) with no data-path
+collective; NCCL carries only the barrier and the max-over-ranks timing.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import speculative_decoding_verification_93_b200 as sv  # noqa: E402
+from speculative_decoding_verification_93_b200 import workloads  # noqa: E402
+
+METRIC = "verified draft positions/sec and achieved HBM GB/s (% of B200 peak) at B×K×V"
+UNIT = "positions/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["speculative_decoding_verification_93_b200/csrc/sv_verify.cu",
+                  "speculative_decoding_verification_93_b200/csrc/sv_device.cuh"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "verify_kernel_c2_traffic.md")
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def committed_traffic():
+    """DRAM bytes per launch of the main kernel from the committed ncu
+    summary, if it was taken on the current kernel source."""
+    try:
+        text = open(TRAFFIC_FILE).read()
+    except OSError:
+        return None
+    mh = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
+    mt = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not mh or not mt or mh.group(1) != kernel_hash():
+        return None
+    return float(mt.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi sampling during the timed region (clocks, throttle reasons)."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+def algorithmic_bytes(lengths: np.ndarray, temperature: np.ndarray, V: int, esize: int,
+                      has_draft: bool = True) -> int:
+    """Logit bytes the verification must stream once: per row
+    esize * V * ((L + 1) target vectors + L draft vectors if T > 0)."""
+    L = lengths.astype(np.int64)
+    drafts = np.where((temperature > 0) & has_draft, L, 0)
+    return int((esize * V * ((L + 1) + drafts)).sum())
+
+
+def oracle_sample(batch, lengths_np, budget_s: float, seed0: int = 0):
+    """Time the fp64 CPU oracle, as it stands, on whole passes over the batch
+    (one verification seed per pass) until ~budget_s of CPU time is spent."""
+    import oracle
+    from speculative_decoding_verification_93_b200.workloads import to_host_logits
+    zt = to_host_logits(batch.zt)
+    zd = to_host_logits(batch.zd)
+    tok = batch.tokens.cpu().numpy()
+    tmp = batch.temperature.cpu().numpy()
+    nthreads = oracle.default_threads()
+    positions, passes = 0, 0
+    t0 = time.perf_counter()
+    while True:
+        oracle.verify(zt, zd, tok, lengths_np, tmp, seed0 + passes, nthreads=nthreads)
+        passes += 1
+        positions += int(lengths_np.sum())
+        el = time.perf_counter() - t0
+        if el >= budget_s or passes >= 1000:
+            break
+    return dict(value=positions / el, unit=UNIT, cores=nthreads, kind="oracle",
+                sample=f"{passes} full pass(es) over the {batch.spec.B}-row batch "
+                       f"(seeds {seed0}..{seed0 + passes - 1}), {el:.1f} s wall, "
+                       f"OpenMP over rows")
+
+
+def workload_config(batch, lengths_np, esize):
+    s = batch.spec
+    dt = "bf16" if s.dtype == torch.bfloat16 else "fp32"
+    inputs = (batch.zt.numel() + batch.zd.numel()) * esize
+    return {"workload": (f"{s.name}: B={s.B} K={s.K} V={s.V} {dt} logits; "
+                         f"T per row from {list(s.temps)}; "
+                         + (f"lengths from sv_schedule (conf~Beta{s.beta}, tau={batch.tau})"
+                            if s.fixed_length is None else f"lengths={s.fixed_length}")),
+            "B": s.B, "K": s.K, "V": s.V, "logits": dt,
+            "mean_L": float(lengths_np.mean()),
+            "l2": f"inputs {inputs / 1e9:.2f} GB > 126 MB L2 (no flush)",
+            "data_seed": s.data_seed}
+
+
+def run_ours(args, rank, world, local_rank):
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+    batch = workloads.make_batch(args.workload, device=dev,
+                                 data_seed=workloads.SPECS[args.workload].data_seed + 1000 * rank)
+    s = batch.spec
+    B, K, V = s.B, s.K, s.V
+    esize = 2 if s.dtype == torch.bfloat16 else 4
+    dt = sv.SV_BF16 if esize == 2 else sv.SV_F32
+    ws = torch.empty(sv.sv_verify_workspace_bytes(B, K, V, dt), dtype=torch.uint8, device=dev)
+    out_tok = torch.empty(B, K + 1, dtype=torch.int32, device=dev)
+    out_acc = torch.empty(B, dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    lengths = torch.empty(B, dtype=torch.int32, device=dev)
+    row_base = rank * B
+    fixed = batch.lengths
+
+    def step(i, zt, zd, tokens, temp, conf, ln):
+        if fixed is None:
+            sv.sv_schedule(conf, batch.tau, ln)
+        sv.sv_verify(zt, zd, tokens, ln, temp, args.seed + i, out_tok, out_acc, ws,
+                     status=status, row_base=row_base)
+
+    ln_buf = lengths if fixed is None else fixed
+    for i in range(args.warmup):
+        step(i, batch.zt, batch.zd, batch.tokens, batch.temperature, batch.conf, ln_buf)
+    torch.cuda.synchronize()
+    lengths_np = ln_buf.cpu().numpy()
+    temp_np = batch.temperature.cpu().numpy()
+    positions = int(lengths_np.sum())
+    alg_bytes = algorithmic_bytes(lengths_np, temp_np, V, esize)
+
+    # ---- device-timed region ------------------------------------------------
+    clocks = ClockSampler(local_rank)
+    if rank == 0:
+        clocks.start()
+    sv.sv_profile_begin(args.steps)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i, batch.zt, batch.zd, batch.tokens, batch.temperature, batch.conf,
+             ln_buf)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    ms_total = e0.elapsed_time(e1)
+    kernel_ms = sv.sv_profile_read(args.steps)
+    sv.sv_profile_begin(0)
+    clk = clocks.stop() if rank == 0 else None
+    if dist:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    value = positions * world / (ms_step / 1e3)
+    st = int(status.item())
+
+    # ---- end-to-end through host buffers ------------------------------------
+    e2e = None
+    if not args.no_e2e:
+        host = {n: getattr(batch, n).cpu().pin_memory() for n in
+                ("zt", "zd", "tokens", "temperature", "conf")}
+        dzt = torch.empty_like(batch.zt)
+        dzd = torch.empty_like(batch.zd)
+        dtok = torch.empty_like(batch.tokens)
+        dtmp = torch.empty_like(batch.temperature)
+        dconf = torch.empty_like(batch.conf)
+        h_tok = torch.empty(B, K + 1, dtype=torch.int32).pin_memory()
+        h_acc = torch.empty(B, dtype=torch.int32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        if fixed is not None:
+            host["lengths"] = fixed.cpu().pin_memory()
+            h2d += host["lengths"].numel() * 4
+        d2h = h_tok.numel() * 4 + h_acc.numel() * 4
+        e2e_steps = max(1, min(args.steps, args.e2e_steps))
+
+        def e2e_step(i):
+            dzt.copy_(host["zt"], non_blocking=True)
+            dzd.copy_(host["zd"], non_blocking=True)
+            dtok.copy_(host["tokens"], non_blocking=True)
+            dtmp.copy_(host["temperature"], non_blocking=True)
+            dconf.copy_(host["conf"], non_blocking=True)
+            ln = ln_buf
+            if fixed is not None:
+                ln.copy_(host["lengths"], non_blocking=True)
+            step(i, dzt, dzd, dtok, dtmp, dconf, ln)
+            h_tok.copy_(out_tok, non_blocking=True)
+            h_acc.copy_(out_acc, non_blocking=True)
+
+        e2e_step(0)
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        e0.record(stream)
+        for i in range(e2e_steps):
+            e2e_step(i + 1)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms_e2e = e0.elapsed_time(e1)
+        if dist:
+            t = torch.tensor([ms_e2e], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        e2e = {"value": positions * world / (ms_e2e / e2e_steps / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": e2e_steps}
+        del host, dzt, dzd
+
+    # ---- roofline of the main kernel ----------------------------------------
+    peak, peak_src = measured_hbm_peak()
+    kms = [t for t in kernel_ms if t > 0]
+    avg_kernel_ms = sum(kms) / len(kms) if kms else float("nan")
+    achieved = alg_bytes / (avg_kernel_ms / 1e3) / 1e9
+    traffic = committed_traffic()
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src ==
+                "measured" else "fallback 6650 GB/s",
+                "kernel": "sv::verify_kernel", "kernel_ms": round(avg_kernel_ms, 5),
+                "algorithmic_bytes_per_launch": alg_bytes,
+                "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+                "step_gbs": round(alg_bytes / (ms_step / 1e3) / 1e9, 1)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = oracle_sample(batch, lengths_np, args.cpu_seconds)
+
+    if rank == 0:
+        out = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+               "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+               "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+               "dtype": "f32", "data": "synthetic",
+               "config": dict(workload_config(batch, lengths_np, esize),
+                              parallelism=f"dp{world} (row shards, no collective)"),
+               "e2e": e2e, "gpu_launches": args.steps * (sv.sv_verify_launches()
+                                                         + (1 if fixed is None else 0)),
+               "roofline": roofline, "cpu_baseline": cpu, "clocks": clk,
+               "device_status": st, "impl": "ours"}
+        print(json.dumps(out), flush=True)
+    del batch
+    if dist:
+        dist.barrier()
+
+
+def run_reference(args, rank, world):
+    """The oracle (fp64 CPU) timed as it stands on the host cores: each step is
+    one bounded pass over a row sample of the same workload."""
+    if rank != 0:
+        return
+    batch = workloads.make_batch(args.workload, device="cpu")
+    s = batch.spec
+    import oracle
+    from speculative_decoding_verification_93_b200.workloads import to_host_logits
+    if batch.lengths is None:
+        lengths_np, _, _ = oracle.schedule(batch.conf.numpy(), batch.tau)
+    else:
+        lengths_np = batch.lengths.numpy()
+    rows = np.arange(min(s.B, args.ref_rows))
+    zt = to_host_logits(batch.zt[: len(rows)])
+    zd = to_host_logits(batch.zd[: len(rows)])
+    tok = batch.tokens[: len(rows)].numpy()
+    tmp = batch.temperature[: len(rows)].numpy()
+    ln = lengths_np[: len(rows)]
+    nthreads = oracle.default_threads()
+    for i in range(args.warmup):
+        oracle.verify(zt, zd, tok, ln, tmp, args.seed + i, nthreads=nthreads)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle.schedule(batch.conf[: len(rows)].numpy(), batch.tau)
+        oracle.verify(zt, zd, tok, ln, tmp, args.seed + args.warmup + i, nthreads=nthreads)
+    el = time.perf_counter() - t0
+    positions = int(ln.sum())
+    value = positions * args.steps / el
+    esize = 2 if s.dtype == torch.bfloat16 else 4
+    sample = f"rows 0..{len(rows) - 1} of the {s.B}-row batch per step"
+    out = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": dict(workload_config(batch, lengths_np, esize),
+                          parallelism="host cores (OpenMP over rows)"),
+           "impl": "reference",
+           "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": nthreads,
+                            "kind": "oracle", "sample": sample},
+           "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="c2", choices=sorted(workloads.SPECS))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-rows", type=int, default=64)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,231 @@
+/*
+ * sv.h -- C ABI of the B200 (sm_100a) speculative-verification library.
+ *
+ * The library implements the data-parallel hot path of confidence-scheduled
+ * speculative decoding: the per-row verify length from the drafter's
+ * survival confidences (sv_schedule) and batched draft verification by
+ * speculative rejection sampling (sv_verify).
+ *
+ * Conventions for every entry point:
+ *  - Pointers named as device pointers must be CUDA device memory (or
+ *    managed memory) owned by the caller.  The library never allocates
+ *    device memory, never frees caller memory and never synchronises the
+ *    stream; all work is enqueued on `stream` (a cudaStream_t passed as
+ *    void*, NULL = legacy default stream) and completes asynchronously.
+ *  - Argument errors are detected on the host before anything is launched
+ *    and returned synchronously; nothing is written in that case.
+ *  - Data errors that can only be seen on the device never fault or trap:
+ *    the affected row is marked in the outputs and a bit is OR-ed into the
+ *    optional device status word.
+ *  - Row-major layouts; the vocabulary index is the contiguous one.
+ *
+ * Sources are cited as page title + section.  The pages describe the method
+ * in words; the symbolic rule implemented here is the standard
+ * speculative-sampling rule that their words describe.
+ */
+#ifndef SV_H
+#define SV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SV_OK = 0,
+    SV_ERR_ARG = 1,        /* null pointer, negative size, bad seed/row base, misaligned pointer */
+    SV_ERR_SHAPE = 2,      /* B, K or V out of the supported range */
+    SV_ERR_DTYPE = 3,      /* unknown logit dtype */
+    SV_ERR_WORKSPACE = 4,  /* workspace smaller than sv_verify_workspace_bytes() */
+    SV_ERR_CUDA = 5        /* a CUDA launch or query failed (see sv_last_cuda_error) */
+} sv_status;
+
+typedef enum { SV_F32 = 0, SV_BF16 = 1 } sv_dtype;
+
+/* Bits OR-ed into the optional device status word by sv_verify. */
+#define SV_ROW_BAD_TOKEN        1   /* a verified draft token lies outside [0, V) */
+#define SV_ROW_BAD_LENGTH       2   /* lengths[b] outside [0, K] */
+#define SV_ROW_BAD_TEMPERATURE  4   /* T < 0, NaN, inf, or 0 < T < 1e-6 */
+#define SV_NOTE_ZERO_RESIDUAL   8   /* informational: a rejection left zero residual mass (drew from p_j) */
+#define SV_NOTE_CDF_FALLBACK   16   /* informational: rounding put the CDF target past the total */
+
+/* Supported sizes. */
+#define SV_MAX_K  64
+#define SV_MAX_V  (1 << 28)
+
+/*
+ * sv_schedule -- per-row verify length from prefix survival.
+ *
+ * Defined by: umans.ai, "DeepSeek V4 Pro DSpark: the model isn't ready, the
+ * architecture is", section "What DSpark adds", item "2. Verify smarter"
+ * (a confidence head gives, per draft position, the probability that the
+ * token survives given that every earlier one survived; multiplying along the
+ * block gives the survival probability of every prefix length); aiweekly.co
+ * alert (verify length from estimated prefix survival and system load);
+ * en.5iter.com article, section "What DSpark changed is how to generate a
+ * draft", and techvisionai "DeepSeek-V4: Breaking the Efficiency Barrier",
+ * Ch. 7 "Confidence-Scheduled Verification" (verify longer when idle, only
+ * the confident prefix when busy).
+ *
+ * Computes, per row b, S_i = prod_{j<=i} clamp(conf[b, j-1], 0, 1) (NaN
+ * counts as 0) for i = 1..K, left to right in fp32, and
+ * lengths[b] = max{ i in 0..K : S_i >= load } with S_0 = 1.  `load` is the
+ * load-dependent threshold tau (larger under heavier load).
+ *
+ *   conf     device, float32 [B, K], read only.
+ *   B, K     rows and drafts per row; B >= 1, 1 <= K <= SV_MAX_K.
+ *   load     threshold tau; any float (tau <= 0 keeps every draft, tau > 1
+ *            keeps none, NaN keeps none).
+ *   lengths  device, int32 [B], written.
+ * Returns SV_OK, SV_ERR_ARG (null pointer), SV_ERR_SHAPE, or SV_ERR_CUDA.
+ *
+ * The confidences must be causal with respect to this step's sampling (the
+ * umans.ai page sizes the truncation from confidences measured two steps
+ * earlier); that is the caller's contract, not checked here.
+ */
+sv_status sv_schedule(const float *conf, int B, int K, float load,
+                      int32_t *lengths, void *stream);
+
+/*
+ * sv_verify_workspace_bytes -- device scratch that sv_verify needs for
+ * (B, K, V, dtype): per-row work counters, per-row work offsets and the
+ * per-chunk softmax partials.  Returns 0 for unsupported sizes.
+ */
+size_t sv_verify_workspace_bytes(int B, int K, int V, sv_dtype dtype);
+
+/*
+ * sv_verify -- batched speculative verification.
+ *
+ * Defined by: umans.ai page above, section "Speculative decoding, briefly"
+ * (the target verifies the whole draft block in one pass, accepts the prefix
+ * it agrees with plus a bonus token of its own, and discards the rest; the
+ * acceptance rule is rejection sampling under which accepted tokens follow
+ * the target distribution exactly, and a rejected token is replaced by one
+ * the target would produce); zhichai.net DSpark topic, section "Why LLMs
+ * speak so slowly" (rejection sampling on the target/draft probability
+ * ratio; generation restarts from the first error).  In symbols, per row b
+ * with verify length L = lengths[b] and temperature T = temperature[b]:
+ *
+ *   p_i = softmax(zt[b, i, :] / T),  q_i = softmax(zd[b, i, :] / T);
+ *   for i = 0..L-1: accept x_i = draft_tokens[b, i] iff
+ *       u(seed, row, i, 0) < min(1, p_i(x_i) / q_i(x_i));
+ *   j = first rejected i, or L if all survive;
+ *   y drawn by inverse CDF, in token order, with u(seed, row, j, 1) from
+ *       max(0, p_j - q_j) (j < L) or p_L (j == L): the smallest v whose
+ *       cumulative weight exceeds u * (total weight);
+ *   out_tokens[b] = x_0 .. x_{j-1}, y, then -1;  out_accept_len[b] = j.
+ *   T == 0 is greedy verification: accept while x_i equals the target argmax
+ *   (lowest index on ties), y = target argmax at j; no uniforms are drawn and
+ *   the draft logits are not read.
+ *   draft_logits == NULL selects a greedy drafter (q_i one-hot at x_i, the
+ *   techvisionai page, Ch. 7 "Deployment with vLLM", draft_sample_method
+ *   greedy): accept with probability p_i(x_i), resample from p_j with x_j
+ *   removed.
+ *
+ * u(seed, row, pos, draw) = (w0 >> 8) * 2^-24 where w0 is word 0 of
+ * Philox4x32-10 (Salmon et al., SC'11) with key (seed_lo, seed_hi) and
+ * counter (row_lo, pos, draw, row_hi); row = row_base + b, so that shards of
+ * one batch verified separately with their row offsets reproduce the
+ * unsharded result.  Change `seed` every decoding step.
+ *
+ *   target_logits  device [B, K+1, V] of `dtype`; read only.  Positions
+ *                  i > L of row b are never read.
+ *   draft_logits   device [B, K, V] of `dtype`, or NULL (greedy drafter);
+ *                  read only; positions i >= L and rows with T == 0 are
+ *                  never read.
+ *   dtype          SV_F32 or SV_BF16; both logit arrays share it.  Logits
+ *                  must be finite or -inf, with at least one finite logit
+ *                  per vector that is read.
+ *   B, K, V        1 <= B, 1 <= K <= SV_MAX_K, 1 <= V <= SV_MAX_V.
+ *   draft_tokens   device int32 [B, K]; entries i >= L are ignored.
+ *   lengths        device int32 [B] (e.g. the output of sv_schedule).
+ *   temperature    device float32 [B].
+ *   seed           Philox key.
+ *   row_base       Philox row id of local row 0 (>= 0).
+ *   out_tokens     device int32 [B, K+1], written.
+ *   out_accept_len device int32 [B], written; -1 for an invalid row.
+ *   workspace      device, >= sv_verify_workspace_bytes(B, K, V, dtype)
+ *                  bytes, 16-byte aligned; scratch owned by the caller,
+ *                  contents need not be initialised and are undefined
+ *                  afterwards.  Calls that share a workspace must be
+ *                  stream-ordered.
+ *   status         device int32, nullable; SV_ROW_* and SV_NOTE_* bits are
+ *                  OR-ed in (the library never clears it).
+ * Logit pointers must be aligned to their element size; any 16-byte
+ * misalignment of individual vectors is handled.
+ * Returns SV_OK, SV_ERR_ARG, SV_ERR_SHAPE, SV_ERR_DTYPE, SV_ERR_WORKSPACE or
+ * SV_ERR_CUDA.  An invalid row (bad length, temperature or token) gets
+ * out_accept_len = -1 and a row of -1 in out_tokens; other rows are
+ * unaffected.
+ */
+sv_status sv_verify(const void *target_logits, const void *draft_logits, sv_dtype dtype,
+                    int B, int K, int V,
+                    const int32_t *draft_tokens, const int32_t *lengths,
+                    const float *temperature, uint64_t seed, int64_t row_base,
+                    int32_t *out_tokens, int32_t *out_accept_len,
+                    void *workspace, size_t workspace_bytes, int32_t *status,
+                    void *stream);
+
+/*
+ * sv_verify_debug -- sv_verify plus an export of the softmax normalisers it
+ * computed: stats_out (device float32 [B, 2K+1, 2]) receives, for every
+ * vector the call read, (m, Sigma) with m = max_v z_v and
+ * Sigma = sum_v exp((z_v - m) / T) (Sigma = 1 at T == 0).  Slot i <= K is
+ * target position i, slot K+1+i is draft position i.  Slots that were not
+ * read are left untouched.  For tests and diagnostics.
+ */
+sv_status sv_verify_debug(const void *target_logits, const void *draft_logits, sv_dtype dtype,
+                          int B, int K, int V,
+                          const int32_t *draft_tokens, const int32_t *lengths,
+                          const float *temperature, uint64_t seed, int64_t row_base,
+                          int32_t *out_tokens, int32_t *out_accept_len,
+                          void *workspace, size_t workspace_bytes, int32_t *status,
+                          float *stats_out, void *stream);
+
+/*
+ * sv_philox_uniforms -- the uniforms sv_verify draws, for tests:
+ * out[k] = u(seed, row[k], pos[k], draw[k]) as defined above.
+ * row: device int64 [n] (>= 0); pos, draw: device int32 [n]; out: device
+ * float32 [n].  n >= 0.
+ */
+sv_status sv_philox_uniforms(uint64_t seed, const int64_t *row, const int32_t *pos,
+                             const int32_t *draw, int n, float *out, void *stream);
+
+/*
+ * sv_philox4x32_10 -- raw Philox4x32-10 blocks (Salmon et al., SC'11), for
+ * tests: out[4k..4k+3] = Philox(ctr[4k..4k+3], key[2k..2k+1]).
+ * ctr, out: device uint32 [n, 4]; key: device uint32 [n, 2].
+ */
+sv_status sv_philox4x32_10(const uint32_t *ctr, const uint32_t *key, int n, uint32_t *out,
+                           void *stream);
+
+/*
+ * Profiling hooks (benchmark use).  sv_profile_begin(capacity) makes the
+ * next `capacity` sv_verify calls on this process record CUDA events around
+ * their main verification kernel (capacity <= 0 disables recording).
+ * sv_profile_read(ms, max) waits for those events and writes up to `max`
+ * per-launch durations in milliseconds; returns how many were recorded.
+ * Not thread-safe.
+ */
+sv_status sv_profile_begin(int capacity);
+int sv_profile_read(float *ms, int max);
+
+/* Number of CUDA kernels one sv_verify call launches. */
+int sv_verify_launches(void);
+
+/* Human-readable status name; never NULL. */
+const char *sv_status_string(sv_status s);
+
+/* The last CUDA error code seen by the calling thread (0 if none). */
+int sv_last_cuda_error(void);
+
+/* Library ABI version. */
+int sv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SV_H */

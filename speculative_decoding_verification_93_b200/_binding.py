@@ -1,0 +1,195 @@
+"""ctypes binding of the C ABI in ``include/sv.h`` (same names, same
+arguments).  Tensors are passed by device pointer; the stream defaults to
+PyTorch's current stream on the tensors' device."""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+SV_F32, SV_BF16 = 0, 1
+SV_ROW_BAD_TOKEN, SV_ROW_BAD_LENGTH, SV_ROW_BAD_TEMPERATURE = 1, 2, 4
+SV_NOTE_ZERO_RESIDUAL, SV_NOTE_CDF_FALLBACK = 8, 16
+_STATUS = {0: "SV_OK", 1: "SV_ERR_ARG", 2: "SV_ERR_SHAPE", 3: "SV_ERR_DTYPE",
+           4: "SV_ERR_WORKSPACE", 5: "SV_ERR_CUDA"}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libsv.so")
+_lib = None
+
+
+class SVError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        extra = ""
+        if code == 5 and _lib is not None:
+            extra = f" (cuda error {_lib.sv_last_cuda_error()})"
+        super().__init__(f"{fn} failed: {_STATUS.get(code, code)}{extra}")
+        self.code = code
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib():
+    """Load ``libsv.so``; raises if it is missing (no fallback exists)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"{_LIB_PATH} is missing: build it with "
+                          "`python -m speculative_decoding_verification_93_b200.build`")
+    L = ctypes.CDLL(_LIB_PATH)
+    vp, i32, i64, u64, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64,
+                             ctypes.c_size_t)
+    L.sv_schedule.argtypes = [vp, i32, i32, ctypes.c_float, vp, vp]
+    L.sv_verify_workspace_bytes.argtypes = [i32, i32, i32, i32]
+    L.sv_verify_workspace_bytes.restype = sz
+    L.sv_verify.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, u64, i64, vp, vp, vp, sz, vp,
+                            vp]
+    L.sv_verify_debug.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, u64, i64, vp, vp, vp,
+                                  sz, vp, vp, vp]
+    L.sv_philox_uniforms.argtypes = [u64, vp, vp, vp, i32, vp, vp]
+    L.sv_philox4x32_10.argtypes = [vp, vp, i32, vp, vp]
+    L.sv_profile_begin.argtypes = [i32]
+    L.sv_profile_read.argtypes = [vp, i32]
+    L.sv_profile_read.restype = i32
+    L.sv_status_string.argtypes = [i32]
+    L.sv_status_string.restype = ctypes.c_char_p
+    for name in ("sv_schedule", "sv_verify", "sv_verify_debug", "sv_philox_uniforms",
+                 "sv_philox4x32_10", "sv_profile_begin"):
+        getattr(L, name).restype = i32
+    L.sv_last_cuda_error.restype = i32
+    L.sv_version.restype = i32
+    L.sv_verify_launches.restype = i32
+    _lib = L
+    return L
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, like: torch.Tensor):
+    if stream is None:
+        stream = torch.cuda.current_stream(like.device)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise SVError(fn, code)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return SV_F32
+    if t.dtype == torch.bfloat16:
+        return SV_BF16
+    raise TypeError(f"logits must be float32 or bfloat16, got {t.dtype}")
+
+
+def _need(t: torch.Tensor, dtype, name: str):
+    if t.dtype != dtype or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous {dtype} tensor")
+
+
+def sv_schedule(conf: torch.Tensor, load: float, lengths: torch.Tensor, stream=None) -> None:
+    _need(conf, torch.float32, "conf")
+    _need(lengths, torch.int32, "lengths")
+    B, K = conf.shape
+    _check("sv_schedule", lib().sv_schedule(_ptr(conf), B, K, float(load), _ptr(lengths),
+                                            _stream(stream, conf)))
+
+
+def sv_verify_workspace_bytes(B: int, K: int, V: int, dtype: int) -> int:
+    return int(lib().sv_verify_workspace_bytes(B, K, V, dtype))
+
+
+def _verify_args(target_logits, draft_logits, draft_tokens, lengths, temperature):
+    B, K1, V = target_logits.shape
+    K = K1 - 1
+    dt = _dtype(target_logits)
+    if not target_logits.is_contiguous():
+        raise TypeError("target_logits must be contiguous")
+    if draft_logits is not None and (draft_logits.dtype != target_logits.dtype
+                                     or not draft_logits.is_contiguous()
+                                     or tuple(draft_logits.shape) != (B, K, V)):
+        raise TypeError("draft_logits must be a contiguous [B, K, V] tensor of the target dtype")
+    _need(draft_tokens, torch.int32, "draft_tokens")
+    _need(lengths, torch.int32, "lengths")
+    _need(temperature, torch.float32, "temperature")
+    return B, K, V, dt
+
+
+def sv_verify(target_logits, draft_logits, draft_tokens, lengths, temperature, seed: int,
+              out_tokens, out_accept_len, workspace, status=None, row_base: int = 0,
+              stream=None) -> None:
+    B, K, V, dt = _verify_args(target_logits, draft_logits, draft_tokens, lengths, temperature)
+    _check("sv_verify", lib().sv_verify(
+        _ptr(target_logits), _ptr(draft_logits), dt, B, K, V, _ptr(draft_tokens), _ptr(lengths),
+        _ptr(temperature), ctypes.c_uint64(seed & (2**64 - 1)), int(row_base), _ptr(out_tokens),
+        _ptr(out_accept_len), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _ptr(status), _stream(stream, target_logits)))
+
+
+def sv_verify_debug(target_logits, draft_logits, draft_tokens, lengths, temperature, seed: int,
+                    out_tokens, out_accept_len, workspace, stats_out, status=None,
+                    row_base: int = 0, stream=None) -> None:
+    B, K, V, dt = _verify_args(target_logits, draft_logits, draft_tokens, lengths, temperature)
+    _check("sv_verify_debug", lib().sv_verify_debug(
+        _ptr(target_logits), _ptr(draft_logits), dt, B, K, V, _ptr(draft_tokens), _ptr(lengths),
+        _ptr(temperature), ctypes.c_uint64(seed & (2**64 - 1)), int(row_base), _ptr(out_tokens),
+        _ptr(out_accept_len), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _ptr(status), _ptr(stats_out), _stream(stream, target_logits)))
+
+
+def sv_philox_uniforms(seed: int, row, pos, draw, out, stream=None) -> None:
+    n = out.numel()
+    _check("sv_philox_uniforms", lib().sv_philox_uniforms(
+        ctypes.c_uint64(seed & (2**64 - 1)), _ptr(row), _ptr(pos), _ptr(draw), n, _ptr(out),
+        _stream(stream, out)))
+
+
+def sv_philox4x32_10(ctr, key, out, stream=None) -> None:
+    n = out.numel() // 4
+    _check("sv_philox4x32_10", lib().sv_philox4x32_10(_ptr(ctr), _ptr(key), n, _ptr(out),
+                                                      _stream(stream, out)))
+
+
+def sv_profile_begin(capacity: int) -> None:
+    _check("sv_profile_begin", lib().sv_profile_begin(int(capacity)))
+
+
+def sv_profile_read(max_n: int = 4096):
+    buf = (ctypes.c_float * max_n)()
+    n = lib().sv_profile_read(ctypes.cast(buf, ctypes.c_void_p), max_n)
+    return [buf[i] for i in range(n)]
+
+
+def sv_verify_launches() -> int:
+    return int(lib().sv_verify_launches())
+
+
+def sv_status_string(code: int) -> str:
+    return lib().sv_status_string(int(code)).decode()
+
+
+def verify(target_logits, draft_logits, draft_tokens, lengths, temperature, seed: int,
+           row_base: int = 0, workspace=None, status=None, stream=None):
+    """Allocate the outputs (and workspace, if not given) with PyTorch and call
+    :func:`sv_verify`.  Returns (out_tokens [B, K+1], out_accept_len [B])."""
+    B, K1, V = target_logits.shape
+    dev = target_logits.device
+    out_tokens = torch.empty(B, K1, dtype=torch.int32, device=dev)
+    out_acc = torch.empty(B, dtype=torch.int32, device=dev)
+    if workspace is None:
+        n = sv_verify_workspace_bytes(B, K1 - 1, V, _dtype(target_logits))
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=dev)
+    sv_verify(target_logits, draft_logits, draft_tokens, lengths, temperature, seed, out_tokens,
+              out_acc, workspace, status=status, row_base=row_base, stream=stream)
+    return out_tokens, out_acc

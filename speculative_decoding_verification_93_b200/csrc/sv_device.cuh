@@ -1,0 +1,172 @@
+// sv_device.cuh -- device helpers for the verification kernels (sm_100a).
+//
+// Philox4x32-10 follows Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers:
+// As Easy as 1, 2, 3" (SC'11): each round multiplies the two even words by the
+// round multipliers, XORs the high halves with the odd words and the key,
+// keeps the low halves, permutes the words, and bumps the key by the Weyl
+// constants.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace sv {
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10 and the verification uniforms.
+// ---------------------------------------------------------------------------
+struct Philox4 { uint32_t w[4]; };
+
+__device__ __forceinline__ Philox4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2,
+                                                 uint32_t c3, uint32_t k0, uint32_t k1) {
+    constexpr uint32_t kMulA = 0xD2511F53u, kMulB = 0xCD9E8D57u;
+    constexpr uint32_t kWeylA = 0x9E3779B9u, kWeylB = 0xBB67AE85u;
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        const uint32_t hiA = __umulhi(kMulA, c0), loA = kMulA * c0;
+        const uint32_t hiB = __umulhi(kMulB, c2), loB = kMulB * c2;
+        const uint32_t n0 = hiB ^ c1 ^ k0;
+        const uint32_t n2 = hiA ^ c3 ^ k1;
+        c0 = n0; c1 = loB; c2 = n2; c3 = loA;
+        k0 += kWeylA; k1 += kWeylB;
+    }
+    Philox4 o;
+    o.w[0] = c0; o.w[1] = c1; o.w[2] = c2; o.w[3] = c3;
+    return o;
+}
+
+// u(seed, row, pos, draw): top 24 bits of word 0 of the block for counter
+// (row_lo, pos, draw, row_hi) under key (seed_lo, seed_hi); exact in fp32.
+__device__ __forceinline__ float uniform24(uint64_t seed, uint64_t row, uint32_t pos,
+                                           uint32_t draw) {
+    const Philox4 o = philox4x32_10(static_cast<uint32_t>(row), pos, draw,
+                                    static_cast<uint32_t>(row >> 32),
+                                    static_cast<uint32_t>(seed),
+                                    static_cast<uint32_t>(seed >> 32));
+    return static_cast<float>(o.w[0] >> 8) * (1.0f / 16777216.0f);
+}
+
+// ---------------------------------------------------------------------------
+// Arithmetic.
+// ---------------------------------------------------------------------------
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kNegInf = -__builtin_huge_valf();
+
+// 2^x on the special-function unit (ex2.approx, flush-to-zero); 2^-inf = 0.
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Widen the two bf16 halves of a 32-bit word to fp32 (exact).  The element
+// at the lower address is the low half.
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
+    __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162 *>(&a);
+    __nv_bfloat162 y = *reinterpret_cast<__nv_bfloat162 *>(&b);
+    __nv_bfloat162 r = __hmax2(x, y);
+    return *reinterpret_cast<uint32_t *>(&r);
+}
+
+// Combine two (max, sum) online-softmax partials taken at scale k = log2e/T:
+// sum is relative to its own max.  A partial with max -inf has sum 0.
+__device__ __forceinline__ void lse_merge(float &m, float &s, float m2, float s2, float k) {
+    const float mn = fmaxf(m, m2);
+    if (mn == kNegInf) { m = mn; s = 0.f; return; }
+    s = s * ex2((m - mn) * k) + s2 * ex2((m2 - mn) * k);
+    m = mn;
+}
+
+// ---------------------------------------------------------------------------
+// Memory.
+// ---------------------------------------------------------------------------
+// Streaming 16-byte load: read-only, not kept in L1 (the pass touches every
+// byte once).
+__device__ __forceinline__ uint4 ld_stream(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// 16-byte load that may be cached (re-reads of recently streamed rows).
+__device__ __forceinline__ uint4 ld_reuse(const void *p) {
+    return __ldg(reinterpret_cast<const uint4 *>(p));
+}
+
+// Geometry of one logit vector of V elements split into a head (elements
+// before the first 16-byte boundary), n16 full 16-byte units, and a tail.
+struct VecGeom {
+    const char *base;   // element 0
+    const char *body;   // first 16-byte aligned byte (base + head * esize)
+    int head;
+    int n16;
+    int tail;
+};
+
+template <int ESIZE>
+__device__ __forceinline__ VecGeom vec_geom(const void *base, int V) {
+    constexpr int kPer = 16 / ESIZE;
+    VecGeom g;
+    g.base = static_cast<const char *>(base);
+    const uint32_t mis = static_cast<uint32_t>(reinterpret_cast<uintptr_t>(base) & 15u);
+    int h = mis ? static_cast<int>((16u - mis) / ESIZE) : 0;
+    if (h > V) h = V;
+    g.head = h;
+    g.body = g.base + h * ESIZE;
+    g.n16 = (V - h) / kPer;
+    g.tail = V - h - g.n16 * kPer;
+    return g;
+}
+
+// Scalar element load widened to fp32.
+template <int ESIZE>
+__device__ __forceinline__ float ld_elem(const char *base, long long v) {
+    if (ESIZE == 4) return __ldg(reinterpret_cast<const float *>(base) + v);
+    const unsigned short h = __ldg(reinterpret_cast<const unsigned short *>(base) + v);
+    return __uint_as_float(static_cast<uint32_t>(h) << 16);
+}
+
+// Element value pattern for padding: -inf in both dtypes.
+template <int ESIZE> __device__ __forceinline__ uint32_t neg_inf_word();
+template <> __device__ __forceinline__ uint32_t neg_inf_word<4>() { return 0xff800000u; }
+template <> __device__ __forceinline__ uint32_t neg_inf_word<2>() { return 0xff80ff80u; }
+
+// A partial unit (head or tail): up to 16/ESIZE elements starting at element
+// `first`, padded with -inf, packed like a body unit.
+template <int ESIZE>
+__device__ __forceinline__ uint4 ld_partial_unit(const char *base, int first, int count) {
+    uint32_t w[4];
+    const uint32_t pad = neg_inf_word<ESIZE>();
+    w[0] = w[1] = w[2] = w[3] = pad;
+    if (ESIZE == 4) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            if (e < count) w[e] = __float_as_uint(ld_elem<4>(base, first + e));
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            if (e < count) {
+                const uint32_t h = __float_as_uint(ld_elem<2>(base, first + e)) >> 16;
+                w[e >> 1] = (e & 1) ? ((w[e >> 1] & 0x0000ffffu) | (h << 16))
+                                    : ((w[e >> 1] & 0xffff0000u) | h);
+            }
+        }
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Element e (0 .. 16/ESIZE-1) of a packed unit, widened to fp32.
+template <int ESIZE>
+__device__ __forceinline__ float unit_elem(const uint4 &u, int e) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    if (ESIZE == 4) return __uint_as_float(w[e]);
+    return (e & 1) ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]);
+}
+
+}  // namespace sv

@@ -1,0 +1,98 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function that ``include/sv.h`` declares, sizes its workspace, and
+rejects bad arguments synchronously, before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import speculative_decoding_verification_93_b200 as sv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sv.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sv_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = sv.lib()
+    names = declared_functions()
+    assert "sv_verify" in names and "sv_schedule" in names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings_and_version():
+    assert sv.sv_status_string(0) == "SV_OK"
+    assert sv.sv_status_string(4) == "SV_ERR_WORKSPACE"
+    assert sv.sv_status_string(99) == "SV_UNKNOWN"
+    assert sv.lib().sv_version() >= 1
+    assert sv.sv_verify_launches() == 2
+
+
+def test_workspace_bytes():
+    n = sv.sv_verify_workspace_bytes(256, 8, 129280, sv.SV_BF16)
+    # counters + row counters + row offsets + partials (B * (2K+1) * C float4)
+    assert n >= 256 * 17 * 4 * 16
+    assert n < 2 * 1024 * 1024
+    assert sv.sv_verify_workspace_bytes(0, 8, 100, sv.SV_F32) == 0
+    assert sv.sv_verify_workspace_bytes(4, 0, 100, sv.SV_F32) == 0
+    assert sv.sv_verify_workspace_bytes(4, 65, 100, sv.SV_F32) == 0
+    assert sv.sv_verify_workspace_bytes(4, 4, 0, sv.SV_F32) == 0
+    assert sv.sv_verify_workspace_bytes(4, 4, 100, 7) == 0
+    # fp32 needs twice the chunks of bf16 at the same V
+    a = sv.sv_verify_workspace_bytes(64, 4, 129280, sv.SV_F32)
+    b = sv.sv_verify_workspace_bytes(64, 4, 129280, sv.SV_BF16)
+    assert a > b
+
+
+def _call_verify(**kw):
+    L = sv.lib()
+    args = dict(zt=1 << 20, zd=1 << 21, dtype=sv.SV_BF16, B=4, K=4, V=1000, tok=1 << 22,
+                ln=1 << 23, temp=1 << 24, seed=0, row_base=0, ot=1 << 25, oa=1 << 26,
+                ws=1 << 27, wsb=1 << 30, status=None, stream=None)
+    args.update(kw)
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return L.sv_verify(v(args["zt"]), v(args["zd"]), args["dtype"], args["B"], args["K"],
+                       args["V"], v(args["tok"]), v(args["ln"]), v(args["temp"]),
+                       ctypes.c_uint64(args["seed"]), args["row_base"], v(args["ot"]),
+                       v(args["oa"]), v(args["ws"]), args["wsb"], v(args["status"]),
+                       v(args["stream"]))
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(zt=None), 1), (dict(tok=None), 1), (dict(ln=None), 1), (dict(temp=None), 1),
+    (dict(ot=None), 1), (dict(oa=None), 1), (dict(ws=None), 1),
+    (dict(dtype=5), 3), (dict(B=0), 2), (dict(K=0), 2), (dict(K=65), 2), (dict(V=0), 2),
+    (dict(row_base=-1), 1), (dict(zt=(1 << 20) + 1), 1), (dict(ws=(1 << 27) + 8), 1),
+    (dict(wsb=16), 4),
+])
+def test_verify_rejects_bad_arguments_on_host(kw, code):
+    assert _call_verify(**kw) == code
+
+
+def test_schedule_and_philox_reject_bad_arguments_on_host():
+    L = sv.lib()
+    p = ctypes.c_void_p(1 << 20)
+    assert L.sv_schedule(None, 4, 4, ctypes.c_float(0.3), p, None) == 1
+    assert L.sv_schedule(p, 0, 4, ctypes.c_float(0.3), p, None) == 2
+    assert L.sv_schedule(p, 4, 65, ctypes.c_float(0.3), p, None) == 2
+    assert L.sv_philox_uniforms(ctypes.c_uint64(0), None, p, p, 4, p, None) == 1
+    assert L.sv_philox_uniforms(ctypes.c_uint64(0), p, p, p, -1, p, None) == 2
+    assert L.sv_philox_uniforms(ctypes.c_uint64(0), None, None, None, 0, None, None) == 0
+    assert L.sv_philox4x32_10(None, p, 3, p, None) == 1
+    assert L.sv_verify_debug(p, p, 1, 4, 4, 10, p, p, p, ctypes.c_uint64(0), 0, p, p, p,
+                             1 << 20, None, None, None) == 1
+
+
+def test_python_binding_marshals_only():
+    import torch
+    zt = torch.zeros(2, 3, 5)
+    with pytest.raises(TypeError):
+        sv.sv_verify(zt.double(), None, torch.zeros(2, 2, dtype=torch.int32),
+                     torch.zeros(2, dtype=torch.int32), torch.zeros(2), 0, None, None, None)

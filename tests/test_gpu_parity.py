@@ -1,0 +1,171 @@
+"""GPU vs oracle parity of sv_verify through the C ABI on small and ragged
+cases, normalisers, the greedy drafter, edge cases, sharding and
+determinism."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import speculative_decoding_verification_93_b200 as sv
+from speculative_decoding_verification_93_b200 import workloads
+from speculative_decoding_verification_93_b200.workloads import to_host_logits
+from _parity import check_structure, compare, gpu_verify, oracle_verify
+
+pytestmark = pytest.mark.gpu
+
+
+def _cuda(batch):
+    for name in ("zt", "zd", "tokens", "temperature", "conf", "lengths"):
+        t = getattr(batch, name)
+        if t is not None:
+            setattr(batch, name, t.cuda())
+    return batch
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2, 3, 12345])
+def test_c0_matches_oracle(seed):
+    b = _cuda(workloads.make_batch("c0", device="cpu"))
+    g = gpu_verify(b.zt, b.zd, b.tokens, b.lengths, b.temperature, seed)
+    o = oracle_verify(b.zt, b.zd, b.tokens, b.lengths.cpu().numpy(), b.temperature, seed)
+    check_structure(g, b.tokens.cpu().numpy(), b.lengths.cpu().numpy())
+    res = compare(g, o)
+    assert g["status"] == 0 and o["status"] == 0
+    assert res["ties"] == 0
+
+
+SMALL = [
+    # V, dtype, K, B: ragged tails (V not a multiple of 16 bytes), several
+    # chunks per vector (V > 4096 units), tiny vocabularies.
+    (1, torch.float32, 3, 16), (2, torch.bfloat16, 2, 32), (5, torch.float32, 4, 32),
+    (7, torch.bfloat16, 8, 32), (8, torch.bfloat16, 3, 16), (33, torch.float32, 5, 32),
+    (1000, torch.bfloat16, 4, 32), (1001, torch.bfloat16, 6, 32), (1003, torch.float32, 2, 24),
+    (4099, torch.float32, 3, 16), (8193, torch.bfloat16, 7, 16), (20011, torch.float32, 3, 12),
+    (40000, torch.bfloat16, 4, 12), (65543, torch.bfloat16, 2, 8),
+]
+
+
+@pytest.mark.parametrize("V,dtype,K,B", SMALL)
+def test_small_ragged_matches_oracle(V, dtype, K, B):
+    b = _cuda(workloads.random_small(B, K, V, dtype=dtype, seed=V + K,
+                                     temps=(0.0, 0.6, 1.0, 2.5)))
+    total = dict(rows=0, ties=0)
+    for seed in (7, 8):
+        g = gpu_verify(b.zt, b.zd, b.tokens, b.lengths, b.temperature, seed, debug=True)
+        ln = b.lengths.cpu().numpy()
+        o = oracle_verify(b.zt, b.zd, b.tokens, ln, b.temperature, seed)
+        check_structure(g, b.tokens.cpu().numpy(), ln)
+        r = compare(g, o)
+        total["rows"] += r["rows"]
+        total["ties"] += r["ties"]
+        total["tie_mismatches"] = total.get("tie_mismatches", 0) + r["tie_mismatches"]
+        assert g["status"] == 0
+    # rows inside a tie window are excluded from the bit-exact check and
+    # counted; a CDF window of 1e-5 * R is hit by roughly 2e-5 * R / r(y) of
+    # draws.  Rows that actually differ must be rare even inside it.
+    assert total["tie_mismatches"] <= max(2, total["rows"] // 50)
+
+
+@pytest.mark.parametrize("V,dtype", [(1000, torch.float32), (129280, torch.bfloat16),
+                                     (20011, torch.float32), (1001, torch.bfloat16)])
+def test_normalisers_match_oracle(V, dtype):
+    """m bit-exact, Sigma within 1e-5 relative, for every vector the call read."""
+    B, K = 16, 4
+    b = _cuda(workloads.random_small(B, K, V, dtype=dtype, seed=3, temps=(0.0, 0.6, 1.0, 1.7),
+                                     lengths=K))
+    g = gpu_verify(b.zt, b.zd, b.tokens, b.lengths, b.temperature, 5, debug=True)
+    st = g["stats"]
+    T = b.temperature.cpu().numpy()
+    mt, St, _ = oracle.stats(to_host_logits(b.zt), T[:, None])
+    md, Sd, _ = oracle.stats(to_host_logits(b.zd), T[:, None])
+    for r in range(B):
+        for i in range(K + 1):
+            assert st[r, i, 0] == mt[r, i]
+            if T[r] > 0:
+                assert abs(st[r, i, 1] - St[r, i]) <= 1e-5 * St[r, i]
+        for i in range(K):
+            if T[r] > 0:
+                assert st[r, K + 1 + i, 0] == md[r, i]
+                assert abs(st[r, K + 1 + i, 1] - Sd[r, i]) <= 1e-5 * Sd[r, i]
+            else:
+                assert np.isnan(st[r, K + 1 + i, 0])      # greedy rows never read drafts
+
+
+@pytest.mark.parametrize("V,dtype", [(7, torch.float32), (1000, torch.bfloat16),
+                                     (129280, torch.bfloat16)])
+def test_greedy_drafter_matches_oracle(V, dtype):
+    b = _cuda(workloads.random_small(24, 5, V, dtype=dtype, seed=11, temps=(0.0, 0.7, 1.0)))
+    for seed in (1, 2):
+        g = gpu_verify(b.zt, None, b.tokens, b.lengths, b.temperature, seed)
+        ln = b.lengths.cpu().numpy()
+        o = oracle_verify(b.zt, None, b.tokens, ln, b.temperature, seed)
+        check_structure(g, b.tokens.cpu().numpy(), ln)
+        compare(g, o)
+
+
+def test_edge_cases():
+    dev = "cuda"
+    # all-equal logits, -inf masks, L = 0 everywhere, T at the smallest legal value
+    B, K, V = 12, 3, 300
+    zt = torch.zeros(B, K + 1, V, device=dev)
+    zd = torch.zeros(B, K, V, device=dev)
+    zt[:, :, 50:] = float("-inf")
+    zd[:, :, 100:] = float("-inf")
+    zt[6:, :, :] = torch.randn(B - 6, K + 1, V, device=dev)
+    tokens = torch.randint(0, 50, (B, K), dtype=torch.int32, device=dev)
+    temp = torch.tensor([1.0, 1e-6, 0.0, 2.0] * 3, device=dev)
+    for L in (0, 1, K):
+        ln = torch.full((B,), L, dtype=torch.int32, device=dev)
+        g = gpu_verify(zt, zd, tokens, ln, temp, 3)
+        o = oracle_verify(zt, zd, tokens, ln.cpu().numpy(), temp, 3)
+        check_structure(g, tokens.cpu().numpy(), ln.cpu().numpy())
+        compare(g, o)
+        # masked tokens are never emitted by sampled rows' final draw
+        fin = g["tokens"][np.arange(B), g["accept"]]
+        assert np.all(fin[:6] < 50)
+
+
+def test_invalid_rows_marked_not_fatal():
+    dev = "cuda"
+    B, K, V = 6, 3, 64
+    zt = torch.randn(B, K + 1, V, device=dev)
+    zd = torch.randn(B, K, V, device=dev)
+    tokens = torch.randint(0, V, (B, K), dtype=torch.int32, device=dev)
+    tokens[1, 0] = V
+    tokens[5, 2] = -3            # beyond L: ignored
+    ln = torch.tensor([3, 3, 4, 1, -1, 2], dtype=torch.int32, device=dev)
+    temp = torch.tensor([1.0, 1.0, 1.0, float("nan"), 1.0, 1.0], device=dev)
+    g = gpu_verify(zt, zd, tokens, ln, temp, 1)
+    assert g["status"] == (sv.SV_ROW_BAD_TOKEN | sv.SV_ROW_BAD_LENGTH
+                           | sv.SV_ROW_BAD_TEMPERATURE)
+    assert list(g["accept"][[1, 2, 3, 4]]) == [-1, -1, -1, -1]
+    assert np.all(g["tokens"][[1, 2, 3, 4]] == -1)
+    o = oracle_verify(zt, zd, tokens, ln.cpu().numpy(), temp, 1)
+    assert o["status"] == g["status"]
+    compare(g, o)
+
+
+def test_sharding_by_row_base_and_determinism():
+    b = _cuda(workloads.random_small(64, 4, 5000, dtype=torch.bfloat16, seed=4,
+                                     temps=(0.0, 1.0)))
+    full = gpu_verify(b.zt, b.zd, b.tokens, b.lengths, b.temperature, 99)
+    again = gpu_verify(b.zt, b.zd, b.tokens, b.lengths, b.temperature, 99)
+    assert np.array_equal(full["tokens"], again["tokens"])
+    parts = [gpu_verify(b.zt[r0:r0 + 16].contiguous(), b.zd[r0:r0 + 16].contiguous(),
+                        b.tokens[r0:r0 + 16].contiguous(), b.lengths[r0:r0 + 16].contiguous(),
+                        b.temperature[r0:r0 + 16].contiguous(), 99, row_base=r0)
+             for r0 in range(0, 64, 16)]
+    assert np.array_equal(np.concatenate([p["tokens"] for p in parts]), full["tokens"])
+    other = gpu_verify(b.zt, b.zd, b.tokens, b.lengths, b.temperature, 100)
+    assert not np.array_equal(other["tokens"], full["tokens"])
+
+
+def test_workspace_reuse_and_garbage():
+    """The workspace needs no initialisation and can be reused across calls."""
+    b = _cuda(workloads.random_small(32, 4, 3000, dtype=torch.float32, seed=8))
+    n = sv.sv_verify_workspace_bytes(32, 4, 3000, sv.SV_F32)
+    ws = torch.randint(0, 255, (n,), dtype=torch.uint8, device="cuda")
+    g1 = gpu_verify(b.zt, b.zd, b.tokens, b.lengths, b.temperature, 5, workspace=ws)
+    g2 = gpu_verify(b.zt, b.zd, b.tokens, b.lengths, b.temperature, 5, workspace=ws)
+    assert np.array_equal(g1["tokens"], g2["tokens"])
+    o = oracle_verify(b.zt, b.zd, b.tokens, b.lengths.cpu().numpy(), b.temperature, 5)
+    compare(g1, o)
