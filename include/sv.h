@@ -50,10 +50,11 @@ typedef enum { SV_F32 = 0, SV_BF16 = 1 } sv_dtype;
 #define SV_ROW_BAD_TEMPERATURE  4   /* T < 0, NaN, inf, or 0 < T < 1e-6 */
 #define SV_NOTE_ZERO_RESIDUAL   8   /* informational: a rejection left zero residual mass (drew from p_j) */
 #define SV_NOTE_CDF_FALLBACK   16   /* informational: rounding put the CDF target past the total */
+#define SV_NOTE_TIMEOUT        32   /* an internal wait exceeded its 1 s bound; outputs are undefined */
 
 /* Supported sizes. */
 #define SV_MAX_K  64
-#define SV_MAX_V  (1 << 28)
+#define SV_MAX_V  (1 << 20)
 
 /*
  * sv_schedule -- per-row verify length from prefix survival.

@@ -20,18 +20,25 @@
 // positions 0..L, draft positions 0..L-1 for sampled rows).  Every vector is
 // cut into C equal chunks of 16-byte units, and one *item* is one chunk.
 //   1. prologue_kernel (1 CTA): validates rows, counts items per row, writes
-//      the exclusive prefix of item counts (the work list is implicit in
-//      it) and resets the counters.
-//   2. verify_kernel (persistent, 2 CTAs/SM): CTAs take items from a global
-//      atomic counter in row-major order.  An item is one HBM pass over its
-//      chunk: 16-byte streaming loads, 8 per thread in flight, packed bf16x2
-//      max, then one exp2 per element against the thread's max, then a
-//      block (max, sum) merge; greedy rows keep (max, first argmax) instead.
-//      The partial is published and a per-row atomic counter is bumped.  The
-//      CTA that completes a row's last item (no waiting: the atomic tells it)
-//      merges the row's partials, runs the accept test with Philox uniforms,
-//      and draws the final token, re-reading only position j while the row's
-//      bytes are still resident in L2.  No CTA ever waits on another.
+//      the exclusive prefix of item counts (the work list is implicit in it)
+//      and resets the per-row counters.
+//   2. stream_kernel (persistent, 2 CTAs/SM, warp-specialised): one HBM pass
+//      over every scheduled vector.  A producer warp takes items from a
+//      global atomic counter, decodes them and streams their bytes into a
+//      6-stage shared-memory ring with bulk copies (cp.async.bulk, mbarrier
+//      completion), running ahead of the math across item boundaries.  Eight
+//      consumer warps reduce each stage -- packed bf16x2 max, one exp2 per
+//      element against the running max -- and publish one (max, sum) partial
+//      per item (greedy rows: max and first argmax).  Every mbarrier wait is
+//      bounded in wall time and reports SV_NOTE_TIMEOUT instead of hanging.
+//   3. draw_kernel (one CTA per row and chunk): merges the partials into the
+//      normalisers, runs the accept test with Philox uniforms, and draws the
+//      final token by inverse CDF in two steps: over chunks, then inside the
+//      chosen chunk.  Chunk masses of p_j (bonus, greedy drafter) come from
+//      the stream partials without touching the logits again; the residual
+//      max(0, p_j - q_j) is summed chunk by chunk by the row's CTAs in
+//      parallel, and the last of them (atomic counter, no waiting) locates
+//      the token.  Only position j of a rejecting row is read a second time.
 #include <climits>
 #include <cstdint>
 #include <cstdio>
@@ -42,11 +49,16 @@
 
 namespace sv {
 
-constexpr int kThreads = 512;
-constexpr int kWarps = kThreads / 32;
-constexpr int kUnroll = 8;                     // 16-byte units per thread per item
-constexpr int kMaxUnitsPerItem = kThreads * kUnroll;
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = kConsumerWarps * 32;   // consumer group (warps 0..7)
+constexpr int kBlock = kConsumers + 32;           // + one producer warp
+constexpr int kStages = 4;                        // shared-memory ring depth
+constexpr int kStageUnits = 1024;                 // 16-byte units per stage (16 KB)
+constexpr int kRingBytes = kStages * kStageUnits * 16;
+constexpr int kMaxUnitsPerItem = 4 * kStageUnits; // an item spans up to 4 stages
 constexpr int kMaxSlots = 2 * SV_MAX_K + 1;
+constexpr int kMaxChunks = 64;                    // V <= SV_MAX_V keeps C within this
+constexpr int kPartsPerItem = kConsumerWarps;     // one softmax partial per consumer warp
 constexpr int kPrologueThreads = 1024;
 
 struct VerifyArgs {
@@ -63,9 +75,11 @@ struct VerifyArgs {
     int32_t *status;           // nullable
     float *dbg;                // nullable [B, S, 2]
     int *ctr;                  // [0] next item, [1] total items
-    int *row_cnt;              // [B]
+    int *rcnt;                 // [B]  chunks of the residual draw done
     int *row_off;              // [B+1]
     float4 *part;              // [B, S, C]: (m, s, argmax bits, 0)
+    float *rseg;               // [B, C, 8] residual mass per chunk segment
+    struct DrawRecord *rec;    // [B] accept result and draw set-up
 };
 
 template <int ESIZE>
@@ -117,7 +131,7 @@ __global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(VerifyArgs a
             } else {
                 n = row_slots(a, a.lengths[b], a.temp[b]) * a.C;
             }
-            a.row_cnt[b] = 0;
+            a.rcnt[b] = 0;
         }
         int x = n;
 #pragma unroll
@@ -151,57 +165,73 @@ __global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(VerifyArgs a
 }
 
 // ---------------------------------------------------------------------------
-// 2a. One item: a chunk of one vector.
+// 2. Stream kernel: softmax statistics of every scheduled vector.
 // ---------------------------------------------------------------------------
-struct ItemResult { float m, s; int idx; };
+constexpr int kGroup = kConsumers;   // threads of the consumer group
 
-// Per-thread (max, sum exp2((z - max) k)) over the thread's units.
-template <int ESIZE>
-__device__ __forceinline__ void thread_lse(const uint4 (&v)[kUnroll + 1], float k, float &m_out,
-                                           float &s_out) {
-    float m;
+// Online (max, sum) update with a batch of units.  The batch max is a
+// balanced tree of packed bf16x2 (or f32) max operations; the running sum is
+// rescaled once if the max grew; then one exp2 per element with the
+// argument formed by one packed FMA, z * k + c with c = RN(-m * k).  The
+// rounding of c is exact to recover, -m * k = c + e with e = fma(-m, k, -c),
+// and common to the batch, so the batch sum is multiplied by 2^e
+// (= 1 + e ln 2 to far below fp32 resolution, |e| < 1e-6).  Two packed
+// accumulators halve the add chain.
+template <int ESIZE, int N>
+__device__ __forceinline__ void lse_update(const uint4 (&v)[N], float k, float &m, float &s) {
+    float bm;
     if (ESIZE == 2) {
-        uint32_t mx = v[0].x;
+        uint32_t t[N];
 #pragma unroll
-        for (int j = 0; j <= kUnroll; ++j) {
-            mx = bmax2(mx, v[j].x); mx = bmax2(mx, v[j].y);
-            mx = bmax2(mx, v[j].z); mx = bmax2(mx, v[j].w);
-        }
-        m = fmaxf(bf16_lo(mx), bf16_hi(mx));
+        for (int j = 0; j < N; ++j) t[j] = bmax2(bmax2(v[j].x, v[j].y), bmax2(v[j].z, v[j].w));
+#pragma unroll
+        for (int w = 1; w < N; w <<= 1)
+#pragma unroll
+            for (int j = 0; j + w < N; j += 2 * w) t[j] = bmax2(t[j], t[j + w]);
+        bm = fmaxf(bf16_lo(t[0]), bf16_hi(t[0]));
     } else {
-        m = kNegInf;
+        float t[N];
 #pragma unroll
-        for (int j = 0; j <= kUnroll; ++j)
-            m = fmaxf(fmaxf(fmaxf(m, __uint_as_float(v[j].x)), __uint_as_float(v[j].y)),
-                      fmaxf(__uint_as_float(v[j].z), __uint_as_float(v[j].w)));
+        for (int j = 0; j < N; ++j)
+            t[j] = fmaxf(fmaxf(__uint_as_float(v[j].x), __uint_as_float(v[j].y)),
+                         fmaxf(__uint_as_float(v[j].z), __uint_as_float(v[j].w)));
+#pragma unroll
+        for (int w = 1; w < N; w <<= 1)
+#pragma unroll
+            for (int j = 0; j + w < N; j += 2 * w) t[j] = fmaxf(t[j], t[j + w]);
+        bm = t[0];
     }
-    float s = 0.f;
-    if (m != kNegInf) {
-        const float2 nm = make_float2(-m, -m), kk = make_float2(k, k);
-        float2 acc = make_float2(0.f, 0.f);
+    if (bm == kNegInf) return;              // nothing but padding / -inf
+    if (bm > m) {
+        s = (m == kNegInf) ? 0.f : s * ex2((m - bm) * k);
+        m = bm;
+    }
+    const float c = -m * k;
+    const float e = fmaf(-m, k, -c);
+    const float2 cc = make_float2(c, c), kk = make_float2(k, k);
+    float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int j = 0; j <= kUnroll; ++j) {
-            const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
-            if (ESIZE == 2) {
+    for (int j = 0; j < N; ++j) {
+        const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+        if (ESIZE == 2) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float2 z = make_float2(bf16_lo(w[q]), bf16_hi(w[q]));
-                    const float2 d = __fmul2_rn(__fadd2_rn(z, nm), kk);
-                    acc = __fadd2_rn(acc, make_float2(ex2(d.x), ex2(d.y)));
-                }
-            } else {
+            for (int q = 0; q < 4; ++q) {
+                const float2 z = make_float2(bf16_lo(w[q]), bf16_hi(w[q]));
+                const float2 d = __ffma2_rn(z, kk, cc);
+                const float2 e = make_float2(ex2(d.x), ex2(d.y));
+                if (q & 1) acc1 = __fadd2_rn(acc1, e); else acc0 = __fadd2_rn(acc0, e);
+            }
+        } else {
 #pragma unroll
-                for (int q = 0; q < 4; q += 2) {
-                    const float2 z = make_float2(__uint_as_float(w[q]), __uint_as_float(w[q + 1]));
-                    const float2 d = __fmul2_rn(__fadd2_rn(z, nm), kk);
-                    acc = __fadd2_rn(acc, make_float2(ex2(d.x), ex2(d.y)));
-                }
+            for (int q = 0; q < 4; q += 2) {
+                const float2 z = make_float2(__uint_as_float(w[q]), __uint_as_float(w[q + 1]));
+                const float2 d = __ffma2_rn(z, kk, cc);
+                const float2 e = make_float2(ex2(d.x), ex2(d.y));
+                if (q & 2) acc1 = __fadd2_rn(acc1, e); else acc0 = __fadd2_rn(acc0, e);
             }
         }
-        s = acc.x + acc.y;
     }
-    m_out = m;
-    s_out = s;
+    s = fmaf((acc0.x + acc0.y) + (acc1.x + acc1.y), fmaf(e, 0.69314718055994531f, 1.f), s);
 }
 
 template <int ESIZE>
@@ -214,329 +244,723 @@ __device__ __forceinline__ void consider_unit(const uint4 &u, int first, float &
     }
 }
 
+struct __align__(16) StageDesc {
+    int b;        // row; -1 = no more work
+    int slot;
+    int chunk;
+    int unit0;    // first body unit of the stage, relative to the vector
+    int nunits;   // body units in the stage
+    int flags;    // kFirst | kLast
+    float k;      // log2(e)/T; 0 for greedy rows
+    int pad;
+};
+constexpr int kFirst = 1, kLast = 2;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s: no legitimate wait comes close
+
+__device__ __forceinline__ int vload(const int &x) {
+    return *reinterpret_cast<const volatile int *>(&x);
+}
+__device__ __forceinline__ void vstore(int &x, int v) {
+    *reinterpret_cast<volatile int *>(&x) = v;
+}
+
+struct StreamSmem {
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    StageDesc desc[kStages];
+    int abort;
+};
+
+// Producer: fetch items (global atomic counter, prefetched one item ahead),
+// decode them, stream their 16-byte body units into the ring.
 template <int ESIZE>
-__device__ ItemResult process_item(const VerifyArgs &a, const char *vbase, int chunk, bool greedy,
-                                   float k, float *s_red_m, float *s_red_s, int *s_red_i) {
+__device__ void producer(const VerifyArgs &a, StreamSmem &sm, uint4 *ring, int total) {
+    uint32_t it = 0;
+    bool ok = true;
+    int w = atomicAdd(&a.ctr[0], 1);
+    while (ok) {
+        if (w >= total) {
+            const int st = it % kStages;
+            const uint32_t ph = (it / kStages) & 1u;
+            if (!mbar_wait(&sm.empty[st], ph ^ 1u, kWaitLimitNs)) { ok = false; break; }
+            sm.desc[st].b = -1;
+            mbar_arrive(&sm.full[st]);
+            ++it;
+            break;
+        }
+        // Decode item w: row b (largest b with row_off[b] <= w), slot, chunk.
+        int lo = 0, hi = a.B - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (__ldg(&a.row_off[mid]) <= w) lo = mid; else hi = mid - 1;
+        }
+        const int b = lo;
+        const int r = w - __ldg(&a.row_off[b]);
+        const int L = __ldg(&a.lengths[b]);
+        const float T = __ldg(&a.temp[b]);
+        const int q = r / a.C, chunk = r - q * a.C;
+        const int slot = q <= L ? q : (a.K + 1 + (q - L - 1));
+        const float k = (T > 0.f) ? kLog2e / T : 0.f;
+        const VecGeom g = vec_geom<ESIZE>(vec_ptr<ESIZE>(a, b, slot), a.V);
+        const int u0 = chunk * a.U;
+        const int u1 = max(u0, min(u0 + a.U, g.n16));
+        const int wnext = atomicAdd(&a.ctr[0], 1);   // next item, consumed after this one
+        const int npieces = max(1, (u1 - u0 + kStageUnits - 1) / kStageUnits);
+        for (int p = 0; p < npieces; ++p) {
+            const int st = it % kStages;
+            const uint32_t ph = (it / kStages) & 1u;
+            if (!mbar_wait(&sm.empty[st], ph ^ 1u, kWaitLimitNs) || vload(sm.abort)) {
+                ok = false;
+                break;
+            }
+            const int pu0 = u0 + p * kStageUnits;
+            const int pn = max(0, min(u1 - pu0, kStageUnits));
+            StageDesc &d = sm.desc[st];
+            d.b = b; d.slot = slot; d.chunk = chunk; d.unit0 = pu0; d.nunits = pn;
+            d.flags = (p == 0 ? kFirst : 0) | (p == npieces - 1 ? kLast : 0);
+            d.k = k;
+            if (pn > 0) {
+                mbar_arrive_expect_tx(&sm.full[st], static_cast<uint32_t>(pn) * 16u);
+                bulk_g2s(ring + static_cast<size_t>(st) * kStageUnits,
+                         g.body + static_cast<long long>(pu0) * 16, static_cast<uint32_t>(pn) * 16u,
+                         &sm.full[st]);
+            } else {
+                mbar_arrive(&sm.full[st]);
+            }
+            ++it;
+        }
+        w = wnext;
+    }
+    if (!ok) {
+        // Unwind: report, then wait (bounded) for the copies still in flight
+        // so that none lands in shared memory after the block exits.
+        vstore(sm.abort, 1);
+        if (a.status) atomicOr(a.status, SV_NOTE_TIMEOUT);
+        const uint32_t n = it < kStages ? it : kStages;
+        for (uint32_t i = 0; i < n; ++i) {
+            const uint32_t t = it - 1 - i;
+            mbar_wait(&sm.full[t % kStages], (t / kStages) & 1u, kWaitLimitNs / 4);
+        }
+    }
+}
+
+// Consumers: reduce each stage into the running (max, sum) -- or (max,
+// first argmax) for greedy rows -- and publish one partial per item.
+template <int ESIZE>
+__device__ void consumers(const VerifyArgs &a, StreamSmem &sm, const uint4 *ring) {
     constexpr int kPer = 16 / ESIZE;
+    constexpr int kPerThread = kStageUnits / kGroup;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const VecGeom g = vec_geom<ESIZE>(vbase, a.V);
-    const int u0 = chunk * a.U;
-    const int u1 = min(u0 + a.U, g.n16);
     const uint32_t pw = neg_inf_word<ESIZE>();
     const uint4 pad = make_uint4(pw, pw, pw, pw);
-
-    uint4 v[kUnroll + 1];
-#pragma unroll
-    for (int j = 0; j < kUnroll; ++j) {
-        const int u = u0 + tid + j * kThreads;
-        v[j] = (u < u1) ? ld_stream(g.body + static_cast<long long>(u) * 16) : pad;
-    }
-    // Head (chunk 0, thread 0) and tail (last chunk, thread 1) elements.
-    v[kUnroll] = pad;
-    int extra_first = 0;
-    bool extra_is_head = false;
-    if (chunk == 0 && tid == 0 && g.head > 0) {
-        v[kUnroll] = ld_partial_unit<ESIZE>(g.base, 0, g.head);
-        extra_is_head = true;
-    }
-    if (chunk == a.C - 1 && tid == 1 && g.tail > 0) {
-        extra_first = g.head + g.n16 * kPer;
-        v[kUnroll] = ld_partial_unit<ESIZE>(g.base, extra_first, g.tail);
-    }
-
-    ItemResult r;
-    if (!greedy) {
-        float m, s;
-        thread_lse<ESIZE>(v, k, m, s);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-            const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
-            lse_merge(m, s, m2, s2, k);
+    uint32_t it = 0;
+    float m = kNegInf, s = 0.f;
+    int bidx = INT_MAX;
+    while (true) {
+        const int st = it % kStages;
+        const uint32_t ph = (it / kStages) & 1u;
+        if (!mbar_wait(&sm.full[st], ph, kWaitLimitNs) || vload(sm.abort)) {
+            vstore(sm.abort, 1);
+            if (a.status && tid == 0) atomicOr(a.status, SV_NOTE_TIMEOUT);
+            break;
         }
-        if (lane == 0) { s_red_m[warp] = m; s_red_s[warp] = s; }
-        __syncthreads();
-        if (warp == 0) {
-            m = lane < kWarps ? s_red_m[lane] : kNegInf;
-            s = lane < kWarps ? s_red_s[lane] : 0.f;
+        const StageDesc d = sm.desc[st];
+        if (d.b < 0) break;
+        const bool greedy = d.k == 0.f;
+        if (d.flags & kFirst) { m = kNegInf; s = 0.f; bidx = INT_MAX; }
+        const uint4 *src = ring + static_cast<size_t>(st) * kStageUnits;
+        uint4 v[kPerThread];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-                const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
-                lse_merge(m, s, m2, s2, k);
+        for (int j = 0; j < kPerThread; ++j) {
+            const int u = tid + j * kGroup;
+            v[j] = u < d.nunits ? src[u] : pad;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[st]);
+        ++it;
+
+        // Head (first stage of chunk 0, thread 0) and tail (last stage of the
+        // last chunk, thread 1) elements, loaded directly.
+        uint4 extra = pad;
+        int extra_first = 0;
+        bool have_head = false, have_tail = false;
+        const bool head_here = (d.flags & kFirst) && d.chunk == 0 && tid == 0;
+        const bool tail_here = (d.flags & kLast) && d.chunk == a.C - 1 && tid == 1;
+        int vhead = 0;
+        if (head_here || tail_here || greedy) {
+            const VecGeom g = vec_geom<ESIZE>(vec_ptr<ESIZE>(a, d.b, d.slot), a.V);
+            vhead = g.head;
+            if (head_here && g.head > 0) {
+                extra = ld_partial_unit<ESIZE>(g.base, 0, g.head);
+                have_head = true;
+            }
+            if (tail_here && g.tail > 0) {
+                extra_first = g.head + g.n16 * kPer;
+                extra = ld_partial_unit<ESIZE>(g.base, extra_first, g.tail);
+                have_tail = true;
             }
         }
-        r.m = m; r.s = s; r.idx = 0;
-    } else {
-        // (max, first index of max); each thread scans its units in index order.
-        float best = kNegInf;
-        int bidx = INT_MAX;
-        if (extra_is_head) consider_unit<ESIZE>(v[kUnroll], 0, best, bidx);
+        if (!greedy) {
+            lse_update<ESIZE, kPerThread>(v, d.k, m, s);
+            if (have_head || have_tail) {
+                uint4 e1[1] = {extra};
+                lse_update<ESIZE, 1>(e1, d.k, m, s);
+            }
+        } else {
+            // Index order within the thread: head, then body, then tail.
+            if (have_head) consider_unit<ESIZE>(extra, 0, m, bidx);
 #pragma unroll
-        for (int j = 0; j < kUnroll; ++j)
-            consider_unit<ESIZE>(v[j], g.head + (u0 + tid + j * kThreads) * kPer, best, bidx);
-        if (!extra_is_head) consider_unit<ESIZE>(v[kUnroll], extra_first, best, bidx);
+            for (int j = 0; j < kPerThread; ++j)
+                consider_unit<ESIZE>(v[j], vhead + (d.unit0 + tid + j * kGroup) * kPer, m, bidx);
+            if (have_tail) consider_unit<ESIZE>(extra, extra_first, m, bidx);
+        }
+
+        if (!(d.flags & kLast)) continue;
+        // End of item: warp reduction; one partial per (row, slot, chunk,
+        // warp), so the warps never wait for one another.
+        float rm = m, rs = s;
+        int ri = bidx;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
-            const float b2 = __shfl_xor_sync(0xffffffffu, best, o);
-            const int i2 = __shfl_xor_sync(0xffffffffu, bidx, o);
-            if (b2 > best || (b2 == best && i2 < bidx)) { best = b2; bidx = i2; }
-        }
-        if (lane == 0) { s_red_m[warp] = best; s_red_i[warp] = bidx; }
-        __syncthreads();
-        if (warp == 0) {
-            best = lane < kWarps ? s_red_m[lane] : kNegInf;
-            bidx = lane < kWarps ? s_red_i[lane] : INT_MAX;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float b2 = __shfl_xor_sync(0xffffffffu, best, o);
-                const int i2 = __shfl_xor_sync(0xffffffffu, bidx, o);
-                if (b2 > best || (b2 == best && i2 < bidx)) { best = b2; bidx = i2; }
+            const float m2 = __shfl_xor_sync(0xffffffffu, rm, o);
+            const float s2 = __shfl_xor_sync(0xffffffffu, rs, o);
+            const int i2 = __shfl_xor_sync(0xffffffffu, ri, o);
+            if (greedy) {
+                if (m2 > rm || (m2 == rm && i2 < ri)) { rm = m2; ri = i2; }
+            } else {
+                lse_merge(rm, rs, m2, s2, d.k);
             }
         }
-        r.m = best; r.s = 0.f; r.idx = bidx;
+        if (lane == 0)
+            a.part[((static_cast<long long>(d.b) * a.S + d.slot) * a.C + d.chunk) * kPartsPerItem +
+                   warp] = make_float4(rm, greedy ? 0.f : rs, __int_as_float(greedy ? ri : 0), 0.f);
     }
-    return r;   // valid in thread 0
+}
+
+// Persistent warp-specialised kernel: warp kConsumerWarps is the producer
+// (work fetch + bulk copies into the shared-memory ring), warps
+// 0..kConsumerWarps-1 consume stages.
+template <int ESIZE>
+__global__ void __launch_bounds__(kBlock, 3) stream_kernel(VerifyArgs a) {
+    extern __shared__ __align__(128) uint4 ring[];
+    __shared__ StreamSmem sm;
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&sm.full[i], 1);
+            mbar_init(&sm.empty[i], kConsumerWarps);
+        }
+        sm.abort = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const int total = __ldcg(&a.ctr[1]);
+    if (tid >= kConsumers) {
+        if (tid == kConsumers) producer<ESIZE>(a, sm, ring, total);
+        return;
+    }
+    consumers<ESIZE>(a, sm, ring);
 }
 
 // ---------------------------------------------------------------------------
-// 2b. Row finisher: merge partials, accept test, final draw.
+// 3. Draw kernel: one CTA per (row, chunk).  Accept test from the partials,
+//    then the final token by inverse CDF over chunks, then within a chunk.
 // ---------------------------------------------------------------------------
-struct FinSmem {
+constexpr int kDrawThreads = 256;
+constexpr int kDrawWarps = kDrawThreads / 32;
+
+struct DrawSmem {
     float m[kMaxSlots];
     float s[kMaxSlots];
     int arg[kMaxSlots];
-    float wsum[kWarps];
-    float tsum_warp[kWarps];
+    float cm[kMaxChunks];
+    float wsum[kDrawWarps];
+    float tsum_warp[kDrawWarps];
     int j;
     int gsel;
     float dsel;
     int tsel;
     int lastpos;
     int ysel;
-    int mode;
+    int last;
 };
 
-enum DrawMode { kDrawP = 0, kDrawResidual = 1, kDrawResidualOneHot = 2 };
+enum DrawMode { kDrawP = 0, kDrawResidual = 1, kDrawOneHot = 2 };
 
 struct DrawCtx {
     VecGeom gt, gd;
     bool aligned;      // target and draft vectors share their 16-byte phase
     int mode;
-    float k, ct, cd;   // p(v) = 2^((zt_v - mt) k - ct), q(v) = 2^((zd_v - md) k - cd)
+    float k;
+    float ct, cd;      // weight offsets: p(v) = 2^((zt_v - mt) k - ct), q likewise
     float mt, md;
     int xj;
+    // chunk range in local units: 0 = head (if any), 1..nbody = body units
+    // [ubody0, ubody0 + nbody), nbody+1 = tail (if any)
+    int ubody0, nbody;
+    bool has_head, has_tail;
 };
 
-// Weights of the elements of unit u (0 = head, 1..n16 = body, n16+1 = tail)
-// of the draw at position j; returns the element count and first index.
-template <int ESIZE>
-__device__ __forceinline__ int unit_weights(const DrawCtx &c, int u, float (&w)[8], int &first) {
+// Raw data of one local unit of the chunk: 0 = head (if any), 1..nbody =
+// body units, nbody+1 = tail (if any).  `d` is the draft unit, loaded only
+// for residual draws of aligned vectors.
+struct UnitData {
+    uint4 t, d;
+    int count, first;
+};
+
+template <int ESIZE, int MODE>
+__device__ __forceinline__ UnitData load_unit(const DrawCtx &c, int lu) {
     constexpr int kPer = 16 / ESIZE;
-    int count;
-    uint4 ut, ud = make_uint4(0, 0, 0, 0);
-    const bool resid = c.mode == kDrawResidual;
-    if (u == 0) {
-        count = c.gt.head; first = 0;
-        ut = ld_partial_unit<ESIZE>(c.gt.base, 0, count);
-        if (resid && c.aligned) ud = ld_partial_unit<ESIZE>(c.gd.base, 0, count);
-    } else if (u <= c.gt.n16) {
-        count = kPer; first = c.gt.head + (u - 1) * kPer;
-        ut = ld_reuse(c.gt.body + static_cast<long long>(u - 1) * 16);
-        if (resid && c.aligned) ud = ld_reuse(c.gd.body + static_cast<long long>(u - 1) * 16);
+    constexpr bool kResid = MODE == kDrawResidual;
+    UnitData r;
+    r.d = make_uint4(0, 0, 0, 0);
+    if (lu == 0) {
+        r.count = c.has_head ? c.gt.head : 0; r.first = 0;
+        r.t = ld_partial_unit<ESIZE>(c.gt.base, 0, r.count);
+        if (kResid && c.aligned) r.d = ld_partial_unit<ESIZE>(c.gd.base, 0, r.count);
+    } else if (lu <= c.nbody) {
+        const int u = c.ubody0 + lu - 1;
+        r.count = kPer; r.first = c.gt.head + u * kPer;
+        r.t = ld_reuse(c.gt.body + static_cast<long long>(u) * 16);
+        if (kResid && c.aligned) r.d = ld_reuse(c.gd.body + static_cast<long long>(u) * 16);
     } else {
-        count = c.gt.tail; first = c.gt.head + c.gt.n16 * kPer;
-        ut = ld_partial_unit<ESIZE>(c.gt.base, first, count);
-        if (resid && c.aligned) ud = ld_partial_unit<ESIZE>(c.gd.base, first, count);
+        r.count = c.has_tail ? c.gt.tail : 0; r.first = c.gt.head + c.gt.n16 * kPer;
+        r.t = ld_partial_unit<ESIZE>(c.gt.base, r.first, r.count);
+        if (kResid && c.aligned) r.d = ld_partial_unit<ESIZE>(c.gd.base, r.first, r.count);
     }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        float x = 0.f;
-        if (e < kPer && e < count) {
-            const float p = ex2(fmaf(unit_elem<ESIZE>(ut, e) - c.mt, c.k, -c.ct));
-            if (c.mode == kDrawP) {
-                x = p;
-            } else if (c.mode == kDrawResidual) {
-                const float zd = c.aligned ? unit_elem<ESIZE>(ud, e)
-                                           : ld_elem<ESIZE>(c.gd.base, first + e);
-                const float q = ex2(fmaf(zd - c.md, c.k, -c.cd));
-                x = fmaxf(p - q, 0.f);
-            } else {
-                x = (first + e == c.xj) ? 0.f : p;
-            }
-        }
-        w[e] = x;
-    }
-    return count;
+    return r;
 }
 
-// Inverse-CDF draw over one vector with the whole block: warp segments give
-// the coarse CDF, one block pass over the selected segment gives the thread,
-// and that thread walks its elements.  Returns the token, -1 if the total
-// weight is zero (then *zero_mass is set).
+__device__ __forceinline__ UnitData empty_unit() {
+    UnitData r;
+    r.t = r.d = make_uint4(0, 0, 0, 0);
+    r.count = 0;
+    r.first = 0;
+    return r;
+}
+
+// Draw weight of element e of a loaded unit (0 past its count).
+template <int ESIZE, int MODE>
+__device__ __forceinline__ float elem_weight(const DrawCtx &c, const UnitData &u, int e) {
+    if (e >= u.count) return 0.f;
+    const float p = ex2(fmaf(unit_elem<ESIZE>(u.t, e) - c.mt, c.k, -c.ct));
+    if (MODE == kDrawP) return p;
+    if (MODE == kDrawOneHot) return (u.first + e == c.xj) ? 0.f : p;
+    const float zd = c.aligned ? unit_elem<ESIZE>(u.d, e) : ld_elem<ESIZE>(c.gd.base, u.first + e);
+    const float q = ex2(fmaf(zd - c.md, c.k, -c.cd));
+    return fmaxf(p - q, 0.f);
+}
+
+// Element pair q (elements 2q, 2q+1) of a packed unit, widened to fp32.
 template <int ESIZE>
-__device__ int block_draw(const DrawCtx &c, float u, FinSmem &fs, bool *zero_mass, bool *fallback) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int NU = c.gt.n16 + 2;
-    const int SU = (NU + kWarps - 1) / kWarps;
-    const int seg0 = warp * SU, seg1 = min(seg0 + SU, NU);
-    // Pass A: per-warp segment totals.
+__device__ __forceinline__ float2 unit_pair(const uint4 &u, int q) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    if (ESIZE == 2) return make_float2(bf16_lo(w[q]), bf16_hi(w[q]));
+    return make_float2(__uint_as_float(w[2 * q]), __uint_as_float(w[2 * q + 1]));
+}
+
+// Sum of the draw weights of a unit.  Full body units take a packed path:
+// per element pair, (z - m) by one packed add, (z - m) k - c by one packed
+// FMA, two exp2, and for the residual the same for q, a packed p - q, and
+// the clamp at 0.  Partial units, the one-hot unit that holds x_j, and
+// draft vectors out of phase with the target take the scalar path.
+template <int ESIZE, int MODE>
+__device__ __forceinline__ float unit_sum(const DrawCtx &c, const UnitData &u) {
+    constexpr int kPer = 16 / ESIZE;
+    const bool fast = u.count == kPer && (MODE != kDrawResidual || c.aligned) &&
+                      (MODE != kDrawOneHot || c.xj < u.first || c.xj >= u.first + kPer);
+    if (fast) {
+        const float2 kk = make_float2(c.k, c.k);
+        const float2 nmt = make_float2(-c.mt, -c.mt), nct = make_float2(-c.ct, -c.ct);
+        const float2 nmd = make_float2(-c.md, -c.md), ncd = make_float2(-c.cd, -c.cd);
+        const float2 neg1 = make_float2(-1.f, -1.f);
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < kPer / 2; ++q) {
+            const float2 at = __ffma2_rn(__fadd2_rn(unit_pair<ESIZE>(u.t, q), nmt), kk, nct);
+            float2 w = make_float2(ex2(at.x), ex2(at.y));
+            if (MODE == kDrawResidual) {
+                const float2 ad = __ffma2_rn(__fadd2_rn(unit_pair<ESIZE>(u.d, q), nmd), kk, ncd);
+                const float2 qv = make_float2(ex2(ad.x), ex2(ad.y));
+                const float2 r = __ffma2_rn(qv, neg1, w);
+                w = make_float2(fmaxf(r.x, 0.f), fmaxf(r.y, 0.f));
+            }
+            acc = __fadd2_rn(acc, w);
+        }
+        return acc.x + acc.y;
+    }
+    float t = 0.f;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) t += elem_weight<ESIZE, MODE>(c, u, e);
+    return t;
+}
+
+constexpr int kRunMax = 4;      // units per thread in the located segment
+
+// Segment g of the chunk (for warp g of the draw CTA): local units
+// [g * SU, min((g+1) * SU, NU)), SU = ceil(NU / kDrawWarps).
+__device__ __forceinline__ void segment_range(const DrawCtx &c, int g, int &s0, int &s1) {
+    const int NU = c.nbody + 2;
+    const int SU = (NU + kDrawWarps - 1) / kDrawWarps;
+    s0 = min(g * SU, NU);
+    s1 = min(s0 + SU, NU);
+}
+
+// Sum of the draw weights of a full body unit given as raw 16-byte words
+// (packed path; -inf padding contributes 0).  One-hot exclusion is not
+// applied here.
+template <int ESIZE, int MODE>
+__device__ __forceinline__ float body_sum(const DrawCtx &c, const uint4 &t, const uint4 &d) {
+    constexpr int kPer = 16 / ESIZE;
+    const float2 kk = make_float2(c.k, c.k);
+    const float2 nmt = make_float2(-c.mt, -c.mt), nct = make_float2(-c.ct, -c.ct);
+    const float2 nmd = make_float2(-c.md, -c.md), ncd = make_float2(-c.cd, -c.cd);
+    const float2 neg1 = make_float2(-1.f, -1.f);
+    float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < kPer / 2; ++q) {
+        const float2 at = __ffma2_rn(__fadd2_rn(unit_pair<ESIZE>(t, q), nmt), kk, nct);
+        float2 w = make_float2(ex2(at.x), ex2(at.y));
+        if (MODE == kDrawResidual) {
+            const float2 ad = __ffma2_rn(__fadd2_rn(unit_pair<ESIZE>(d, q), nmd), kk, ncd);
+            const float2 r = __ffma2_rn(make_float2(ex2(ad.x), ex2(ad.y)), neg1, w);
+            w = make_float2(fmaxf(r.x, 0.f), fmaxf(r.y, 0.f));
+        }
+        acc = __fadd2_rn(acc, w);
+    }
+    return acc.x + acc.y;
+}
+
+// Total draw weight of segment `warp` of the chunk.  Body units go through a
+// tight loop -- lanes stride through the segment (coalesced), 8 units per
+// lane in flight, raw 16-byte loads padded with -inf -- and the head, the
+// tail and the one-hot exclusion are applied once by lane 0.  A draft
+// vector out of 16-byte phase with the target takes the generic path.  All
+// lanes get the total.
+template <int ESIZE, int MODE>
+__device__ float warp_segment_total(const DrawCtx &c) {
+    constexpr int kPer = 16 / ESIZE;
+    constexpr int kB = 8;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int s0, s1;
+    segment_range(c, warp, s0, s1);
     float acc = 0.f;
-#pragma unroll 4
-    for (int uu = seg0 + lane; uu < seg1; uu += 32) {
-        float w[8];
-        int first;
-        unit_weights<ESIZE>(c, uu, w, first);
-        acc += ((w[0] + w[1]) + (w[2] + w[3])) + ((w[4] + w[5]) + (w[6] + w[7]));
+    if (MODE == kDrawResidual && !c.aligned) {
+        for (int lu = s0 + lane; lu < s1; lu += 32)
+            acc += unit_sum<ESIZE, MODE>(c, load_unit<ESIZE, MODE>(c, lu));
+    } else {
+        const int b0 = max(s0, 1), b1 = min(s1, c.nbody + 1);   // body local units
+        const uint32_t pw = neg_inf_word<ESIZE>();
+        const uint4 pad = make_uint4(pw, pw, pw, pw);
+        for (int base = b0; base < b1; base += 32 * kB) {
+            uint4 t[kB], d[kB];
+#pragma unroll
+            for (int i = 0; i < kB; ++i) {
+                const int lu = base + lane + 32 * i;
+                const long long off = static_cast<long long>(c.ubody0 + lu - 1) * 16;
+                t[i] = lu < b1 ? ld_reuse(c.gt.body + off) : pad;
+                if (MODE == kDrawResidual) d[i] = lu < b1 ? ld_reuse(c.gd.body + off) : pad;
+                else d[i] = pad;
+            }
+#pragma unroll
+            for (int i = 0; i < kB; ++i) acc += body_sum<ESIZE, MODE>(c, t[i], d[i]);
+        }
+        if (lane == 0) {
+            if (s0 == 0) acc += unit_sum<ESIZE, MODE>(c, load_unit<ESIZE, MODE>(c, 0));
+            const int lt = c.nbody + 1;
+            if (s0 <= lt && lt < s1) acc += unit_sum<ESIZE, MODE>(c, load_unit<ESIZE, MODE>(c, lt));
+            if (MODE == kDrawOneHot) {
+                // the body loop counted p(x_j); take it out if x_j is ours
+                const int ux = c.xj - c.gt.head;
+                if (c.xj >= c.gt.head && ux / kPer < c.gt.n16) {
+                    const int lx = ux / kPer - c.ubody0 + 1;
+                    if (lx >= b0 && lx < b1) {
+                        const float zx = ld_elem<ESIZE>(c.gt.base, c.xj);
+                        acc -= ex2(fmaf(zx - c.mt, c.k, -c.ct));
+                    }
+                }
+            }
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) fs.wsum[warp] = acc;
-    __syncthreads();
+    return acc;
+}
+
+// Smallest element of the chunk whose cumulative weight exceeds d, given
+// the chunk's segment totals in ds.wsum.  The block splits the selected
+// segment into contiguous runs (one per thread), scans the run totals, and
+// the owning thread walks its elements (weights recomputed from the units
+// it holds).  If rounding leaves d at or past the total, the last element
+// with positive weight is returned and *fallback is set; -1 if the chunk
+// has none.
+template <int ESIZE, int MODE>
+__device__ int chunk_locate(const DrawCtx &c, float d, DrawSmem &ds, bool *fallback) {
+    constexpr int kPer = 16 / ESIZE;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (tid == 0) {
-        float P = 0.f;
-        for (int g = 0; g < kWarps; ++g) P += fs.wsum[g];
-        const float R = P;
-        int gsel = -1;
-        float dsel = 0.f;
-        if (R > 0.f) {
-            const float t = u * R;
-            float pre = 0.f;
-            int lastg = -1;
-            for (int g = 0; g < kWarps; ++g) {
-                const float d = t - pre;
-                if (fs.wsum[g] > 0.f) lastg = g;
-                if (gsel < 0 && fs.wsum[g] > d) { gsel = g; dsel = d; }
-                pre += fs.wsum[g];
-            }
-            if (gsel < 0) { gsel = lastg; dsel = __int_as_float(0x7f800000); }
+        int gsel = -1, lastg = -1;
+        float dsel = 0.f, pre = 0.f;
+        for (int g = 0; g < kDrawWarps; ++g) {
+            const float dd = d - pre;
+            if (ds.wsum[g] > 0.f) lastg = g;
+            if (gsel < 0 && ds.wsum[g] > dd) { gsel = g; dsel = dd; }
+            pre += ds.wsum[g];
         }
-        fs.gsel = gsel;
-        fs.dsel = dsel;
-        fs.tsel = INT_MAX;
-        fs.lastpos = -1;
-        fs.ysel = -1;
+        if (gsel < 0) { gsel = lastg; dsel = __int_as_float(0x7f800000); }
+        ds.gsel = gsel;
+        ds.dsel = dsel;
+        ds.tsel = INT_MAX;
+        ds.lastpos = -1;
+        ds.ysel = -1;
     }
     __syncthreads();
-    const int gsel = fs.gsel;
-    if (gsel < 0) { *zero_mass = true; return -1; }
-    const float dsel = fs.dsel;
-    // Pass B: the block splits segment gsel into contiguous runs per thread.
-    const int s0 = gsel * SU, s1 = min(s0 + SU, NU);
-    const int per = (s1 - s0 + kThreads - 1) / kThreads;
-    const int r0 = min(s0 + tid * per, s1), r1 = min(r0 + per, s1);
+    const int gsel = ds.gsel;
+    if (gsel < 0) return -1;
+    const float dsel = ds.dsel;
+    int s0, s1;
+    segment_range(c, gsel, s0, s1);
+    const int per = (s1 - s0 + kDrawThreads - 1) / kDrawThreads;   // <= kRunMax
+    const int r0 = min(s0 + tid * per, s1);
+    UnitData ud[kRunMax];
+#pragma unroll
+    for (int i = 0; i < kRunMax; ++i)
+        ud[i] = (i < per && r0 + i < s1) ? load_unit<ESIZE, MODE>(c, r0 + i) : empty_unit();
     float mine = 0.f;
     int lastpos = -1;
-    for (int uu = r0; uu < r1; ++uu) {
-        float w[8];
-        int first;
-        const int cnt = unit_weights<ESIZE>(c, uu, w, first);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            if (e < cnt && w[e] > 0.f) lastpos = first + e;
-            mine += w[e];
+    for (int i = 0; i < kRunMax; ++i) {
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) {
+            const float w = elem_weight<ESIZE, MODE>(c, ud[i], e);
+            if (w > 0.f) lastpos = ud[i].first + e;
+            mine += w;
         }
     }
-    // Block inclusive scan of the per-thread sums.
     float x = mine;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const float y = __shfl_up_sync(0xffffffffu, x, o);
         if (lane >= o) x += y;
     }
-    if (lane == 31) fs.tsum_warp[warp] = x;
+    if (lane == 31) ds.tsum_warp[warp] = x;
     __syncthreads();
     if (warp == 0) {
-        float y = lane < kWarps ? fs.tsum_warp[lane] : 0.f;
+        float y = lane < kDrawWarps ? ds.tsum_warp[lane] : 0.f;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const float z = __shfl_up_sync(0xffffffffu, y, o);
             if (lane >= o) y += z;
         }
-        if (lane < kWarps) fs.tsum_warp[lane] = y;
+        if (lane < kDrawWarps) ds.tsum_warp[lane] = y;
     }
     __syncthreads();
-    const float wpre = warp ? fs.tsum_warp[warp - 1] : 0.f;
+    const float wpre = warp ? ds.tsum_warp[warp - 1] : 0.f;
     const float xprev = __shfl_up_sync(0xffffffffu, x, 1);
     const float incl = x + wpre;
     const float excl = (lane ? xprev : 0.f) + wpre;
-    if (incl > dsel) atomicMin(&fs.tsel, tid);
-    if (lastpos >= 0) atomicMax(&fs.lastpos, lastpos);
+    if (incl > dsel) atomicMin(&ds.tsel, tid);
+    if (lastpos >= 0) atomicMax(&ds.lastpos, lastpos);
     __syncthreads();
-    if (tid == fs.tsel) {
-        // Walk this thread's elements from the exclusive prefix.
+    if (tid == ds.tsel) {
         float cum = excl;
         int y = -1;
-        for (int uu = r0; uu < r1 && y < 0; ++uu) {
-            float w[8];
-            int first;
-            const int cnt = unit_weights<ESIZE>(c, uu, w, first);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                if (y < 0 && e < cnt) {
-                    cum += w[e];
-                    if (cum > dsel) y = first + e;
+        for (int i = 0; i < kRunMax; ++i) {
+#pragma unroll
+            for (int e = 0; e < kPer; ++e) {
+                if (y < 0) {
+                    cum += elem_weight<ESIZE, MODE>(c, ud[i], e);
+                    if (cum > dsel && e < ud[i].count) y = ud[i].first + e;
                 }
             }
         }
         if (y < 0) { y = lastpos; *fallback = true; }
-        fs.ysel = y;
+        ds.ysel = y;
     }
     __syncthreads();
-    int y = fs.ysel;
-    if (y < 0) { y = fs.lastpos; if (tid == 0) *fallback = true; }
+    int y = ds.ysel;
+    if (y < 0) { y = ds.lastpos; if (tid == 0) *fallback = true; }
     return y;
 }
 
+// Mode dispatch (the mode is uniform across the block).
 template <int ESIZE>
-__device__ void finish_row(const VerifyArgs &a, int b, FinSmem &fs) {
+__device__ float segment_total_any(const DrawCtx &c) {
+    if (c.mode == kDrawResidual) return warp_segment_total<ESIZE, kDrawResidual>(c);
+    if (c.mode == kDrawOneHot) return warp_segment_total<ESIZE, kDrawOneHot>(c);
+    return warp_segment_total<ESIZE, kDrawP>(c);
+}
+
+template <int ESIZE>
+__device__ int chunk_locate_any(const DrawCtx &c, float d, DrawSmem &ds, bool *fallback) {
+    if (c.mode == kDrawResidual) return chunk_locate<ESIZE, kDrawResidual>(c, d, ds, fallback);
+    if (c.mode == kDrawOneHot) return chunk_locate<ESIZE, kDrawOneHot>(c, d, ds, fallback);
+    return chunk_locate<ESIZE, kDrawP>(c, d, ds, fallback);
+}
+
+template <int ESIZE>
+__device__ __forceinline__ int chunk_of_element(const VecGeom &g, int x, int U, int C) {
+    constexpr int kPer = 16 / ESIZE;
+    if (x < g.head) return 0;
+    const int u = (x - g.head) / kPer;
+    if (u >= g.n16) return C - 1;
+    return min(u / U, C - 1);
+}
+
+// First chunk whose cumulative mass exceeds t = u * R (R = total mass);
+// *d receives t minus the mass before it.  If rounding leaves t at or past
+// the total, the last chunk with mass is chosen and *d = +inf.  -1 if R == 0.
+__device__ __forceinline__ int select_chunk(const float *cm, int C, float u, float *d) {
+    float R = 0.f;
+    for (int cc = 0; cc < C; ++cc) R += cm[cc];
+    if (!(R > 0.f)) { *d = 0.f; return -1; }
+    const float t = u * R;
+    float pre = 0.f;
+    int lastc = -1;
+    for (int cc = 0; cc < C; ++cc) {
+        if (cm[cc] > 0.f) lastc = cc;
+        if (cm[cc] > t - pre) { *d = t - pre; return cc; }
+        pre += cm[cc];
+    }
+    *d = __int_as_float(0x7f800000);
+    return lastc;
+}
+
+// Same masses, computed by a single thread (rare fallback paths).
+__device__ __forceinline__ void chunk_masses_serial(const VerifyArgs &a, int b, int j, float mj,
+                                                    float k, float *cm) {
+    const long long base = (static_cast<long long>(b) * a.S + j) * a.C * kPartsPerItem;
+    for (int cc = 0; cc < a.C; ++cc) {
+        float t = 0.f;
+        for (int w = 0; w < kPartsPerItem; ++w) {
+            const float4 p = __ldcg(&a.part[base + cc * kPartsPerItem + w]);
+            if (p.x != kNegInf) t += p.y * ex2((p.x - mj) * k);
+        }
+        cm[cc] = t;
+    }
+}
+
+// Mass of p_j per chunk, in units of 2^((z - m_j) k), from the stream
+// partials (sum over the chunk's warp partials).  Thread-parallel over the
+// C * kPartsPerItem partials; the result lands in cm[0..C).
+__device__ __forceinline__ void chunk_masses(const VerifyArgs &a, int b, int j, float mj, float k,
+                                             float *cm) {
+    const int tid = threadIdx.x;
+    const long long base = (static_cast<long long>(b) * a.S + j) * a.C * kPartsPerItem;
+    const int n = a.C * kPartsPerItem;
+    const int lane = tid & 31;
+    for (int q0 = tid - lane; q0 < n; q0 += blockDim.x) {   // warp-uniform trip count
+        const int q = q0 + lane;
+        float t = 0.f;
+        if (q < n) {
+            const float4 p = __ldcg(&a.part[base + q]);
+            if (p.x != kNegInf) t = p.y * ex2((p.x - mj) * k);
+        }
+        // kPartsPerItem (8) consecutive lanes hold one chunk
+#pragma unroll
+        for (int o = 1; o < kPartsPerItem; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+        if (q < n && (q & (kPartsPerItem - 1)) == 0) cm[q / kPartsPerItem] = t;
+    }
+}
+
+// Per-row result of the accept test and the set-up of the final draw.
+struct __align__(16) DrawRecord {
+    int j;        // first rejected position, or L
+    int mode;     // kDrawDone (outputs written), kDrawP, kDrawResidual, kDrawOneHot
+    int csel;     // selected chunk (p-mass modes), -1 if none
+    int xj;       // rejected draft token (one-hot mode)
+    float d;      // target inside the selected chunk (p-mass modes)
+    float u;      // resample uniform
+    float k;      // log2(e) / T
+    float mt, ct, md, cd;
+    int note;     // status note bits to raise
+};
+constexpr int kDrawDone = -1;
+
+// ---------------------------------------------------------------------------
+// 3. Accept kernel: one CTA per row.  Merges the partials into the
+//    normalisers, runs the accept test with Philox uniforms, writes the
+//    outputs of greedy rows, and records the final draw of sampled rows
+//    (for p-mass draws the chunk is already chosen here).
+// ---------------------------------------------------------------------------
+template <int ESIZE>
+__global__ void __launch_bounds__(kDrawThreads) accept_kernel(VerifyArgs a) {
+    __shared__ DrawSmem ds;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int b = blockIdx.x;
     const int K = a.K, S = a.S, C = a.C;
-    const int L = a.lengths[b];
-    const float T = a.temp[b];
+    DrawRecord *rec = a.rec + b;
+    if (__ldg(&a.row_off[b + 1]) == __ldg(&a.row_off[b])) {   // invalid row, already marked
+        if (tid == 0) rec->mode = kDrawDone;
+        return;
+    }
+    const int L = __ldg(&a.lengths[b]);
+    const float T = __ldg(&a.temp[b]);
     const bool greedy = !(T > 0.f);
     const bool has_draft = (a.zd != nullptr) && !greedy;
     const float k = greedy ? 0.f : kLog2e / T;
     const uint64_t row = static_cast<uint64_t>(a.row_base) + static_cast<uint64_t>(b);
     const int nslots = L + 1 + (has_draft ? L : 0);
+    const int nparts = C * kPartsPerItem;
 
-    // Merge the C chunk partials of every vector of the row.
-    for (int q = warp; q < nslots; q += kWarps) {
-        const int slot = q <= L ? q : (K + 1 + (q - L - 1));
-        float m = kNegInf, s = 0.f;
-        int idx = INT_MAX;
-        for (int cc = lane; cc < C; cc += 32) {
-            const float4 p = __ldcg(&a.part[(static_cast<long long>(b) * S + slot) * C + cc]);
-            if (greedy) {
-                const int i2 = __float_as_int(p.z);
-                if (p.x > m || (p.x == m && i2 < idx)) { m = p.x; idx = i2; }
-            } else {
-                lse_merge(m, s, p.x, p.y, k);
+    // Merge the partials of every vector of the row: warp w takes slots
+    // w, w+8, ... in rounds of kRound, issuing a round's loads before any of
+    // its reductions.
+    constexpr int kRound = 4;
+    for (int r0 = 0; warp + r0 * kDrawWarps < nslots; r0 += kRound) {
+        float4 pv[kRound];
+#pragma unroll
+        for (int r = 0; r < kRound; ++r) {
+            const int q = warp + (r0 + r) * kDrawWarps;
+            pv[r] = make_float4(kNegInf, 0.f, __int_as_float(INT_MAX), 0.f);
+            if (q < nslots && lane < nparts) {
+                const int slot = q <= L ? q : (K + 1 + (q - L - 1));
+                pv[r] = __ldcg(&a.part[(static_cast<long long>(b) * S + slot) * nparts + lane]);
             }
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-            const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
-            const int i2 = __shfl_xor_sync(0xffffffffu, idx, o);
-            if (greedy) {
-                if (m2 > m || (m2 == m && i2 < idx)) { m = m2; idx = i2; }
-            } else {
-                lse_merge(m, s, m2, s2, k);
+        for (int r = 0; r < kRound; ++r) {
+            const int q = warp + (r0 + r) * kDrawWarps;
+            if (q >= nslots) break;
+            const int slot = q <= L ? q : (K + 1 + (q - L - 1));
+            float m = pv[r].x, sm = pv[r].y;
+            int idx = __float_as_int(pv[r].z);
+            for (int cc = lane + 32; cc < nparts; cc += 32) {   // C > 4 only
+                const float4 p =
+                    __ldcg(&a.part[(static_cast<long long>(b) * S + slot) * nparts + cc]);
+                if (greedy) {
+                    const int i2 = __float_as_int(p.z);
+                    if (p.x > m || (p.x == m && i2 < idx)) { m = p.x; idx = i2; }
+                } else {
+                    lse_merge(m, sm, p.x, p.y, k);
+                }
             }
-        }
-        if (lane == 0) {
-            if (idx == INT_MAX) idx = 0;   // every logit -inf: documented as invalid input
-            fs.m[slot] = m;
-            fs.s[slot] = greedy ? 1.f : s;
-            fs.arg[slot] = idx;
-            if (a.dbg) {
-                a.dbg[(static_cast<long long>(b) * S + slot) * 2 + 0] = m;
-                a.dbg[(static_cast<long long>(b) * S + slot) * 2 + 1] = greedy ? 1.f : s;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+                const float s2 = __shfl_xor_sync(0xffffffffu, sm, o);
+                const int i2 = __shfl_xor_sync(0xffffffffu, idx, o);
+                if (greedy) {
+                    if (m2 > m || (m2 == m && i2 < idx)) { m = m2; idx = i2; }
+                } else {
+                    lse_merge(m, sm, m2, s2, k);
+                }
+            }
+            if (lane == 0) {
+                if (idx == INT_MAX) idx = 0;   // every logit -inf: documented as invalid input
+                ds.m[slot] = m;
+                ds.s[slot] = greedy ? 1.f : sm;
+                ds.arg[slot] = idx;
+                if (a.dbg) {
+                    a.dbg[(static_cast<long long>(b) * S + slot) * 2 + 0] = m;
+                    a.dbg[(static_cast<long long>(b) * S + slot) * 2 + 1] = greedy ? 1.f : sm;
+                }
             }
         }
     }
-    if (tid == 0) fs.j = L;
+    if (tid == 0) ds.j = L;
     __syncthreads();
 
     // Accept test, one thread per verified position; first rejection wins.
@@ -545,60 +969,200 @@ __device__ void finish_row(const VerifyArgs &a, int b, FinSmem &fs) {
         const int x = a.tokens[static_cast<long long>(b) * K + i];
         bool acc;
         if (greedy) {
-            acc = (x == fs.arg[i]);
+            acc = (x == ds.arg[i]);
         } else {
             const float zt_x = ld_elem<ESIZE>(vec_ptr<ESIZE>(a, b, i), x);
-            const float lp = fmaf(zt_x - fs.m[i], k, -log2f(fs.s[i]));
+            const float lp = fmaf(zt_x - ds.m[i], k, -log2f(ds.s[i]));
             float lq = 0.f;
             if (has_draft) {
                 const float zd_x = ld_elem<ESIZE>(vec_ptr<ESIZE>(a, b, K + 1 + i), x);
-                lq = fmaf(zd_x - fs.m[K + 1 + i], k, -log2f(fs.s[K + 1 + i]));
+                lq = fmaf(zd_x - ds.m[K + 1 + i], k, -log2f(ds.s[K + 1 + i]));
             }
             const float u = uniform24(a.seed, row, static_cast<uint32_t>(i), 0u);
             if (lp == kNegInf) acc = false;
             else if (lq == kNegInf) acc = true;
             else acc = (lp >= lq) || (u < exp2f(lp - lq));
         }
-        if (!acc) atomicMin(&fs.j, i);
+        if (!acc) atomicMin(&ds.j, i);
     }
     __syncthreads();
-    const int j = fs.j;
+    const int j = ds.j;
 
-    int y;
     if (greedy) {
-        y = fs.arg[j];
-    } else {
-        DrawCtx c;
-        c.k = k;
-        c.gt = vec_geom<ESIZE>(vec_ptr<ESIZE>(a, b, j), a.V);
-        c.mt = fs.m[j];
-        c.ct = log2f(fs.s[j]);
-        c.xj = (j < L) ? a.tokens[static_cast<long long>(b) * K + j] : -1;
-        if (j == L) {
-            c.mode = kDrawP;
-        } else if (has_draft) {
-            c.mode = kDrawResidual;
-            c.gd = vec_geom<ESIZE>(vec_ptr<ESIZE>(a, b, K + 1 + j), a.V);
-            c.md = fs.m[K + 1 + j];
-            c.cd = log2f(fs.s[K + 1 + j]);
-        } else {
-            c.mode = kDrawResidualOneHot;
+        const int y = ds.arg[j];
+        for (int t = tid; t <= K; t += kDrawThreads) {
+            int v = -1;
+            if (t < j) v = a.tokens[static_cast<long long>(b) * K + t];
+            else if (t == j) v = y;
+            a.out_tokens[static_cast<long long>(b) * (K + 1) + t] = v;
         }
-        if (c.mode != kDrawResidual) { c.gd = c.gt; c.md = 0.f; c.cd = 0.f; }
-        c.aligned = (c.gd.head == c.gt.head);
-        const float u = uniform24(a.seed, row, static_cast<uint32_t>(j), 1u);
-        bool zero = false, fb = false;
-        y = block_draw<ESIZE>(c, u, fs, &zero, &fb);
-        if (zero) {
-            // Rejection with no residual mass (p_j == q_j to rounding).
-            c.mode = kDrawP;
-            y = block_draw<ESIZE>(c, u, fs, &zero, &fb);
-            if (a.status && tid == 0) atomicOr(a.status, SV_NOTE_ZERO_RESIDUAL);
-            if (y < 0) y = fs.arg[j];
-        }
-        if (fb && a.status) atomicOr(a.status, SV_NOTE_CDF_FALLBACK);
+        if (tid == 0) { a.out_accept[b] = j; rec->mode = kDrawDone; }
+        return;
     }
-    for (int t = tid; t <= K; t += kThreads) {
+
+    // Sampled row: set up the final draw at position j.
+    const bool resid = (j < L) && has_draft;
+    const float mt = ds.m[j];
+    const float u = uniform24(a.seed, row, static_cast<uint32_t>(j), 1u);
+    const int xj = (j < L) ? a.tokens[static_cast<long long>(b) * K + j] : -1;
+    int mode = (j == L) ? kDrawP : (resid ? kDrawResidual : kDrawOneHot);
+    int note = 0;
+    if (!resid) {
+        // p_j (bonus) or p_j without x_j (greedy drafter): chunk masses come
+        // straight from the stream partials.
+        chunk_masses(a, b, j, mt, k, ds.cm);
+        __syncthreads();
+        if (tid == 0 && mode == kDrawOneHot) {
+            const VecGeom g = vec_geom<ESIZE>(vec_ptr<ESIZE>(a, b, j), a.V);
+            const int cx = chunk_of_element<ESIZE>(g, xj, a.U, C);
+            const float wx = ex2((ld_elem<ESIZE>(g.base, xj) - mt) * k);
+            ds.cm[cx] = fmaxf(ds.cm[cx] - wx, 0.f);
+        }
+        __syncthreads();
+        if (tid == 0) {
+            float d = 0.f;
+            int cs = select_chunk(ds.cm, C, u, &d);
+            if (cs < 0) {
+                // p_j one-hot at the rejected x_j (rounding): draw from p_j.
+                mode = kDrawP;
+                note = SV_NOTE_ZERO_RESIDUAL;
+                chunk_masses_serial(a, b, j, mt, k, ds.cm);
+                cs = select_chunk(ds.cm, C, u, &d);
+            }
+            ds.gsel = cs;
+            ds.dsel = d;
+            ds.lastpos = mode;
+        }
+        __syncthreads();
+    }
+    if (tid == 0) {
+        DrawRecord r;
+        r.j = j;
+        r.mode = resid ? kDrawResidual : ds.lastpos;
+        r.csel = resid ? -1 : ds.gsel;
+        r.xj = xj;
+        r.d = resid ? 0.f : ds.dsel;
+        r.u = u;
+        r.k = k;
+        r.mt = mt;
+        r.ct = resid ? log2f(ds.s[j]) : 0.f;
+        r.md = resid ? ds.m[K + 1 + j] : 0.f;
+        r.cd = resid ? log2f(ds.s[K + 1 + j]) : 0.f;
+        r.note = note;
+        *rec = r;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 4. Resample kernel: one CTA per (row, chunk).  p-mass draws: the CTA of
+//    the selected chunk locates the token inside it.  Residual draws: every
+//    chunk CTA sums max(0, p_j - q_j) over its chunk by segments; the last
+//    one (atomic counter, no waiting) selects the chunk and the segment from
+//    those sums and locates the token.
+// ---------------------------------------------------------------------------
+template <int ESIZE>
+__global__ void __launch_bounds__(kDrawThreads, 3) resample_kernel(VerifyArgs a) {
+    __shared__ DrawSmem ds;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int b = blockIdx.x / a.C;
+    const int chunk = blockIdx.x - b * a.C;
+    const int K = a.K, C = a.C;
+    const DrawRecord r = a.rec[b];   // written by the previous launch
+    if (r.mode == kDrawDone) return;
+    const bool resid = r.mode == kDrawResidual;
+    if (!resid && chunk != (r.csel < 0 ? 0 : r.csel)) return;
+    const int j = r.j;
+
+    DrawCtx c;
+    c.k = r.k;
+    c.mode = r.mode;
+    c.gt = vec_geom<ESIZE>(vec_ptr<ESIZE>(a, b, j), a.V);
+    c.mt = r.mt;
+    c.ct = r.ct;
+    c.xj = r.xj;
+    if (resid) {
+        c.gd = vec_geom<ESIZE>(vec_ptr<ESIZE>(a, b, K + 1 + j), a.V);
+        c.md = r.md;
+        c.cd = r.cd;
+    } else {
+        c.gd = c.gt; c.md = 0.f; c.cd = 0.f;
+    }
+    c.aligned = (c.gd.head == c.gt.head);
+    auto set_chunk = [&](int cc) {
+        c.ubody0 = cc * a.U;
+        c.nbody = max(0, min(c.ubody0 + a.U, c.gt.n16) - c.ubody0);
+        c.has_head = (cc == 0);
+        c.has_tail = (cc == C - 1);
+    };
+    int note = r.note;
+    int csel = r.csel;
+    float d = r.d;
+    bool have_segments = false;
+    if (resid) {
+        set_chunk(chunk);
+        const float segtot = warp_segment_total<ESIZE, kDrawResidual>(c);
+        if (lane == 0)
+            a.rseg[(static_cast<long long>(b) * C + chunk) * kDrawWarps + warp] = segtot;
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) {
+            const int done = atomicAdd(&a.rcnt[b], 1) + 1;
+            __threadfence();
+            ds.last = (done == C);
+        }
+        __syncthreads();
+        if (!ds.last) return;
+        if (tid < C) {
+            float t = 0.f;
+            for (int g = 0; g < kDrawWarps; ++g)
+                t += __ldcg(&a.rseg[(static_cast<long long>(b) * C + tid) * kDrawWarps + g]);
+            ds.cm[tid] = t;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            float dd = 0.f;
+            int cs = select_chunk(ds.cm, C, r.u, &dd);
+            int m = kDrawResidual;
+            if (cs < 0) {
+                // The residual vanished to rounding (p_j == q_j): draw from p_j.
+                m = kDrawP;
+                note |= SV_NOTE_ZERO_RESIDUAL;
+                chunk_masses_serial(a, b, j, r.mt, r.k, ds.cm);
+                cs = select_chunk(ds.cm, C, r.u, &dd);
+            }
+            ds.gsel = cs;
+            ds.dsel = dd;
+            ds.lastpos = m;
+        }
+        __syncthreads();
+        csel = ds.gsel;
+        d = ds.dsel;
+        if (ds.lastpos == kDrawP) {
+            c.mode = kDrawP;
+            c.ct = 0.f;
+        } else {
+            have_segments = true;
+        }
+    }
+    int y = -1;
+    bool fb = false;
+    if (csel >= 0) {
+        set_chunk(csel);
+        if (have_segments) {
+            if (tid < kDrawWarps)
+                ds.wsum[tid] =
+                    __ldcg(&a.rseg[(static_cast<long long>(b) * C + csel) * kDrawWarps + tid]);
+        } else {
+            const float segtot = segment_total_any<ESIZE>(c);
+            if (lane == 0) ds.wsum[warp] = segtot;
+        }
+        __syncthreads();
+        y = chunk_locate_any<ESIZE>(c, d, ds, &fb);
+    }
+    if (y < 0) { y = 0; fb = true; }
+    if (fb) note |= SV_NOTE_CDF_FALLBACK;
+    if (tid == 0 && a.status && note) atomicOr(a.status, note);
+    for (int t = tid; t <= K; t += kDrawThreads) {
         int v = -1;
         if (t < j) v = a.tokens[static_cast<long long>(b) * K + t];
         else if (t == j) v = y;
@@ -607,76 +1171,8 @@ __device__ void finish_row(const VerifyArgs &a, int b, FinSmem &fs) {
     if (tid == 0) a.out_accept[b] = j;
 }
 
-// ---------------------------------------------------------------------------
-// 2c. Persistent kernel.
-// ---------------------------------------------------------------------------
-template <int ESIZE>
-__global__ void __launch_bounds__(kThreads, 2) verify_kernel(VerifyArgs a) {
-    __shared__ float s_red_m[kWarps];
-    __shared__ float s_red_s[kWarps];
-    __shared__ int s_red_i[kWarps];
-    __shared__ int s_w, s_b, s_last;
-    __shared__ FinSmem fs;
-    const int tid = threadIdx.x;
-    const int total = __ldcg(&a.ctr[1]);
-
-    if (tid == 0) {
-        const int w = atomicAdd(&a.ctr[0], 1);
-        s_w = w;
-        if (w < total) {
-            int lo = 0, hi = a.B - 1;   // largest b with row_off[b] <= w
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (__ldcg(&a.row_off[mid]) <= w) lo = mid; else hi = mid - 1;
-            }
-            s_b = lo;
-        }
-    }
-    __syncthreads();
-    while (true) {
-        const int w = s_w;
-        if (w >= total) break;
-        const int b = s_b;
-        const int off = __ldcg(&a.row_off[b]);
-        const int nitems = __ldcg(&a.row_off[b + 1]) - off;
-        const int r = w - off;
-        const int L = a.lengths[b];
-        const float T = a.temp[b];
-        const bool greedy = !(T > 0.f);
-        const int q = r / a.C, chunk = r - q * a.C;
-        const int slot = q <= L ? q : (a.K + 1 + (q - L - 1));
-        const float k = greedy ? 0.f : kLog2e / T;
-        int wnext = 0;
-        if (tid == 0) wnext = atomicAdd(&a.ctr[0], 1);   // consumed after the item
-
-        const ItemResult res = process_item<ESIZE>(a, vec_ptr<ESIZE>(a, b, slot), chunk, greedy, k,
-                                                   s_red_m, s_red_s, s_red_i);
-        if (tid == 0) {
-            a.part[(static_cast<long long>(b) * a.S + slot) * a.C + chunk] =
-                make_float4(res.m, res.s, __int_as_float(res.idx), 0.f);
-            __threadfence();
-            const int done = atomicAdd(&a.row_cnt[b], 1) + 1;
-            __threadfence();
-            s_last = (done == nitems);
-            s_w = wnext;
-            if (wnext < total) {
-                int lo = 0, hi = a.B - 1;
-                while (lo < hi) {
-                    const int mid = (lo + hi + 1) >> 1;
-                    if (__ldcg(&a.row_off[mid]) <= wnext) lo = mid; else hi = mid - 1;
-                }
-                s_b = lo;
-            }
-        }
-        __syncthreads();
-        if (s_last) finish_row<ESIZE>(a, b, fs);
-        __syncthreads();
-    }
-}
-
-// Kernel launched per call, used for occupancy queries.
-template <int ESIZE> static const void *verify_kernel_ptr() {
-    return reinterpret_cast<const void *>(&verify_kernel<ESIZE>);
+template <int ESIZE> static const void *stream_kernel_ptr() {
+    return reinterpret_cast<const void *>(&stream_kernel<ESIZE>);
 }
 
 // ---------------------------------------------------------------------------
@@ -684,7 +1180,7 @@ template <int ESIZE> static const void *verify_kernel_ptr() {
 // ---------------------------------------------------------------------------
 struct Plan {
     int C, U, S;
-    size_t off_rowcnt, off_rowoff, off_part, bytes;
+    size_t off_rcnt, off_rowoff, off_part, off_rseg, off_rec, bytes;
 };
 
 static bool make_plan(int B, int K, int V, sv_dtype dtype, Plan *p) {
@@ -695,24 +1191,30 @@ static bool make_plan(int B, int K, int V, sv_dtype dtype, Plan *p) {
     const long long n16 = (V + per - 1) / per;
     int C = static_cast<int>((n16 + kMaxUnitsPerItem - 1) / kMaxUnitsPerItem);
     if (C < 1) C = 1;
+    if (C > kMaxChunks) return false;
     const int U = static_cast<int>((n16 + C - 1) / C);
     const int S = 2 * K + 1;
     const long long items = static_cast<long long>(B) * S * C;
-    if (items >= INT_MAX / 2) return false;
+    if (items >= INT_MAX / 2 || static_cast<long long>(B) * C >= INT_MAX / 2) return false;
     p->C = C; p->U = U; p->S = S;
     size_t off = 16;
-    p->off_rowcnt = off;
+    p->off_rcnt = off;
     off += sizeof(int) * static_cast<size_t>(B);
     p->off_rowoff = off;
     off += sizeof(int) * static_cast<size_t>(B + 1);
     off = (off + 15) & ~static_cast<size_t>(15);
     p->off_part = off;
-    off += sizeof(float4) * static_cast<size_t>(items);
-    p->bytes = off;
+    off += sizeof(float4) * static_cast<size_t>(items) * kPartsPerItem;
+    p->off_rseg = off;
+    off += sizeof(float) * static_cast<size_t>(B) * C * kDrawWarps;
+    off = (off + 15) & ~static_cast<size_t>(15);
+    p->off_rec = off;
+    off += sizeof(DrawRecord) * static_cast<size_t>(B);
+    p->bytes = (off + 15) & ~static_cast<size_t>(15);
     return true;
 }
 
-static int grid_for(int esize, long long max_items) {
+static int stream_grid(int esize, long long max_items) {
     static int cache[2][64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return -1;
@@ -721,8 +1223,12 @@ static int grid_for(int esize, long long max_items) {
         int sms = 0, per = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return -1;
-        const void *fn = esize == 4 ? verify_kernel_ptr<4>() : verify_kernel_ptr<2>();
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fn, kThreads, 0) != cudaSuccess)
+        const void *fn = esize == 4 ? stream_kernel_ptr<4>() : stream_kernel_ptr<2>();
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kRingBytes) !=
+            cudaSuccess)
+            return -1;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fn, kBlock, kRingBytes) !=
+            cudaSuccess)
             return -1;
         slot = sms * (per > 0 ? per : 1);
     }
@@ -755,18 +1261,28 @@ static sv_status verify_impl(const void *zt, const void *zd, sv_dtype dtype, int
     a.out_tokens = out_tokens; a.out_accept = out_accept; a.status = status; a.dbg = dbg;
     char *w = static_cast<char *>(ws);
     a.ctr = reinterpret_cast<int *>(w);
-    a.row_cnt = reinterpret_cast<int *>(w + p.off_rowcnt);
+    a.rcnt = reinterpret_cast<int *>(w + p.off_rcnt);
     a.row_off = reinterpret_cast<int *>(w + p.off_rowoff);
     a.part = reinterpret_cast<float4 *>(w + p.off_part);
+    a.rseg = reinterpret_cast<float *>(w + p.off_rseg);
+    a.rec = reinterpret_cast<DrawRecord *>(w + p.off_rec);
 
-    const int grid = grid_for(es, static_cast<long long>(B) * p.S * p.C);
+    const int grid = stream_grid(es, static_cast<long long>(B) * p.S * p.C);
     if (grid <= 0) return note_cuda(cudaGetLastError());
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     prologue_kernel<<<1, kPrologueThreads, 0, st>>>(a);
     profile_mark_begin(st);
-    if (es == 4) verify_kernel<4><<<grid, kThreads, 0, st>>>(a);
-    else verify_kernel<2><<<grid, kThreads, 0, st>>>(a);
+    if (es == 4) stream_kernel<4><<<grid, kBlock, kRingBytes, st>>>(a);
+    else stream_kernel<2><<<grid, kBlock, kRingBytes, st>>>(a);
     profile_mark_end(st);
+    const unsigned draw_grid = static_cast<unsigned>(B) * static_cast<unsigned>(p.C);
+    if (es == 4) {
+        accept_kernel<4><<<B, kDrawThreads, 0, st>>>(a);
+        resample_kernel<4><<<draw_grid, kDrawThreads, 0, st>>>(a);
+    } else {
+        accept_kernel<2><<<B, kDrawThreads, 0, st>>>(a);
+        resample_kernel<2><<<draw_grid, kDrawThreads, 0, st>>>(a);
+    }
     return note_cuda(cudaGetLastError());
 }
 
@@ -802,4 +1318,4 @@ extern "C" sv_status sv_verify_debug(const void *target_logits, const void *draf
                            workspace_bytes, status, stats_out, stream);
 }
 
-extern "C" int sv_verify_launches(void) { return 2; }
+extern "C" int sv_verify_launches(void) { return 4; }
