@@ -186,6 +186,38 @@ sv_status sv_verify_debug(const void *target_logits, const void *draft_logits, s
                           float *stats_out, void *stream);
 
 /*
+ * sv_verify_noalloc -- sv_verify without a caller-provided workspace.
+ *
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory when they verify: a serving loop that
+ * plans all of its memory up front and forbids allocation afterwards, a
+ * plain C host program with no device allocator of its own, or code that
+ * must not touch the allocator while other work is in flight.  The scratch
+ * that sv_verify takes as `workspace` lives instead in one fixed device
+ * array inside this library, 16 MiB per GPU, which every GPU that loads the
+ * library holds until the process exits.
+ *
+ *   Arguments and results are those of sv_verify, minus workspace and
+ *   workspace_bytes.  Batches whose sv_verify_workspace_bytes(B, K, V, dtype)
+ *   exceeds 16 MiB (16777216 bytes) are rejected with SV_ERR_WORKSPACE
+ *   before anything is launched; use sv_verify with a workspace for those.
+ *   The library calls no cudaMalloc, cudaFree or other allocating routine.
+ *   The first call on a device looks up the array's device address (once
+ *   per device, thread-safe); make that first call before any stream
+ *   capture.  Every call shares the one array and leaves its contents
+ *   behind: counters that must start at zero are reset by each call's
+ *   first kernel, everything else is written before it is read.  Calls
+ *   whose work overlaps on the GPU (other streams, other host threads on the
+ *   same device) race on the array; order them on one stream.
+ */
+sv_status sv_verify_noalloc(const void *target_logits, const void *draft_logits, sv_dtype dtype,
+                            int B, int K, int V,
+                            const int32_t *draft_tokens, const int32_t *lengths,
+                            const float *temperature, uint64_t seed, int64_t row_base,
+                            int32_t *out_tokens, int32_t *out_accept_len, int32_t *status,
+                            void *stream);
+
+/*
  * sv_philox_uniforms -- the uniforms sv_verify draws, for tests:
  * out[k] = u(seed, row[k], pos[k], draw[k]) as defined above.
  * row: device int64 [n] (>= 0); pos, draw: device int32 [n]; out: device

@@ -51,6 +51,8 @@ def lib():
                             vp]
     L.sv_verify_debug.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, u64, i64, vp, vp, vp,
                                   sz, vp, vp, vp]
+    L.sv_verify_noalloc.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, u64, i64, vp, vp, vp,
+                                    vp]
     L.sv_philox_uniforms.argtypes = [u64, vp, vp, vp, i32, vp, vp]
     L.sv_philox4x32_10.argtypes = [vp, vp, i32, vp, vp]
     L.sv_profile_begin.argtypes = [i32]
@@ -58,7 +60,8 @@ def lib():
     L.sv_profile_read.restype = i32
     L.sv_status_string.argtypes = [i32]
     L.sv_status_string.restype = ctypes.c_char_p
-    for name in ("sv_schedule", "sv_verify", "sv_verify_debug", "sv_philox_uniforms",
+    for name in ("sv_schedule", "sv_verify", "sv_verify_debug", "sv_verify_noalloc",
+                 "sv_philox_uniforms",
                  "sv_philox4x32_10", "sv_profile_begin"):
         getattr(L, name).restype = i32
     L.sv_last_cuda_error.restype = i32
@@ -146,6 +149,18 @@ def sv_verify_debug(target_logits, draft_logits, draft_tokens, lengths, temperat
         _ptr(temperature), ctypes.c_uint64(seed & (2**64 - 1)), int(row_base), _ptr(out_tokens),
         _ptr(out_accept_len), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _ptr(status), _ptr(stats_out), _stream(stream, target_logits)))
+
+
+def sv_verify_noalloc(target_logits, draft_logits, draft_tokens, lengths, temperature, seed: int,
+                      out_tokens, out_accept_len, status=None, row_base: int = 0,
+                      stream=None) -> None:
+    """sv_verify with the library's own fixed scratch instead of a workspace,
+    for callers that must not allocate device memory (see include/sv.h)."""
+    B, K, V, dt = _verify_args(target_logits, draft_logits, draft_tokens, lengths, temperature)
+    _check("sv_verify_noalloc", lib().sv_verify_noalloc(
+        _ptr(target_logits), _ptr(draft_logits), dt, B, K, V, _ptr(draft_tokens), _ptr(lengths),
+        _ptr(temperature), ctypes.c_uint64(seed & (2**64 - 1)), int(row_base), _ptr(out_tokens),
+        _ptr(out_accept_len), _ptr(status), _stream(stream, target_logits)))
 
 
 def sv_philox_uniforms(seed: int, row, pos, draw, out, stream=None) -> None:

@@ -42,6 +42,7 @@
 #include <climits>
 #include <cstdint>
 #include <cstdio>
+#include <mutex>
 
 #include "sv.h"
 #include "sv_device.cuh"
@@ -1319,3 +1320,60 @@ extern "C" sv_status sv_verify_debug(const void *target_logits, const void *draf
 }
 
 extern "C" int sv_verify_launches(void) { return 4; }
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant: the scratch lives in a fixed device array that
+// the library owns, so callers that must not allocate device memory can
+// still verify.  The array is sized for moderate batches; larger ones must
+// use sv_verify with their own workspace.
+// ---------------------------------------------------------------------------
+namespace sv {
+
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;   // 16 MiB per device
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+static std::mutex g_static_scratch_mu;
+static void *g_static_scratch_addr[64];
+
+// Device address of g_static_scratch on the current device.  In host code
+// the symbol names only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+static sv_status static_scratch_address(void **out) {
+    int dev = 0;
+    const cudaError_t e0 = cudaGetDevice(&dev);
+    if (e0 != cudaSuccess) return note_cuda(e0);
+    if (dev < 0 || dev >= 64) return SV_ERR_ARG;
+    std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+    if (g_static_scratch_addr[dev] == nullptr) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+        if (e != cudaSuccess || p == nullptr) return note_cuda(e != cudaSuccess ? e : cudaErrorUnknown);
+        g_static_scratch_addr[dev] = p;
+    }
+    *out = g_static_scratch_addr[dev];
+    return SV_OK;
+}
+
+}  // namespace sv
+
+extern "C" sv_status sv_verify_noalloc(const void *target_logits, const void *draft_logits,
+                                       sv_dtype dtype, int B, int K, int V,
+                                       const int32_t *draft_tokens, const int32_t *lengths,
+                                       const float *temperature, uint64_t seed, int64_t row_base,
+                                       int32_t *out_tokens, int32_t *out_accept_len,
+                                       int32_t *status, void *stream) {
+    if (!target_logits || !draft_tokens || !lengths || !temperature || !out_tokens ||
+        !out_accept_len)
+        return SV_ERR_ARG;
+    const size_t need = sv_verify_workspace_bytes(B, K, V, dtype);
+    if (need == 0) return (dtype != SV_F32 && dtype != SV_BF16) ? SV_ERR_DTYPE : SV_ERR_SHAPE;
+    if (need > sv::kStaticScratchBytes) return SV_ERR_WORKSPACE;
+    void *ws = nullptr;
+    const sv_status st = sv::static_scratch_address(&ws);
+    if (st != SV_OK) return st;
+    // The counters that must start at zero are reset by the first kernel of
+    // every call; everything else in the scratch is written before it is read.
+    return sv::verify_impl(target_logits, draft_logits, dtype, B, K, V, draft_tokens, lengths,
+                           temperature, seed, row_base, out_tokens, out_accept_len, ws,
+                           sv::kStaticScratchBytes, status, nullptr, stream);
+}
