@@ -44,6 +44,7 @@ sys.path.insert(0, ROOT)
 
 import speculative_decoding_verification_93_b200 as sv  # noqa: E402
 from speculative_decoding_verification_93_b200 import workloads  # noqa: E402
+from speculative_decoding_verification_93_b200.sharding import max_over_ranks  # noqa: E402
 
 METRIC = "verified draft positions/sec and achieved HBM GB/s (% of B200 peak) at B×K×V"
 UNIT = "positions/s"
@@ -51,7 +52,7 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["speculative_decoding_verification_93_b200/csrc/sv_verify.cu",
                   "speculative_decoding_verification_93_b200/csrc/sv_device.cuh"]
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "verify_kernel_c2_traffic.md")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "stream_kernel_c2.md")
 
 
 def kernel_hash() -> str:
@@ -242,10 +243,7 @@ def run_ours(args, rank, world, local_rank):
     kernel_ms = sv.sv_profile_read(args.steps)
     sv.sv_profile_begin(0)
     clk = clocks.stop() if rank == 0 else None
-    if dist:
-        t = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, dev)
     ms_step = ms_total / args.steps
     value = positions * world / (ms_step / 1e3)
     st = int(status.item())
@@ -292,10 +290,7 @@ def run_ours(args, rank, world, local_rank):
         e1.record(stream)
         torch.cuda.synchronize()
         ms_e2e = e0.elapsed_time(e1)
-        if dist:
-            t = torch.tensor([ms_e2e], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
+        ms_e2e = max_over_ranks(ms_e2e, dev)
         e2e = {"value": positions * world / (ms_e2e / e2e_steps / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": e2e_steps}
@@ -311,7 +306,7 @@ def run_ours(args, rank, world, local_rank):
                 "frac": round(achieved / peak, 4), "traffic": traffic,
                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src ==
                 "measured" else "fallback 6650 GB/s",
-                "kernel": "sv::verify_kernel", "kernel_ms": round(avg_kernel_ms, 5),
+                "kernel": "sv::stream_kernel", "kernel_ms": round(avg_kernel_ms, 5),
                 "algorithmic_bytes_per_launch": alg_bytes,
                 "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
                 "step_gbs": round(alg_bytes / (ms_step / 1e3) / 1e9, 1)}
