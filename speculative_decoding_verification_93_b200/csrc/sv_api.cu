@@ -31,6 +31,8 @@ sv_status note_cuda(cudaError_t e) {
 // ---------------------------------------------------------------------------
 __global__ void schedule_kernel(const float *__restrict__ conf, int B, int K, float tau,
                                 int32_t *__restrict__ lengths) {
+    griddep_wait();                 // the previous step may still read `lengths`
+    griddep_launch_dependents();    // the verification prologue may launch now
     for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < B; b += gridDim.x * blockDim.x) {
         const float *c = conf + static_cast<long long>(b) * K;
         float S = 1.f;
@@ -101,9 +103,9 @@ extern "C" sv_status sv_schedule(const float *conf, int B, int K, float load, in
     const int threads = 256;
     int blocks = (B + threads - 1) / threads;
     if (blocks > 65535) blocks = 65535;
-    sv::schedule_kernel<<<blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(conf, B, K,
-                                                                                   load, lengths);
-    return sv::note_cuda(cudaGetLastError());
+    return sv::note_cuda(sv::launch_pdl(sv::schedule_kernel, dim3(blocks), dim3(threads), 0,
+                                        static_cast<cudaStream_t>(stream), conf, B, K, load,
+                                        lengths));
 }
 
 extern "C" sv_status sv_philox_uniforms(uint64_t seed, const int64_t *row, const int32_t *pos,

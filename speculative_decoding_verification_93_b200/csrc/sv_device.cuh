@@ -249,4 +249,17 @@ __device__ __forceinline__ void group_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(N) : "memory");
 }
 
+// Programmatic dependent launch (sm_90+): a kernel launched with
+// programmatic stream serialisation may start before the previous kernel in
+// the stream has finished; griddep_wait() blocks until that kernel has
+// completed and its writes are visible, and must precede every global
+// access that could conflict with it.  griddep_launch_dependents() lets the
+// next kernel start launching early.
+__device__ __forceinline__ void griddep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 }  // namespace sv

@@ -117,6 +117,8 @@ __global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(VerifyArgs a
     __shared__ int s_warp[kPrologueThreads / 32];
     __shared__ int s_carry;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    griddep_wait();
+    griddep_launch_dependents();   // the stream kernel may take its SMs now
     if (tid == 0) s_carry = 0;
     __syncthreads();
     for (int base = 0; base < a.B; base += kPrologueThreads) {
@@ -455,12 +457,15 @@ __global__ void __launch_bounds__(kBlock, 3) stream_kernel(VerifyArgs a) {
         fence_mbar_init();
     }
     __syncthreads();
+    griddep_wait();
     const int total = __ldcg(&a.ctr[1]);
     if (tid >= kConsumers) {
         if (tid == kConsumers) producer<ESIZE>(a, sm, ring, total);
         return;
     }
     consumers<ESIZE>(a, sm, ring);
+    // This CTA has no work left: the accept kernel may start launching.
+    griddep_launch_dependents();
 }
 
 // ---------------------------------------------------------------------------
@@ -890,6 +895,8 @@ template <int ESIZE>
 __global__ void __launch_bounds__(kDrawThreads) accept_kernel(VerifyArgs a) {
     __shared__ DrawSmem ds;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    griddep_wait();
+    griddep_launch_dependents();   // resample CTAs wait for this grid anyway
     const int b = blockIdx.x;
     const int K = a.K, S = a.S, C = a.C;
     DrawRecord *rec = a.rec + b;
@@ -1065,6 +1072,7 @@ template <int ESIZE>
 __global__ void __launch_bounds__(kDrawThreads, 3) resample_kernel(VerifyArgs a) {
     __shared__ DrawSmem ds;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    griddep_wait();
     const int b = blockIdx.x / a.C;
     const int chunk = blockIdx.x - b * a.C;
     const int K = a.K, C = a.C;
@@ -1102,9 +1110,10 @@ __global__ void __launch_bounds__(kDrawThreads, 3) resample_kernel(VerifyArgs a)
     if (resid) {
         set_chunk(chunk);
         const float segtot = warp_segment_total<ESIZE, kDrawResidual>(c);
-        if (lane == 0)
+        if (lane == 0) {
             a.rseg[(static_cast<long long>(b) * C + chunk) * kDrawWarps + warp] = segtot;
-        __threadfence();
+            __threadfence();
+        }
         __syncthreads();
         if (tid == 0) {
             const int done = atomicAdd(&a.rcnt[b], 1) + 1;
@@ -1271,19 +1280,28 @@ static sv_status verify_impl(const void *zt, const void *zd, sv_dtype dtype, int
     const int grid = stream_grid(es, static_cast<long long>(B) * p.S * p.C);
     if (grid <= 0) return note_cuda(cudaGetLastError());
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    prologue_kernel<<<1, kPrologueThreads, 0, st>>>(a);
+    // Every launch below may overlap the tail of the one before it
+    // (programmatic dependent launch); each kernel waits for its
+    // predecessor before touching global memory.  Profiling events, when
+    // enabled, sit between launches and serialise them as usual.
+    cudaError_t e = launch_pdl(prologue_kernel, dim3(1), dim3(kPrologueThreads), 0, st, a);
+    if (e != cudaSuccess) return note_cuda(e);
     profile_mark_begin(st);
-    if (es == 4) stream_kernel<4><<<grid, kBlock, kRingBytes, st>>>(a);
-    else stream_kernel<2><<<grid, kBlock, kRingBytes, st>>>(a);
+    e = (es == 4) ? launch_pdl(stream_kernel<4>, dim3(grid), dim3(kBlock), kRingBytes, st, a)
+                  : launch_pdl(stream_kernel<2>, dim3(grid), dim3(kBlock), kRingBytes, st, a);
+    if (e != cudaSuccess) return note_cuda(e);
     profile_mark_end(st);
     const unsigned draw_grid = static_cast<unsigned>(B) * static_cast<unsigned>(p.C);
     if (es == 4) {
-        accept_kernel<4><<<B, kDrawThreads, 0, st>>>(a);
-        resample_kernel<4><<<draw_grid, kDrawThreads, 0, st>>>(a);
+        e = launch_pdl(accept_kernel<4>, dim3(B), dim3(kDrawThreads), 0, st, a);
+        if (e == cudaSuccess)
+            e = launch_pdl(resample_kernel<4>, dim3(draw_grid), dim3(kDrawThreads), 0, st, a);
     } else {
-        accept_kernel<2><<<B, kDrawThreads, 0, st>>>(a);
-        resample_kernel<2><<<draw_grid, kDrawThreads, 0, st>>>(a);
+        e = launch_pdl(accept_kernel<2>, dim3(B), dim3(kDrawThreads), 0, st, a);
+        if (e == cudaSuccess)
+            e = launch_pdl(resample_kernel<2>, dim3(draw_grid), dim3(kDrawThreads), 0, st, a);
     }
+    if (e != cudaSuccess) return note_cuda(e);
     return note_cuda(cudaGetLastError());
 }
 
