@@ -137,13 +137,25 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
-def algorithmic_bytes(lengths: np.ndarray, temperature: np.ndarray, V: int, esize: int,
-                      has_draft: bool = True) -> int:
-    """Logit bytes the verification must stream once: per row
+def scheduled_bytes(lengths: np.ndarray, temperature: np.ndarray, V: int, esize: int,
+                    has_draft: bool = True) -> int:
+    """Logit bytes of every scheduled vector: per row
     esize * V * ((L + 1) target vectors + L draft vectors if T > 0)."""
     L = lengths.astype(np.int64)
     drafts = np.where((temperature > 0) & has_draft, L, 0)
     return int((esize * V * ((L + 1) + drafts)).sum())
+
+
+def needed_bytes(accept: np.ndarray, lengths: np.ndarray, temperature: np.ndarray, V: int,
+                 esize: int, has_draft: bool = True) -> int:
+    """Logit bytes the outcome depends on, i.e. what verification must read
+    once: target positions 0..a and, for sampled rows, draft positions
+    0..min(a, L-1), where a is the accepted length (the first rejection, or
+    L).  Positions after the first rejection never change the output."""
+    a = accept.astype(np.int64)
+    L = lengths.astype(np.int64)
+    drafts = np.where((temperature > 0) & has_draft, np.minimum(a + 1, L), 0)
+    return int((esize * V * ((a + 1) + drafts)).sum())
 
 
 def oracle_sample(batch, lengths_np, budget_s: float, seed0: int = 0):
@@ -218,7 +230,7 @@ def run_ours(args, rank, world, local_rank):
     lengths_np = ln_buf.cpu().numpy()
     temp_np = batch.temperature.cpu().numpy()
     positions = int(lengths_np.sum())
-    alg_bytes = algorithmic_bytes(lengths_np, temp_np, V, esize)
+    sched_bytes = scheduled_bytes(lengths_np, temp_np, V, esize)
 
     # ---- device-timed region ------------------------------------------------
     clocks = ClockSampler(local_rank)
@@ -251,12 +263,36 @@ def run_ours(args, rank, world, local_rank):
     # from overlapping, which costs the step about 10 us) -------------------
     sv.sv_profile_begin(args.steps)
     torch.cuda.synchronize()
+    need = []
     for i in range(args.steps):
         step(args.warmup + args.steps + i, batch.zt, batch.zd, batch.tokens, batch.temperature,
              batch.conf, ln_buf)
+        need.append(needed_bytes(out_acc.cpu().numpy(), lengths_np, temp_np, V, esize))
     torch.cuda.synchronize()
     kernel_ms = sv.sv_profile_read(args.steps)
     sv.sv_profile_begin(0)
+    alg_bytes = sum(need) / len(need)
+
+    # ---- hardware-aware admission on the same confidences (next row of the
+    # scheduler): a profiled speed table of the shape steps/s = s0/(1+n/n0) -------
+    admit = None
+    if rank == 0:
+        n_tab = torch.arange(B * (K + 1) + 2, device=dev, dtype=torch.float32)
+        speed_tab = (1000.0 / (1.0 + n_tab / (4.0 * B))).contiguous()
+        adm_len = torch.empty(B, dtype=torch.int32, device=dev)
+        adm_tau = torch.empty(1, dtype=torch.float32, device=dev)
+        for _ in range(3):
+            sv.sv_schedule_admit(batch.conf, speed_tab, adm_len, adm_tau)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            sv.sv_schedule_admit(batch.conf, speed_tab, adm_len, adm_tau)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        admit = {"kernel": "sv::admit_kernel", "us_per_call": round(e0.elapsed_time(e1) /
+                                                                   args.steps * 1e3, 2),
+                 "candidates": B * K, "admitted": int(adm_len.sum().item()),
+                 "tau": round(float(adm_tau.item()), 6), "bound": "latency (one CTA)"}
 
     # ---- end-to-end through host buffers ------------------------------------
     e2e = None
@@ -310,16 +346,25 @@ def run_ours(args, rank, world, local_rank):
     peak, peak_src = measured_hbm_peak()
     kms = [t for t in kernel_ms if t > 0]
     avg_kernel_ms = sum(kms) / len(kms) if kms else float("nan")
-    achieved = alg_bytes / (avg_kernel_ms / 1e3) / 1e9
+    # achieved: per launch, the bytes that launch's outcome depends on over
+    # its own duration, averaged
+    achieved = (sum(nb / (t / 1e3) for nb, t in zip(need, kernel_ms) if t > 0) / len(kms) / 1e9
+                if kms else float("nan"))
     traffic = committed_traffic()
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src ==
                 "measured" else "fallback 6650 GB/s",
                 "kernel": "sv::stream_kernel", "kernel_ms": round(avg_kernel_ms, 5),
-                "algorithmic_bytes_per_launch": alg_bytes,
+                "algorithmic_bytes_per_launch": int(alg_bytes),
+                "algorithmic_bytes": "logits the outcome depends on: target positions 0..a and "
+                                     "draft positions 0..min(a, L-1) per row (a = accepted "
+                                     "length); the kernel skips positions after a row's first "
+                                     "rejection once it is known",
+                "scheduled_bytes_per_launch": sched_bytes,
                 "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
                 "step_gbs": round(alg_bytes / (ms_step / 1e3) / 1e9, 1),
+                "scheduled_step_gbs": round(sched_bytes / (ms_step / 1e3) / 1e9, 1),
                 "kernel_timing": "CUDA events around each stream-kernel launch over a second "
                                  "timed pass of the same steps"}
 
@@ -336,7 +381,7 @@ def run_ours(args, rank, world, local_rank):
                               parallelism=f"dp{world} (row shards, no collective)"),
                "e2e": e2e, "gpu_launches": args.steps * (sv.sv_verify_launches()
                                                          + (1 if fixed is None else 0)),
-               "roofline": roofline, "cpu_baseline": cpu, "clocks": clk,
+               "roofline": roofline, "cpu_baseline": cpu, "clocks": clk, "admission": admit,
                "device_status": st, "impl": "ours"}
         print(json.dumps(out), flush=True)
     del batch

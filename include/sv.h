@@ -55,6 +55,7 @@ typedef enum { SV_F32 = 0, SV_BF16 = 1 } sv_dtype;
 /* Supported sizes. */
 #define SV_MAX_K  64
 #define SV_MAX_V  (1 << 20)
+#define SV_MAX_ADMIT 8192   /* B * K candidates for sv_schedule_admit */
 
 /*
  * sv_schedule -- per-row verify length from prefix survival.
@@ -88,6 +89,44 @@ typedef enum { SV_F32 = 0, SV_BF16 = 1 } sv_dtype;
  */
 sv_status sv_schedule(const float *conf, int B, int K, float load,
                       int32_t *lengths, void *stream);
+
+/*
+ * sv_schedule_admit -- per-row verify lengths by hardware-aware admission.
+ *
+ * Defined by: umans.ai, "DeepSeek V4 Pro DSpark: the model isn't ready, the
+ * architecture is", section "What DSpark adds", item "2. Verify smarter"
+ * (profile the engine's steps per second as a function of batch size; every
+ * step, sort every candidate token of every request by survival
+ * probability, admit them one at a time, and stop the moment expected
+ * accepted tokens times the speed at that batch size stops rising);
+ * techvisionai "DeepSeek-V4: Breaking the Efficiency Barrier", Ch. 7
+ * "Hardware-Aware Scheduling"; zhichai.net DSpark topic, "Under the hood".
+ *
+ * Per row, S_i = prod_{j<=i} clamp(conf[b, j-1], 0, 1) (NaN counts as 0),
+ * computed in fp64.  Candidates (b, i) are taken in order of S descending,
+ * ties by (b, i) ascending.  After k admissions the verify batch holds
+ * n = B + k tokens (every row verifies its final position) and the expected
+ * emitted tokens are E(k) = B + (sum of the admitted S).  Candidate k+1 is
+ * admitted iff n + 1 < n_speed and E(k+1) * speed[n+1] > E(k) * speed[n];
+ * admission stops at the first candidate that fails.
+ *
+ *   conf     device float32 [B, K], read only.
+ *   B, K     1 <= B, 1 <= K <= SV_MAX_K, B * K <= SV_MAX_ADMIT.
+ *   speed    device float32 [n_speed]: the profiled verification steps per
+ *            second at a batch of n tokens, n = 0 .. n_speed-1 (the load
+ *            enters through this table).  n_speed >= 1.
+ *   lengths  device int32 [B], written: admitted candidates of each row (a
+ *            prefix of its draft block).
+ *   tau_out  device float32 [1], nullable: S of the last admitted candidate,
+ *            rounded to fp32 (+inf if none), the threshold that sv_schedule
+ *            would need to keep the same prefixes.
+ * Returns SV_OK, SV_ERR_ARG, SV_ERR_SHAPE or SV_ERR_CUDA.  One CTA; no
+ * workspace.  The partial sums run in a parallel order, so a candidate whose
+ * throughput gain is zero to ~1e-15 relative may be decided differently from
+ * a strictly sequential sum.
+ */
+sv_status sv_schedule_admit(const float *conf, int B, int K, const float *speed, int n_speed,
+                            int32_t *lengths, float *tau_out, void *stream);
 
 /*
  * sv_verify_workspace_bytes -- device scratch that sv_verify needs for

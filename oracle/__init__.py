@@ -54,6 +54,8 @@ def lib():
         L.oracle_stats_batch.restype = None
         L.oracle_schedule.argtypes = [vp, i64, i32, dbl, vp, vp]
         L.oracle_schedule.restype = dbl
+        L.oracle_schedule_admit.argtypes = [vp, i32, i32, vp, i32, vp, vp, vp]
+        L.oracle_schedule_admit.restype = i32
         L.oracle_ndiag.restype = i32
         assert L.oracle_ndiag() == NDIAG
         _lib = L
@@ -175,6 +177,21 @@ def schedule(conf, tau):
     S = np.zeros((B, K), dtype=np.float64)
     closest = lib().oracle_schedule(_p(c), B, K, float(tau), _p(ln), _p(S))
     return ln, S, closest
+
+
+def schedule_admit(conf, speed):
+    """Hardware-aware admission: candidates sorted by prefix survival are
+    admitted while (expected emitted tokens) x speed[batch tokens] rises.
+    conf [B, K] float32, speed [n] float32 (steps/s at n verified tokens).
+    Returns (lengths [B] int32, tau, k admitted, f [k_evaluated+1] fp64)."""
+    c = np.ascontiguousarray(conf, dtype=np.float32)
+    B, K = c.shape
+    sp = np.ascontiguousarray(speed, dtype=np.float32).reshape(-1)
+    ln = np.zeros(B, dtype=np.int32)
+    tau = np.zeros(1, dtype=np.float64)
+    f = np.full(B * K + 1, np.nan, dtype=np.float64)
+    k = lib().oracle_schedule_admit(_p(c), B, K, _p(sp), sp.size, _p(ln), _p(tau), _p(f))
+    return ln, float(tau[0]), int(k), f
 
 
 def default_threads() -> int:

@@ -453,3 +453,70 @@ double oracle_schedule(const float *conf, int64_t B, int K, double tau,
 }
 
 int oracle_ndiag(void) { return OR_NDIAG; }
+
+/* ---------------------------------------------------------------------------
+ * Hardware-aware admission [P1 "What DSpark adds", item "2. Verify
+ * smarter"; P3 "Under the hood"; P4 Ch.7 "Hardware-Aware Scheduling"]: the
+ * engine's speed (verification steps per second) is profiled once as a
+ * function of the verify batch size; every step the candidate draft tokens of
+ * all rows are sorted by prefix survival, admitted one at a time, and
+ * admission stops the moment expected system throughput -- expected accepted
+ * tokens times the speed at that batch size -- stops rising.
+ *
+ * Reading: row b always verifies its final position, so the batch holds
+ * n = B + k tokens after k admissions; expected emitted tokens are
+ * E(k) = B + (sum of the admitted S); f(k) = E(k) * speed[n]; candidate k+1
+ * is admitted iff n + 1 is inside the table and f(k+1) > f(k).  Candidates
+ * are ordered by S descending, ties by (row, position) ascending, so the
+ * admitted candidates of a row form a prefix.  S is the fp64 running product
+ * of the clamped confidences (NaN -> 0), as in oracle_schedule.
+ * Outputs: lengths[b] = admitted candidates of row b; *tau = S of the last
+ * admitted candidate (+inf if none); returns k.
+ * ------------------------------------------------------------------------- */
+typedef struct { double s; int idx; } cand_t;
+
+static int cand_cmp(const void *a, const void *b)
+{
+    const cand_t *x = (const cand_t *)a, *y = (const cand_t *)b;
+    if (x->s > y->s) return -1;
+    if (x->s < y->s) return 1;
+    return (x->idx > y->idx) - (x->idx < y->idx);
+}
+
+int oracle_schedule_admit(const float *conf, int B, int K, const float *speed, int n_speed,
+                          int32_t *lengths, double *tau, double *fvals /* [B*K+1] nullable */)
+{
+    int n = B * K;
+    cand_t *c = (cand_t *)malloc(sizeof(cand_t) * (size_t)(n > 0 ? n : 1));
+    for (int b = 0; b < B; ++b) {
+        double S = 1.0;
+        for (int i = 1; i <= K; ++i) {
+            double ci = (double)conf[b * K + (i - 1)];
+            if (isnan(ci)) ci = 0.0;
+            if (ci < 0.0) ci = 0.0;
+            if (ci > 1.0) ci = 1.0;
+            S = S * ci;
+            c[b * K + (i - 1)].s = S;
+            c[b * K + (i - 1)].idx = b * K + (i - 1);
+        }
+        lengths[b] = 0;
+    }
+    qsort(c, (size_t)n, sizeof(cand_t), cand_cmp);
+    double E = (double)B;
+    double f = (B < n_speed) ? E * (double)speed[B] : -INFINITY;
+    if (fvals) fvals[0] = f;
+    int k = 0;
+    while (k < n && B + k + 1 < n_speed) {
+        double E2 = E + c[k].s;
+        double f2 = E2 * (double)speed[B + k + 1];
+        if (fvals) fvals[k + 1] = f2;
+        if (!(f2 > f)) break;
+        E = E2;
+        f = f2;
+        lengths[c[k].idx / K] += 1;
+        ++k;
+    }
+    *tau = k > 0 ? c[k - 1].s : INFINITY;
+    free(c);
+    return k;
+}

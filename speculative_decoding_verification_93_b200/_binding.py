@@ -45,6 +45,7 @@ def lib():
     vp, i32, i64, u64, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64,
                              ctypes.c_size_t)
     L.sv_schedule.argtypes = [vp, i32, i32, ctypes.c_float, vp, vp]
+    L.sv_schedule_admit.argtypes = [vp, i32, i32, vp, i32, vp, vp, vp]
     L.sv_verify_workspace_bytes.argtypes = [i32, i32, i32, i32]
     L.sv_verify_workspace_bytes.restype = sz
     L.sv_verify.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, u64, i64, vp, vp, vp, sz, vp,
@@ -60,7 +61,7 @@ def lib():
     L.sv_profile_read.restype = i32
     L.sv_status_string.argtypes = [i32]
     L.sv_status_string.restype = ctypes.c_char_p
-    for name in ("sv_schedule", "sv_verify", "sv_verify_debug", "sv_verify_noalloc",
+    for name in ("sv_schedule", "sv_schedule_admit", "sv_verify", "sv_verify_debug", "sv_verify_noalloc",
                  "sv_philox_uniforms",
                  "sv_philox4x32_10", "sv_profile_begin"):
         getattr(L, name).restype = i32
@@ -107,6 +108,17 @@ def sv_schedule(conf: torch.Tensor, load: float, lengths: torch.Tensor, stream=N
     B, K = conf.shape
     _check("sv_schedule", lib().sv_schedule(_ptr(conf), B, K, float(load), _ptr(lengths),
                                             _stream(stream, conf)))
+
+
+def sv_schedule_admit(conf: torch.Tensor, speed: torch.Tensor, lengths: torch.Tensor,
+                      tau_out: Optional[torch.Tensor] = None, stream=None) -> None:
+    _need(conf, torch.float32, "conf")
+    _need(speed, torch.float32, "speed")
+    _need(lengths, torch.int32, "lengths")
+    B, K = conf.shape
+    _check("sv_schedule_admit", lib().sv_schedule_admit(
+        _ptr(conf), B, K, _ptr(speed), speed.numel(), _ptr(lengths), _ptr(tau_out),
+        _stream(stream, conf)))
 
 
 def sv_verify_workspace_bytes(B: int, K: int, V: int, dtype: int) -> int:

@@ -263,3 +263,13 @@ __device__ __forceinline__ void griddep_launch_dependents() {
 }
 
 }  // namespace sv
+
+namespace sv {
+// Relaxed load of a flag that other CTAs update (a stale value only makes
+// the caller do redundant work).
+__device__ __forceinline__ int ld_relaxed(const int *p) {
+    int v;
+    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+}  // namespace sv

@@ -52,14 +52,14 @@ namespace sv {
 
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = kConsumerWarps * 32;   // consumer group (warps 0..7)
-constexpr int kBlock = kConsumers + 32;           // + one producer warp
+constexpr int kBlock = kConsumers + 64;           // + one producer and one publisher warp
 constexpr int kStages = 4;                        // shared-memory ring depth
 constexpr int kStageUnits = 1024;                 // 16-byte units per stage (16 KB)
 constexpr int kRingBytes = kStages * kStageUnits * 16;
 constexpr int kMaxUnitsPerItem = 4 * kStageUnits; // an item spans up to 4 stages
 constexpr int kMaxSlots = 2 * SV_MAX_K + 1;
 constexpr int kMaxChunks = 64;                    // V <= SV_MAX_V keeps C within this
-constexpr int kPartsPerItem = kConsumerWarps;     // one softmax partial per consumer warp
+constexpr int kPartsPerItem = 1;                  // one merged softmax partial per item
 constexpr int kPrologueThreads = 1024;
 
 struct VerifyArgs {
@@ -77,7 +77,11 @@ struct VerifyArgs {
     float *dbg;                // nullable [B, S, 2]
     int *ctr;                  // [0] next item, [1] total items
     int *rcnt;                 // [B]  chunks of the residual draw done
-    int *row_off;              // [B+1]
+    int *leff;                 // [B]  verify length of a valid row, -1 for an invalid one
+    int *row_j;                // [B]  first rejection found so far (starts at L)
+    int *pcnt;                 // [B, K+1] item partials published per (row, position)
+    int *lvl_off;              // [K+2] first item of each position level
+    int *lvl_row;              // [K+1, B+1] per-level exclusive prefix of row item counts
     float4 *part;              // [B, S, C]: (m, s, argmax bits, 0)
     float *rseg;               // [B, C, 8] residual mass per chunk segment
     struct DrawRecord *rec;    // [B] accept result and draw set-up
@@ -111,59 +115,72 @@ __device__ __forceinline__ int row_slots(const VerifyArgs &a, int L, float T) {
 }
 
 // ---------------------------------------------------------------------------
-// 1. Prologue: validation, item counts, exclusive prefix, counter reset.
+// 1. Prologue: validation, the position-major work list, counter reset.
+//    Items are ordered by position level i = 0..K, then by row: level i holds
+//    the C chunks of target position i of every row with L >= i, followed in
+//    each row by the C chunks of draft position i when i < L and the row
+//    samples with draft logits.  The list is implicit in per-level row
+//    prefixes (one warp scans each level).
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ int level_items(const VerifyArgs &a, int Lb, bool sampled, int i) {
+    if (Lb < 0 || i > Lb) return 0;
+    return a.C * (1 + ((i < Lb && sampled) ? 1 : 0));
+}
+
 __global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(VerifyArgs a) {
-    __shared__ int s_warp[kPrologueThreads / 32];
-    __shared__ int s_carry;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     griddep_wait();
     griddep_launch_dependents();   // the stream kernel may take its SMs now
-    if (tid == 0) s_carry = 0;
+    const int K1 = a.K + 1;
+    // Rows: validity, effective length, first-rejection marker, counters.
+    for (int b = tid; b < a.B; b += kPrologueThreads) {
+        const int bits = row_errors(a, b);
+        int Lb = -1;
+        if (bits) {
+            a.out_accept[b] = -1;
+            for (int i = 0; i <= a.K; ++i)
+                a.out_tokens[static_cast<long long>(b) * K1 + i] = -1;
+            if (a.status) atomicOr(a.status, bits);
+        } else {
+            Lb = a.lengths[b];
+        }
+        a.leff[b] = Lb;
+        a.row_j[b] = Lb;
+        a.rcnt[b] = 0;
+        for (int i = 0; i < K1; ++i) a.pcnt[static_cast<long long>(b) * K1 + i] = 0;
+    }
     __syncthreads();
-    for (int base = 0; base < a.B; base += kPrologueThreads) {
-        const int b = base + tid;
-        int n = 0;
-        if (b < a.B) {
-            const int bits = row_errors(a, b);
-            if (bits) {
-                a.out_accept[b] = -1;
-                for (int i = 0; i <= a.K; ++i)
-                    a.out_tokens[static_cast<long long>(b) * (a.K + 1) + i] = -1;
-                if (a.status) atomicOr(a.status, bits);
-            } else {
-                n = row_slots(a, a.lengths[b], a.temp[b]) * a.C;
-            }
-            a.rcnt[b] = 0;
-        }
-        int x = n;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
-        }
-        if (lane == 31) s_warp[warp] = x;
-        __syncthreads();
-        if (warp == 0) {
-            int y = s_warp[lane];
+    // Levels: warp w scans levels w, w + 32, ... over the rows.
+    const bool draft = a.zd != nullptr;
+    for (int i = warp; i < K1; i += kPrologueThreads / 32) {
+        int carry = 0;
+        int *off = a.lvl_row + static_cast<long long>(i) * (a.B + 1);
+        for (int b0 = 0; b0 < a.B; b0 += 32) {
+            const int b = b0 + lane;
+            int n = 0;
+            if (b < a.B) n = level_items(a, a.leff[b], draft && a.temp[b] > 0.f, i);
+            int x = n;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const int z = __shfl_up_sync(0xffffffffu, y, o);
-                if (lane >= o) y += z;
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
             }
-            s_warp[lane] = y;
+            if (b < a.B) off[b] = carry + x - n;
+            carry += __shfl_sync(0xffffffffu, x, 31);
         }
-        __syncthreads();
-        const int incl = x + (warp ? s_warp[warp - 1] : 0) + s_carry;
-        if (b < a.B) a.row_off[b] = incl - n;
-        __syncthreads();
-        if (tid == kPrologueThreads - 1) s_carry = incl;
-        __syncthreads();
+        if (lane == 0) { off[a.B] = carry; a.lvl_off[i + 1] = carry; }
     }
+    __syncthreads();
     if (tid == 0) {
-        a.row_off[a.B] = s_carry;
+        int acc = 0;
+        for (int i = 0; i < K1; ++i) {
+            const int c = a.lvl_off[i + 1];
+            a.lvl_off[i] = acc;
+            acc += c;
+        }
+        a.lvl_off[K1] = acc;
         a.ctr[0] = 0;
-        a.ctr[1] = s_carry;
+        a.ctr[1] = acc;
     }
 }
 
@@ -255,7 +272,7 @@ struct __align__(16) StageDesc {
     int nunits;   // body units in the stage
     int flags;    // kFirst | kLast
     float k;      // log2(e)/T; 0 for greedy rows
-    int pad;
+    int level;    // position i of the item
 };
 constexpr int kFirst = 1, kLast = 2;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s: no legitimate wait comes close
@@ -267,20 +284,136 @@ __device__ __forceinline__ void vstore(int &x, int v) {
     *reinterpret_cast<volatile int *>(&x) = v;
 }
 
+constexpr int kItemSlots = 8;   // > kStages: consumer warps are never more than kStages items apart
+
+struct ItemMeta {
+    int b;        // row; -1 = no more items
+    int slot;
+    int chunk;
+    int level;
+    float k;
+    int pad[3];
+};
+
 struct StreamSmem {
     uint64_t full[kStages];
     uint64_t empty[kStages];
     StageDesc desc[kStages];
+    // Mailbox from the consumer warps to the publisher warp, one slot per
+    // recent item: each consumer warp leaves its partial and arrives on
+    // ifull; the publisher merges, arrives on ifree, and publishes.
+    float4 ipart[kItemSlots][kConsumerWarps];
+    ItemMeta imeta[kItemSlots];
+    uint64_t ifull[kItemSlots];
+    uint64_t ifree[kItemSlots];
     int abort;
 };
 
+// Accept test of position i of row b, once every chunk partial of that
+// position is published (one warp; lane 0 decides).  Same rule as the
+// oracle: accept x_i iff u(seed, row, i, 0) < min(1, p_i(x_i) / q_i(x_i)),
+// greedy rows iff x_i is the target argmax.  A rejection lowers row_j[b].
+template <int ESIZE>
+__device__ void decide_position(const VerifyArgs &a, int b, int i) {
+    const int lane = threadIdx.x & 31;
+    const int K = a.K, S = a.S, C = a.C;
+    const float T = __ldg(&a.temp[b]);
+    const bool greedy = !(T > 0.f);
+    const bool has_draft = (a.zd != nullptr) && !greedy;
+    const float k = greedy ? 0.f : kLog2e / T;
+    float mt = kNegInf, st = 0.f, md = kNegInf, sd = 0.f;
+    int at = INT_MAX;
+    const long long bt = (static_cast<long long>(b) * S + i) * C;
+    const long long bd = (static_cast<long long>(b) * S + K + 1 + i) * C;
+    for (int cc = lane; cc < C; cc += 32) {
+        const float4 p = __ldcg(&a.part[bt + cc]);
+        if (greedy) {
+            const int i2 = __float_as_int(p.z);
+            if (p.x > mt || (p.x == mt && i2 < at)) { mt = p.x; at = i2; }
+        } else {
+            lse_merge(mt, st, p.x, p.y, k);
+        }
+        if (has_draft) {
+            const float4 q = __ldcg(&a.part[bd + cc]);
+            lse_merge(md, sd, q.x, q.y, k);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, mt, o);
+        const float s2 = __shfl_xor_sync(0xffffffffu, st, o);
+        const int i2 = __shfl_xor_sync(0xffffffffu, at, o);
+        const float n2 = __shfl_xor_sync(0xffffffffu, md, o);
+        const float d2 = __shfl_xor_sync(0xffffffffu, sd, o);
+        if (greedy) {
+            if (m2 > mt || (m2 == mt && i2 < at)) { mt = m2; at = i2; }
+        } else {
+            lse_merge(mt, st, m2, s2, k);
+            lse_merge(md, sd, n2, d2, k);
+        }
+    }
+    if (lane == 0) {
+        const int x = a.tokens[static_cast<long long>(b) * K + i];
+        bool acc;
+        if (greedy) {
+            acc = (x == (at == INT_MAX ? 0 : at));
+        } else {
+            const float zt_x = ld_elem<ESIZE>(vec_ptr<ESIZE>(a, b, i), x);
+            const float lp = fmaf(zt_x - mt, k, -log2f(st));
+            float lq = 0.f;
+            if (has_draft) {
+                const float zd_x = ld_elem<ESIZE>(vec_ptr<ESIZE>(a, b, K + 1 + i), x);
+                lq = fmaf(zd_x - md, k, -log2f(sd));
+            }
+            const uint64_t row = static_cast<uint64_t>(a.row_base) + static_cast<uint64_t>(b);
+            const float u = uniform24(a.seed, row, static_cast<uint32_t>(i), 0u);
+            if (lp == kNegInf) acc = false;
+            else if (lq == kNegInf) acc = true;
+            else acc = (lp >= lq) || (u < exp2f(lp - lq));
+        }
+        if (!acc) atomicMin(&a.row_j[b], i);
+    }
+}
+
 // Producer: fetch items (global atomic counter, prefetched one item ahead),
 // decode them, stream their 16-byte body units into the ring.
+// Position-major item w decoded: level i, row b, slot and chunk.
+struct ItemRef {
+    int i, b, slot, chunk;
+};
+
+__device__ __forceinline__ ItemRef decode_item(const VerifyArgs &a, int w) {
+    int lo = 0, hi = a.K;   // largest level with lvl_off[i] <= w
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (__ldg(&a.lvl_off[mid]) <= w) lo = mid; else hi = mid - 1;
+    }
+    ItemRef it;
+    it.i = lo;
+    const int r = w - __ldg(&a.lvl_off[lo]);
+    const int *off = a.lvl_row + static_cast<long long>(lo) * (a.B + 1);
+    lo = 0; hi = a.B - 1;   // largest row with off[b] <= r (a row with items)
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (__ldg(&off[mid]) <= r) lo = mid; else hi = mid - 1;
+    }
+    it.b = lo;
+    const int q = r - __ldg(&off[lo]);
+    it.chunk = q < a.C ? q : q - a.C;
+    it.slot = q < a.C ? it.i : a.K + 1 + it.i;
+    return it;
+}
+
 template <int ESIZE>
 __device__ void producer(const VerifyArgs &a, StreamSmem &sm, uint4 *ring, int total) {
     uint32_t it = 0;
     bool ok = true;
+    // Two claims in flight so that the counter's round trip overlaps the
+    // current item.  The row's status is read when the item's turn comes and
+    // again before each later stage: a rejection only ever lowers it, so a
+    // stale value costs redundant bytes, never a wrong result.
     int w = atomicAdd(&a.ctr[0], 1);
+    int wnext = atomicAdd(&a.ctr[0], 1);
     while (ok) {
         if (w >= total) {
             const int st = it % kStages;
@@ -291,48 +424,50 @@ __device__ void producer(const VerifyArgs &a, StreamSmem &sm, uint4 *ring, int t
             ++it;
             break;
         }
-        // Decode item w: row b (largest b with row_off[b] <= w), slot, chunk.
-        int lo = 0, hi = a.B - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (__ldg(&a.row_off[mid]) <= w) lo = mid; else hi = mid - 1;
-        }
-        const int b = lo;
-        const int r = w - __ldg(&a.row_off[b]);
-        const int L = __ldg(&a.lengths[b]);
-        const float T = __ldg(&a.temp[b]);
-        const int q = r / a.C, chunk = r - q * a.C;
-        const int slot = q <= L ? q : (a.K + 1 + (q - L - 1));
-        const float k = (T > 0.f) ? kLog2e / T : 0.f;
-        const VecGeom g = vec_geom<ESIZE>(vec_ptr<ESIZE>(a, b, slot), a.V);
-        const int u0 = chunk * a.U;
-        const int u1 = max(u0, min(u0 + a.U, g.n16));
-        const int wnext = atomicAdd(&a.ctr[0], 1);   // next item, consumed after this one
-        const int npieces = max(1, (u1 - u0 + kStageUnits - 1) / kStageUnits);
-        for (int p = 0; p < npieces; ++p) {
-            const int st = it % kStages;
-            const uint32_t ph = (it / kStages) & 1u;
-            if (!mbar_wait(&sm.empty[st], ph ^ 1u, kWaitLimitNs) || vload(sm.abort)) {
-                ok = false;
-                break;
+        const ItemRef cur = decode_item(a, w);
+        const int rj = ld_relaxed(&a.row_j[cur.b]);
+        const int wfar = atomicAdd(&a.ctr[0], 1);
+        // A row that has already rejected an earlier position never needs
+        // this one: skip it without reading a byte.
+        if (rj >= cur.i) {
+            const int b = cur.b, i = cur.i, slot = cur.slot, chunk = cur.chunk;
+            const float T = __ldg(&a.temp[b]);
+            const float k = (T > 0.f) ? kLog2e / T : 0.f;
+            const VecGeom g = vec_geom<ESIZE>(vec_ptr<ESIZE>(a, b, slot), a.V);
+            const int u0 = chunk * a.U;
+            const int u1 = max(u0, min(u0 + a.U, g.n16));
+            const int npieces = max(1, (u1 - u0 + kStageUnits - 1) / kStageUnits);
+            for (int p = 0; p < npieces; ++p) {
+                // Abandon the rest of the item once the row has rejected an
+                // earlier position: the consumers reset at the next item's
+                // first stage, and no partial of this item is ever read.
+                if (p > 0 && ld_relaxed(&a.row_j[b]) < i) break;
+                const int st = it % kStages;
+                const uint32_t ph = (it / kStages) & 1u;
+                if (!mbar_wait(&sm.empty[st], ph ^ 1u, kWaitLimitNs) || vload(sm.abort)) {
+                    ok = false;
+                    break;
+                }
+                const int pu0 = u0 + p * kStageUnits;
+                const int pn = max(0, min(u1 - pu0, kStageUnits));
+                StageDesc &d = sm.desc[st];
+                d.b = b; d.slot = slot; d.chunk = chunk; d.unit0 = pu0; d.nunits = pn;
+                d.flags = (p == 0 ? kFirst : 0) | (p == npieces - 1 ? kLast : 0);
+                d.k = k;
+                d.level = i;
+                if (pn > 0) {
+                    mbar_arrive_expect_tx(&sm.full[st], static_cast<uint32_t>(pn) * 16u);
+                    bulk_g2s(ring + static_cast<size_t>(st) * kStageUnits,
+                             g.body + static_cast<long long>(pu0) * 16,
+                             static_cast<uint32_t>(pn) * 16u, &sm.full[st]);
+                } else {
+                    mbar_arrive(&sm.full[st]);
+                }
+                ++it;
             }
-            const int pu0 = u0 + p * kStageUnits;
-            const int pn = max(0, min(u1 - pu0, kStageUnits));
-            StageDesc &d = sm.desc[st];
-            d.b = b; d.slot = slot; d.chunk = chunk; d.unit0 = pu0; d.nunits = pn;
-            d.flags = (p == 0 ? kFirst : 0) | (p == npieces - 1 ? kLast : 0);
-            d.k = k;
-            if (pn > 0) {
-                mbar_arrive_expect_tx(&sm.full[st], static_cast<uint32_t>(pn) * 16u);
-                bulk_g2s(ring + static_cast<size_t>(st) * kStageUnits,
-                         g.body + static_cast<long long>(pu0) * 16, static_cast<uint32_t>(pn) * 16u,
-                         &sm.full[st]);
-            } else {
-                mbar_arrive(&sm.full[st]);
-            }
-            ++it;
         }
         w = wnext;
+        wnext = wfar;
     }
     if (!ok) {
         // Unwind: report, then wait (bounded) for the copies still in flight
@@ -357,6 +492,7 @@ __device__ void consumers(const VerifyArgs &a, StreamSmem &sm, const uint4 *ring
     const uint32_t pw = neg_inf_word<ESIZE>();
     const uint4 pad = make_uint4(pw, pw, pw, pw);
     uint32_t it = 0;
+    uint32_t iseq = 0;   // items finished by this warp (same sequence in every warp)
     float m = kNegInf, s = 0.f;
     int bidx = INT_MAX;
     while (true) {
@@ -419,8 +555,8 @@ __device__ void consumers(const VerifyArgs &a, StreamSmem &sm, const uint4 *ring
         }
 
         if (!(d.flags & kLast)) continue;
-        // End of item: warp reduction; one partial per (row, slot, chunk,
-        // warp), so the warps never wait for one another.
+        // End of item: warp reduction; the CTA-level merge, the publication
+        // and the accept test belong to the publisher warp.
         float rm = m, rs = s;
         int ri = bidx;
 #pragma unroll
@@ -434,15 +570,98 @@ __device__ void consumers(const VerifyArgs &a, StreamSmem &sm, const uint4 *ring
                 lse_merge(rm, rs, m2, s2, d.k);
             }
         }
-        if (lane == 0)
-            a.part[((static_cast<long long>(d.b) * a.S + d.slot) * a.C + d.chunk) * kPartsPerItem +
-                   warp] = make_float4(rm, greedy ? 0.f : rs, __int_as_float(greedy ? ri : 0), 0.f);
+        // Hand the warp partial to the publisher warp and go on streaming.
+        const uint32_t slot_i = iseq % kItemSlots, use = iseq / kItemSlots;
+        ++iseq;
+        int ok = 1;
+        if (lane == 0) {
+            ok = mbar_wait(&sm.ifree[slot_i], (use & 1u) ^ 1u, kWaitLimitNs);
+            if (ok) {
+                sm.ipart[slot_i][warp] = make_float4(rm, rs, __int_as_float(ri), 0.f);
+                if (warp == 0) {
+                    ItemMeta &im = sm.imeta[slot_i];
+                    im.b = d.b; im.slot = d.slot; im.chunk = d.chunk; im.level = d.level;
+                    im.k = d.k;
+                }
+                mbar_arrive(&sm.ifull[slot_i]);
+            }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+            vstore(sm.abort, 1);
+            if (a.status && lane == 0) atomicOr(a.status, SV_NOTE_TIMEOUT);
+            break;
+        }
+    }
+    // No more items: tell the publisher through the next mailbox slot.
+    if (lane == 0 && !vload(sm.abort)) {
+        const uint32_t slot_i = iseq % kItemSlots, use = iseq / kItemSlots;
+        if (mbar_wait(&sm.ifree[slot_i], (use & 1u) ^ 1u, kWaitLimitNs)) {
+            if (warp == 0) sm.imeta[slot_i].b = -1;
+            mbar_arrive(&sm.ifull[slot_i]);
+        } else {
+            vstore(sm.abort, 1);
+        }
     }
 }
 
-// Persistent warp-specialised kernel: warp kConsumerWarps is the producer
-// (work fetch + bulk copies into the shared-memory ring), warps
-// 0..kConsumerWarps-1 consume stages.
+// Publisher warp: merges each item's eight warp partials in fixed order
+// (the result does not depend on timing), publishes one partial per item,
+// counts completed chunks per (row, position), and runs the accept test of a
+// position the moment its last chunk lands.
+template <int ESIZE>
+__device__ void publisher(const VerifyArgs &a, StreamSmem &sm) {
+    const int lane = threadIdx.x & 31;
+    uint32_t iseq = 0;
+    while (true) {
+        const uint32_t slot_i = iseq % kItemSlots, use = iseq / kItemSlots;
+        if (!mbar_wait(&sm.ifull[slot_i], use & 1u, kWaitLimitNs) || vload(sm.abort)) {
+            vstore(sm.abort, 1);
+            if (a.status && lane == 0) atomicOr(a.status, SV_NOTE_TIMEOUT);
+            break;
+        }
+        const ItemMeta im = sm.imeta[slot_i];
+        if (im.b < 0) break;
+        const bool greedy = im.k == 0.f;
+        float4 pv = make_float4(kNegInf, 0.f, __int_as_float(INT_MAX), 0.f);
+        if (lane < kConsumerWarps) pv = sm.ipart[slot_i][lane];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.ifree[slot_i]);
+        ++iseq;
+        float rm = pv.x, rs = pv.y;
+        int ri = __float_as_int(pv.z);
+#pragma unroll
+        for (int o = 1; o < kConsumerWarps; o <<= 1) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, rm, o);
+            const float s2 = __shfl_xor_sync(0xffffffffu, rs, o);
+            const int i2 = __shfl_xor_sync(0xffffffffu, ri, o);
+            if (greedy) {
+                if (m2 > rm || (m2 == rm && i2 < ri)) { rm = m2; ri = i2; }
+            } else {
+                lse_merge(rm, rs, m2, s2, im.k);
+            }
+        }
+        int complete = 0;
+        if (lane == 0) {
+            a.part[(static_cast<long long>(im.b) * a.S + im.slot) * a.C + im.chunk] =
+                make_float4(rm, greedy ? 0.f : rs, __int_as_float(greedy ? ri : 0), 0.f);
+            __threadfence();
+            const int Lb = __ldg(&a.leff[im.b]);
+            const bool draft_here = (a.zd != nullptr) && !greedy && im.level < Lb;
+            const int need = a.C * (draft_here ? 2 : 1);
+            const int done =
+                atomicAdd(&a.pcnt[static_cast<long long>(im.b) * (a.K + 1) + im.level], 1) + 1;
+            complete = (done == need) && (im.level < Lb);
+            if (complete) __threadfence();
+        }
+        complete = __shfl_sync(0xffffffffu, complete, 0);
+        if (complete) decide_position<ESIZE>(a, im.b, im.level);
+    }
+}
+
+// Persistent warp-specialised kernel: warps 0..7 consume stages, warp 8 is
+// the producer (work fetch + bulk copies into the shared-memory ring), warp
+// 9 is the publisher (item partials, completion counts, accept tests).
 template <int ESIZE>
 __global__ void __launch_bounds__(kBlock, 3) stream_kernel(VerifyArgs a) {
     extern __shared__ __align__(128) uint4 ring[];
@@ -453,12 +672,20 @@ __global__ void __launch_bounds__(kBlock, 3) stream_kernel(VerifyArgs a) {
             mbar_init(&sm.full[i], 1);
             mbar_init(&sm.empty[i], kConsumerWarps);
         }
+        for (int i = 0; i < kItemSlots; ++i) {
+            mbar_init(&sm.ifull[i], kConsumerWarps);
+            mbar_init(&sm.ifree[i], 1);
+        }
         sm.abort = 0;
         fence_mbar_init();
     }
     __syncthreads();
     griddep_wait();
     const int total = __ldcg(&a.ctr[1]);
+    if (tid >= kConsumers + 32) {
+        publisher<ESIZE>(a, sm);
+        return;
+    }
     if (tid >= kConsumers) {
         if (tid == kConsumers) producer<ESIZE>(a, sm, ring, total);
         return;
@@ -900,101 +1127,58 @@ __global__ void __launch_bounds__(kDrawThreads) accept_kernel(VerifyArgs a) {
     const int b = blockIdx.x;
     const int K = a.K, S = a.S, C = a.C;
     DrawRecord *rec = a.rec + b;
-    if (__ldg(&a.row_off[b + 1]) == __ldg(&a.row_off[b])) {   // invalid row, already marked
+    const int L = __ldg(&a.leff[b]);
+    if (L < 0) {                   // invalid row, already marked
         if (tid == 0) rec->mode = kDrawDone;
         return;
     }
-    const int L = __ldg(&a.lengths[b]);
     const float T = __ldg(&a.temp[b]);
     const bool greedy = !(T > 0.f);
     const bool has_draft = (a.zd != nullptr) && !greedy;
     const float k = greedy ? 0.f : kLog2e / T;
     const uint64_t row = static_cast<uint64_t>(a.row_base) + static_cast<uint64_t>(b);
-    const int nslots = L + 1 + (has_draft ? L : 0);
-    const int nparts = C * kPartsPerItem;
-
-    // Merge the partials of every vector of the row: warp w takes slots
-    // w, w+8, ... in rounds of kRound, issuing a round's loads before any of
-    // its reductions.
-    constexpr int kRound = 4;
-    for (int r0 = 0; warp + r0 * kDrawWarps < nslots; r0 += kRound) {
-        float4 pv[kRound];
-#pragma unroll
-        for (int r = 0; r < kRound; ++r) {
-            const int q = warp + (r0 + r) * kDrawWarps;
-            pv[r] = make_float4(kNegInf, 0.f, __int_as_float(INT_MAX), 0.f);
-            if (q < nslots && lane < nparts) {
-                const int slot = q <= L ? q : (K + 1 + (q - L - 1));
-                pv[r] = __ldcg(&a.part[(static_cast<long long>(b) * S + slot) * nparts + lane]);
+    // The stream kernel decided every position up to the first rejection.
+    const int j = min(__ldg(&a.row_j[b]), L);
+    // Normalisers of the positions that were read in full: target 0..j and
+    // draft 0..min(j, L-1); warp w takes slots w, w+8, ...
+    const int ntgt = j + 1;
+    const int nslots = ntgt + (has_draft ? min(j + 1, L) : 0);
+    for (int q = warp; q < nslots; q += kDrawWarps) {
+        const int slot = q < ntgt ? q : (K + 1 + (q - ntgt));
+        float m = kNegInf, sm = 0.f;
+        int idx = INT_MAX;
+        for (int cc = lane; cc < C; cc += 32) {
+            const float4 p = __ldcg(&a.part[(static_cast<long long>(b) * S + slot) * C + cc]);
+            if (greedy) {
+                const int i2 = __float_as_int(p.z);
+                if (p.x > m || (p.x == m && i2 < idx)) { m = p.x; idx = i2; }
+            } else {
+                lse_merge(m, sm, p.x, p.y, k);
             }
         }
 #pragma unroll
-        for (int r = 0; r < kRound; ++r) {
-            const int q = warp + (r0 + r) * kDrawWarps;
-            if (q >= nslots) break;
-            const int slot = q <= L ? q : (K + 1 + (q - L - 1));
-            float m = pv[r].x, sm = pv[r].y;
-            int idx = __float_as_int(pv[r].z);
-            for (int cc = lane + 32; cc < nparts; cc += 32) {   // C > 4 only
-                const float4 p =
-                    __ldcg(&a.part[(static_cast<long long>(b) * S + slot) * nparts + cc]);
-                if (greedy) {
-                    const int i2 = __float_as_int(p.z);
-                    if (p.x > m || (p.x == m && i2 < idx)) { m = p.x; idx = i2; }
-                } else {
-                    lse_merge(m, sm, p.x, p.y, k);
-                }
+        for (int o = 16; o > 0; o >>= 1) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+            const float s2 = __shfl_xor_sync(0xffffffffu, sm, o);
+            const int i2 = __shfl_xor_sync(0xffffffffu, idx, o);
+            if (greedy) {
+                if (m2 > m || (m2 == m && i2 < idx)) { m = m2; idx = i2; }
+            } else {
+                lse_merge(m, sm, m2, s2, k);
             }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-                const float s2 = __shfl_xor_sync(0xffffffffu, sm, o);
-                const int i2 = __shfl_xor_sync(0xffffffffu, idx, o);
-                if (greedy) {
-                    if (m2 > m || (m2 == m && i2 < idx)) { m = m2; idx = i2; }
-                } else {
-                    lse_merge(m, sm, m2, s2, k);
-                }
-            }
-            if (lane == 0) {
-                if (idx == INT_MAX) idx = 0;   // every logit -inf: documented as invalid input
-                ds.m[slot] = m;
-                ds.s[slot] = greedy ? 1.f : sm;
-                ds.arg[slot] = idx;
-                if (a.dbg) {
-                    a.dbg[(static_cast<long long>(b) * S + slot) * 2 + 0] = m;
-                    a.dbg[(static_cast<long long>(b) * S + slot) * 2 + 1] = greedy ? 1.f : sm;
-                }
+        }
+        if (lane == 0) {
+            if (idx == INT_MAX) idx = 0;   // every logit -inf: documented as invalid input
+            ds.m[slot] = m;
+            ds.s[slot] = greedy ? 1.f : sm;
+            ds.arg[slot] = idx;
+            if (a.dbg) {
+                a.dbg[(static_cast<long long>(b) * S + slot) * 2 + 0] = m;
+                a.dbg[(static_cast<long long>(b) * S + slot) * 2 + 1] = greedy ? 1.f : sm;
             }
         }
     }
-    if (tid == 0) ds.j = L;
     __syncthreads();
-
-    // Accept test, one thread per verified position; first rejection wins.
-    if (tid < L) {
-        const int i = tid;
-        const int x = a.tokens[static_cast<long long>(b) * K + i];
-        bool acc;
-        if (greedy) {
-            acc = (x == ds.arg[i]);
-        } else {
-            const float zt_x = ld_elem<ESIZE>(vec_ptr<ESIZE>(a, b, i), x);
-            const float lp = fmaf(zt_x - ds.m[i], k, -log2f(ds.s[i]));
-            float lq = 0.f;
-            if (has_draft) {
-                const float zd_x = ld_elem<ESIZE>(vec_ptr<ESIZE>(a, b, K + 1 + i), x);
-                lq = fmaf(zd_x - ds.m[K + 1 + i], k, -log2f(ds.s[K + 1 + i]));
-            }
-            const float u = uniform24(a.seed, row, static_cast<uint32_t>(i), 0u);
-            if (lp == kNegInf) acc = false;
-            else if (lq == kNegInf) acc = true;
-            else acc = (lp >= lq) || (u < exp2f(lp - lq));
-        }
-        if (!acc) atomicMin(&ds.j, i);
-    }
-    __syncthreads();
-    const int j = ds.j;
 
     if (greedy) {
         const int y = ds.arg[j];
@@ -1190,7 +1374,8 @@ template <int ESIZE> static const void *stream_kernel_ptr() {
 // ---------------------------------------------------------------------------
 struct Plan {
     int C, U, S;
-    size_t off_rcnt, off_rowoff, off_part, off_rseg, off_rec, bytes;
+    size_t off_rcnt, off_leff, off_rowj, off_pcnt, off_lvloff, off_lvlrow, off_part, off_rseg,
+        off_rec, bytes;
 };
 
 static bool make_plan(int B, int K, int V, sv_dtype dtype, Plan *p) {
@@ -1207,20 +1392,19 @@ static bool make_plan(int B, int K, int V, sv_dtype dtype, Plan *p) {
     const long long items = static_cast<long long>(B) * S * C;
     if (items >= INT_MAX / 2 || static_cast<long long>(B) * C >= INT_MAX / 2) return false;
     p->C = C; p->U = U; p->S = S;
+    const size_t iB = sizeof(int) * static_cast<size_t>(B);
+    auto align16 = [](size_t o) { return (o + 15) & ~static_cast<size_t>(15); };
     size_t off = 16;
-    p->off_rcnt = off;
-    off += sizeof(int) * static_cast<size_t>(B);
-    p->off_rowoff = off;
-    off += sizeof(int) * static_cast<size_t>(B + 1);
-    off = (off + 15) & ~static_cast<size_t>(15);
-    p->off_part = off;
-    off += sizeof(float4) * static_cast<size_t>(items) * kPartsPerItem;
-    p->off_rseg = off;
-    off += sizeof(float) * static_cast<size_t>(B) * C * kDrawWarps;
-    off = (off + 15) & ~static_cast<size_t>(15);
-    p->off_rec = off;
-    off += sizeof(DrawRecord) * static_cast<size_t>(B);
-    p->bytes = (off + 15) & ~static_cast<size_t>(15);
+    p->off_rcnt = off;   off = align16(off + iB);
+    p->off_leff = off;   off = align16(off + iB);
+    p->off_rowj = off;   off = align16(off + iB);
+    p->off_pcnt = off;   off = align16(off + iB * (K + 1));
+    p->off_lvloff = off; off = align16(off + sizeof(int) * static_cast<size_t>(K + 2));
+    p->off_lvlrow = off; off = align16(off + sizeof(int) * static_cast<size_t>(K + 1) * (B + 1));
+    p->off_part = off;   off = align16(off + sizeof(float4) * static_cast<size_t>(items));
+    p->off_rseg = off;   off = align16(off + sizeof(float) * static_cast<size_t>(B) * C * kDrawWarps);
+    p->off_rec = off;    off = align16(off + sizeof(DrawRecord) * static_cast<size_t>(B));
+    p->bytes = off;
     return true;
 }
 
@@ -1272,7 +1456,11 @@ static sv_status verify_impl(const void *zt, const void *zd, sv_dtype dtype, int
     char *w = static_cast<char *>(ws);
     a.ctr = reinterpret_cast<int *>(w);
     a.rcnt = reinterpret_cast<int *>(w + p.off_rcnt);
-    a.row_off = reinterpret_cast<int *>(w + p.off_rowoff);
+    a.leff = reinterpret_cast<int *>(w + p.off_leff);
+    a.row_j = reinterpret_cast<int *>(w + p.off_rowj);
+    a.pcnt = reinterpret_cast<int *>(w + p.off_pcnt);
+    a.lvl_off = reinterpret_cast<int *>(w + p.off_lvloff);
+    a.lvl_row = reinterpret_cast<int *>(w + p.off_lvlrow);
     a.part = reinterpret_cast<float4 *>(w + p.off_part);
     a.rseg = reinterpret_cast<float *>(w + p.off_rseg);
     a.rec = reinterpret_cast<DrawRecord *>(w + p.off_rec);

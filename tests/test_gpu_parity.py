@@ -68,7 +68,10 @@ def test_small_ragged_matches_oracle(V, dtype, K, B):
 @pytest.mark.parametrize("V,dtype", [(1000, torch.float32), (129280, torch.bfloat16),
                                      (20011, torch.float32), (1001, torch.bfloat16)])
 def test_normalisers_match_oracle(V, dtype):
-    """m bit-exact, Sigma within 1e-5 relative, for every vector the call read."""
+    """m bit-exact, Sigma within 1e-5 relative, for every vector the outcome
+    depends on: target positions 0..a and draft positions 0..min(a, L-1) of
+    sampled rows (a = accepted length).  Later positions are not read in
+    full and not reported."""
     B, K = 16, 4
     b = _cuda(workloads.random_small(B, K, V, dtype=dtype, seed=3, temps=(0.0, 0.6, 1.0, 1.7),
                                      lengths=K))
@@ -78,16 +81,20 @@ def test_normalisers_match_oracle(V, dtype):
     mt, St, _ = oracle.stats(to_host_logits(b.zt), T[:, None])
     md, Sd, _ = oracle.stats(to_host_logits(b.zd), T[:, None])
     for r in range(B):
+        j = g["accept"][r]
         for i in range(K + 1):
-            assert st[r, i, 0] == mt[r, i]
-            if T[r] > 0:
-                assert abs(st[r, i, 1] - St[r, i]) <= 1e-5 * St[r, i]
+            if i <= j:
+                assert st[r, i, 0] == mt[r, i]
+                if T[r] > 0:
+                    assert abs(st[r, i, 1] - St[r, i]) <= 1e-5 * St[r, i]
+            else:
+                assert np.isnan(st[r, i, 0])
         for i in range(K):
-            if T[r] > 0:
+            if T[r] > 0 and i <= min(j, K - 1):
                 assert st[r, K + 1 + i, 0] == md[r, i]
                 assert abs(st[r, K + 1 + i, 1] - Sd[r, i]) <= 1e-5 * Sd[r, i]
             else:
-                assert np.isnan(st[r, K + 1 + i, 0])      # greedy rows never read drafts
+                assert np.isnan(st[r, K + 1 + i, 0])   # greedy rows never read drafts
 
 
 @pytest.mark.parametrize("V,dtype", [(7, torch.float32), (1000, torch.bfloat16),

@@ -81,7 +81,7 @@ def test_no_alloc_back_to_back_shapes_and_row_base():
 
 
 def test_no_alloc_rejects_batches_beyond_its_scratch():
-    B, K, V = 512, 16, 129280          # fp32: needs more than 16 MiB of scratch
+    B, K, V = 8192, 64, 129280         # fp32: needs more than 16 MiB of scratch
     need = sv.sv_verify_workspace_bytes(B, K, V, sv.SV_F32)
     assert need > SCRATCH_BYTES
     zt = torch.zeros(1, dtype=torch.float32, device="cuda")
