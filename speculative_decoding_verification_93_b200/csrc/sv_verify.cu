@@ -75,7 +75,7 @@ struct VerifyArgs {
     int32_t *out_accept;       // [B]
     int32_t *status;           // nullable
     float *dbg;                // nullable [B, S, 2]
-    int *ctr;                  // [0] next item, [1] total items
+    int *ctr;                  // [0] next item, [1] total items, [2] resample work entries
     int *rcnt;                 // [B]  chunks of the residual draw done
     int *leff;                 // [B]  verify length of a valid row, -1 for an invalid one
     int *row_j;                // [B]  first rejection found so far (starts at L)
@@ -83,7 +83,9 @@ struct VerifyArgs {
     int *lvl_off;              // [K+2] first item of each position level
     int *lvl_row;              // [K+1, B+1] per-level exclusive prefix of row item counts
     float4 *part;              // [B, S, C]: (m, s, argmax bits, 0)
-    float *rseg;               // [B, C, 8] residual mass per chunk segment
+    float *rtbl;               // [B, nsub] residual mass per sub-range
+    int nsub;                  // sub-ranges per row
+    int *work;                 // [B * C] (row * C + chunk) of the resample CTAs with work
     struct DrawRecord *rec;    // [B] accept result and draw set-up
 };
 
@@ -102,10 +104,17 @@ __device__ __forceinline__ int row_errors(const VerifyArgs &a, int b) {
     if (L < 0 || L > a.K) bits |= SV_ROW_BAD_LENGTH;
     if (!(T >= 0.f) || isinf(T) || (T > 0.f && T < 1e-6f)) bits |= SV_ROW_BAD_TEMPERATURE;
     if (!(bits & SV_ROW_BAD_LENGTH)) {
-        for (int i = 0; i < L; ++i) {
-            const int x = a.tokens[static_cast<long long>(b) * a.K + i];
-            if (x < 0 || x >= a.V) { bits |= SV_ROW_BAD_TOKEN; break; }
+        // Eight loads in flight at a time, no early exit.
+        const int32_t *x = a.tokens + static_cast<long long>(b) * a.K;
+        bool bad = false;
+        for (int i0 = 0; i0 < L; i0 += 8) {
+            int v[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) v[q] = (i0 + q < L) ? __ldg(x + i0 + q) : 0;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) bad |= (v[q] < 0 || v[q] >= a.V);
         }
+        if (bad) bits |= SV_ROW_BAD_TOKEN;
     }
     return bits;
 }
@@ -127,11 +136,16 @@ __device__ __forceinline__ int level_items(const VerifyArgs &a, int Lb, bool sam
     return a.C * (1 + ((i < Lb && sampled) ? 1 : 0));
 }
 
+constexpr int kPrologueSmemRows = 8192;   // rows whose (L, sampled) the scans read from shared memory
+
 __global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(VerifyArgs a) {
+    __shared__ int s_row[kPrologueSmemRows];   // L | sampled << 30, -1 for an invalid row
+    __shared__ int s_lvl[SV_MAX_K + 1];         // items per level
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     griddep_wait();
     griddep_launch_dependents();   // the stream kernel may take its SMs now
     const int K1 = a.K + 1;
+    const bool draft = a.zd != nullptr;
     // Rows: validity, effective length, first-rejection marker, counters.
     for (int b = tid; b < a.B; b += kPrologueThreads) {
         const int bits = row_errors(a, b);
@@ -148,17 +162,25 @@ __global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(VerifyArgs a
         a.row_j[b] = Lb;
         a.rcnt[b] = 0;
         for (int i = 0; i < K1; ++i) a.pcnt[static_cast<long long>(b) * K1 + i] = 0;
+        if (b < kPrologueSmemRows)
+            s_row[b] = Lb < 0 ? -1 : (Lb | ((draft && a.temp[b] > 0.f) ? (1 << 30) : 0));
     }
     __syncthreads();
     // Levels: warp w scans levels w, w + 32, ... over the rows.
-    const bool draft = a.zd != nullptr;
     for (int i = warp; i < K1; i += kPrologueThreads / 32) {
         int carry = 0;
         int *off = a.lvl_row + static_cast<long long>(i) * (a.B + 1);
         for (int b0 = 0; b0 < a.B; b0 += 32) {
             const int b = b0 + lane;
             int n = 0;
-            if (b < a.B) n = level_items(a, a.leff[b], draft && a.temp[b] > 0.f, i);
+            if (b < a.B) {
+                if (b < kPrologueSmemRows) {
+                    const int r = s_row[b];
+                    n = r < 0 ? 0 : level_items(a, r & 0xffff, (r >> 30) & 1, i);
+                } else {
+                    n = level_items(a, a.leff[b], draft && a.temp[b] > 0.f, i);
+                }
+            }
             int x = n;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -168,19 +190,20 @@ __global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(VerifyArgs a
             if (b < a.B) off[b] = carry + x - n;
             carry += __shfl_sync(0xffffffffu, x, 31);
         }
-        if (lane == 0) { off[a.B] = carry; a.lvl_off[i + 1] = carry; }
+        if (lane == 0) { off[a.B] = carry; s_lvl[i] = carry; }
     }
     __syncthreads();
     if (tid == 0) {
         int acc = 0;
         for (int i = 0; i < K1; ++i) {
-            const int c = a.lvl_off[i + 1];
+            const int c = s_lvl[i];
             a.lvl_off[i] = acc;
             acc += c;
         }
         a.lvl_off[K1] = acc;
         a.ctr[0] = 0;
         a.ctr[1] = acc;
+        a.ctr[2] = 0;
     }
 }
 
@@ -408,12 +431,12 @@ template <int ESIZE>
 __device__ void producer(const VerifyArgs &a, StreamSmem &sm, uint4 *ring, int total) {
     uint32_t it = 0;
     bool ok = true;
-    // Two claims in flight so that the counter's round trip overlaps the
-    // current item.  The row's status is read when the item's turn comes and
-    // again before each later stage: a rejection only ever lowers it, so a
-    // stale value costs redundant bytes, never a wrong result.
+    // The next claim is taken as the current item starts, so that the
+    // counter's round trip overlaps the item.  The row's status is read when
+    // the item's turn comes and again before each later stage: a rejection
+    // only ever lowers it, so a stale value costs redundant bytes, never a
+    // wrong result.
     int w = atomicAdd(&a.ctr[0], 1);
-    int wnext = atomicAdd(&a.ctr[0], 1);
     while (ok) {
         if (w >= total) {
             const int st = it % kStages;
@@ -426,7 +449,7 @@ __device__ void producer(const VerifyArgs &a, StreamSmem &sm, uint4 *ring, int t
         }
         const ItemRef cur = decode_item(a, w);
         const int rj = ld_relaxed(&a.row_j[cur.b]);
-        const int wfar = atomicAdd(&a.ctr[0], 1);
+        const int wnext = atomicAdd(&a.ctr[0], 1);
         // A row that has already rejected an earlier position never needs
         // this one: skip it without reading a byte.
         if (rj >= cur.i) {
@@ -467,7 +490,6 @@ __device__ void producer(const VerifyArgs &a, StreamSmem &sm, uint4 *ring, int t
             }
         }
         w = wnext;
-        wnext = wfar;
     }
     if (!ok) {
         // Unwind: report, then wait (bounded) for the copies still in flight
@@ -1098,6 +1120,230 @@ __device__ __forceinline__ void chunk_masses(const VerifyArgs &a, int b, int j, 
     }
 }
 
+
+// ---------------------------------------------------------------------------
+// Residual draw by sub-ranges of kSubUnits units.
+// ---------------------------------------------------------------------------
+constexpr int kSubUnits = 64;   // units per sub-range; chunk sizes are multiples of it
+constexpr int kRunUnits = 3;    // local units per lane in a located sub-range (66 / 32)
+constexpr int kResidParts = 1;  // resample CTAs per chunk of a residual draw
+
+// Draw weight of `count` (< one unit) elements from element `first`,
+// loaded directly (vector head or tail).
+template <int ESIZE, int MODE>
+__device__ __forceinline__ float partial_sum(const DrawCtx &c, int first, int count) {
+    constexpr int kPer = 16 / ESIZE;
+    UnitData u;
+    u.first = first;
+    u.count = count;
+    u.t = ld_partial_unit<ESIZE>(c.gt.base, first, count);
+    u.d = (MODE == kDrawResidual && c.aligned) ? ld_partial_unit<ESIZE>(c.gd.base, first, count)
+                                               : make_uint4(0u, 0u, 0u, 0u);
+    float t = 0.f;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) t += elem_weight<ESIZE, MODE>(c, u, e);
+    return t;
+}
+
+// Residual weight of every sub-range of part `part` of chunk `ch` into tbl.
+// Warp w takes the 256-unit blocks w, w + 8, ... of the part with eight units per lane in
+// flight; unit base + lane + 32 q lies in sub-range base / 64 + q / 2.  The
+// head joins sub-range 0 and the tail the last one.  Each sum has a fixed
+// order.
+template <int ESIZE>
+__device__ void residual_subranges(const DrawCtx &c, int ch, int part, int U, float *tbl) {
+    constexpr int kPer = 16 / ESIZE;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int PU = (U / kResidParts + kSubUnits - 1) / kSubUnits * kSubUnits;   // units per part
+    const int u0 = ch * U + part * PU;
+    const int u1 = max(u0, min(min(u0 + PU, (ch + 1) * U), c.gt.n16));
+    const int slast = c.gt.n16 > 0 ? (c.gt.n16 - 1) / kSubUnits : 0;
+    const uint32_t pw = neg_inf_word<ESIZE>();
+    const uint4 pad = make_uint4(pw, pw, pw, pw);
+    int nblk = (u1 - u0 + 255) / 256;
+    if (c.gt.n16 == 0 && ch == 0 && part == 0) nblk = 1;   // head and tail only
+    for (int blk = warp; blk < nblk; blk += kDrawWarps) {
+        const int base = u0 + blk * 256;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        if (c.aligned) {
+            uint4 t[8], d[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int u = base + lane + 32 * q;
+                const long long off = static_cast<long long>(u) * 16;
+                t[q] = u < u1 ? ld_reuse(c.gt.body + off) : pad;
+                d[q] = u < u1 ? ld_reuse(c.gd.body + off) : pad;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[q >> 1] += body_sum<ESIZE, kDrawResidual>(c, t[q], d[q]);
+        } else {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int u = base + lane + 32 * q;
+                if (u < u1) {
+                    UnitData ud;
+                    ud.t = ld_reuse(c.gt.body + static_cast<long long>(u) * 16);
+                    ud.d = make_uint4(0u, 0u, 0u, 0u);
+                    ud.count = kPer;
+                    ud.first = c.gt.head + u * kPer;
+#pragma unroll
+                    for (int e = 0; e < kPer; ++e)
+                        acc[q >> 1] += elem_weight<ESIZE, kDrawResidual>(c, ud, e);
+                }
+            }
+        }
+        const int s0 = base / kSubUnits;
+        if (lane == 0) {
+            if (s0 == 0 && c.gt.head > 0) acc[0] += partial_sum<ESIZE, kDrawResidual>(c, 0, c.gt.head);
+            if (c.gt.tail > 0 && slast >= s0 && slast < s0 + 4)
+                acc[slast - s0] += partial_sum<ESIZE, kDrawResidual>(
+                    c, c.gt.head + c.gt.n16 * kPer, c.gt.tail);
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], o);
+        if (lane == 0) {
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int s = s0 + r;
+                if (s * kSubUnits < u1 || (c.gt.n16 == 0 && s == 0)) tbl[s] = acc[r];
+            }
+        }
+    }
+}
+
+// Inverse CDF over the sub-range table (one warp): the total R (rounds of
+// 32 entries, a fixed tree per round, rounds in order), then the first
+// entry with positive weight whose running sum exceeds t = u R.  *sel = -1
+// with *zero set when R is 0; if rounding leaves t at or past the end, the
+// last entry with weight is returned with *fb set and an infinite target.
+__device__ void scan_table(const float *tb, int nsub, float u, int *sel_out, float *d_out,
+                           bool *zero, bool *fb) {
+    constexpr int kRounds = 8;
+    const int lane = threadIdx.x & 31;
+    float R = 0.f;
+    int lastpos = -1;
+    float v[kRounds];
+    for (int base = 0; base < nsub; base += 32 * kRounds) {
+#pragma unroll
+        for (int q = 0; q < kRounds; ++q) {
+            const int s = base + q * 32 + lane;
+            v[q] = s < nsub ? __ldcg(tb + s) : 0.f;
+        }
+#pragma unroll
+        for (int q = 0; q < kRounds; ++q) {
+            if (v[q] > 0.f) lastpos = base + q * 32 + lane;
+            float r = v[q];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+            R += r;
+        }
+    }
+    *sel_out = -1;
+    *d_out = 0.f;
+    if (!(R > 0.f)) {
+        *zero = true;
+        return;
+    }
+    const float t = u * R;
+    int sel = -1;
+    float dsel = 0.f, cum = 0.f;
+    const bool resident = nsub <= 32 * kRounds;   // pass 1 left the whole table in v
+    for (int base = 0; base < nsub && sel < 0; base += 32 * kRounds) {
+        if (!resident) {
+#pragma unroll
+            for (int q = 0; q < kRounds; ++q) {
+                const int s = base + q * 32 + lane;
+                v[q] = s < nsub ? __ldcg(tb + s) : 0.f;
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < kRounds; ++q) {
+            if (sel >= 0) break;
+            float incl = v[q];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const unsigned hit = __ballot_sync(0xffffffffu, v[q] > 0.f && cum + incl > t);
+            if (hit) {
+                const int l = __ffs(hit) - 1;
+                sel = base + q * 32 + l;
+                dsel = t - (cum + __shfl_sync(0xffffffffu, incl - v[q], l));
+            } else {
+                float r = v[q];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+                cum += r;
+            }
+        }
+    }
+    if (sel < 0) {
+        sel = __reduce_max_sync(0xffffffffu, lastpos);
+        dsel = __int_as_float(0x7f800000);
+        *fb = true;
+    }
+    *sel_out = sel;
+    *d_out = dsel;
+}
+
+// Smallest element of the sub-range described by c (ubody0, nbody, head,
+// tail) whose cumulative weight exceeds d (one warp; lane l owns local units
+// 3l .. 3l+2: 0 = head, 1..nbody = body units, nbody+1 = tail).  If
+// rounding leaves d at or past the total, the last element with positive
+// weight is returned and *fb is set; -1 if there is none.
+template <int ESIZE, int MODE>
+__device__ int locate_in_subrange(const DrawCtx &c, float d, bool *fb) {
+    constexpr int kPer = 16 / ESIZE;
+    const int lane = threadIdx.x & 31;
+    const int NU = c.nbody + 2;
+    const int l0 = min(lane * kRunUnits, NU);
+    const int l1 = min(l0 + kRunUnits, NU);
+    UnitData ud[kRunUnits];
+#pragma unroll
+    for (int q = 0; q < kRunUnits; ++q)
+        ud[q] = (l0 + q < l1) ? load_unit<ESIZE, MODE>(c, l0 + q) : empty_unit();
+    float mine = 0.f;
+    int lastpos = -1;
+#pragma unroll
+    for (int q = 0; q < kRunUnits; ++q)
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) {
+            const float w = elem_weight<ESIZE, MODE>(c, ud[q], e);
+            if (w > 0.f) lastpos = ud[q].first + e;
+            mine += w;
+        }
+    float incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    float excl = __shfl_up_sync(0xffffffffu, incl, 1);
+    if (lane == 0) excl = 0.f;
+    int y = -1;
+    const unsigned hit = __ballot_sync(0xffffffffu, incl > d);
+    if (hit && lane == __ffs(hit) - 1) {
+        float cum = excl;
+#pragma unroll
+        for (int q = 0; q < kRunUnits; ++q)
+#pragma unroll
+            for (int e = 0; e < kPer; ++e) {
+                const float w = elem_weight<ESIZE, MODE>(c, ud[q], e);
+                if (y < 0 && w > 0.f && cum + w > d) y = ud[q].first + e;
+                cum += w;
+            }
+    }
+    y = __reduce_max_sync(0xffffffffu, y);
+    if (y < 0) {
+        *fb = true;
+        y = __reduce_max_sync(0xffffffffu, lastpos);
+    }
+    return y;
+}
+
 // Per-row result of the accept test and the set-up of the final draw.
 struct __align__(16) DrawRecord {
     int j;        // first rejected position, or L
@@ -1242,6 +1488,14 @@ __global__ void __launch_bounds__(kDrawThreads) accept_kernel(VerifyArgs a) {
         r.cd = resid ? log2f(ds.s[K + 1 + j]) : 0.f;
         r.note = note;
         *rec = r;
+        // Resample work: every chunk of a residual draw, the selected chunk
+        // of a p-mass draw.
+        if (resid) {
+            const int base = atomicAdd(&a.ctr[2], C * kResidParts);
+            for (int q = 0; q < C * kResidParts; ++q) a.work[base + q] = b * C * kResidParts + q;
+        } else {
+            a.work[atomicAdd(&a.ctr[2], 1)] = (b * C + (ds.gsel < 0 ? 0 : ds.gsel)) * kResidParts;
+        }
     }
 }
 
@@ -1257,13 +1511,17 @@ __global__ void __launch_bounds__(kDrawThreads, 3) resample_kernel(VerifyArgs a)
     __shared__ DrawSmem ds;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     griddep_wait();
-    const int b = blockIdx.x / a.C;
-    const int chunk = blockIdx.x - b * a.C;
+    // CTA w takes work entry w; the entries of every row with a draw were
+    // appended by the accept kernel, so all the work sits in the first CTAs.
+    if (static_cast<int>(blockIdx.x) >= __ldcg(&a.ctr[2])) return;
+    const int entry = __ldcg(&a.work[blockIdx.x]);
+    const int part = entry % kResidParts;
+    const int b = entry / kResidParts / a.C;
+    const int chunk = entry / kResidParts - b * a.C;
     const int K = a.K, C = a.C;
     const DrawRecord r = a.rec[b];   // written by the previous launch
     if (r.mode == kDrawDone) return;
     const bool resid = r.mode == kDrawResidual;
-    if (!resid && chunk != (r.csel < 0 ? 0 : r.csel)) return;
     const int j = r.j;
 
     DrawCtx c;
@@ -1290,66 +1548,70 @@ __global__ void __launch_bounds__(kDrawThreads, 3) resample_kernel(VerifyArgs a)
     int note = r.note;
     int csel = r.csel;
     float d = r.d;
-    bool have_segments = false;
+    int y = -1;
+    bool fb = false;
     if (resid) {
+        // Residual weight of this chunk by sub-ranges; the last chunk CTA of
+        // the row (atomic counter, no waiting) picks the sub-range from the
+        // row's table and the token inside it.
         set_chunk(chunk);
-        const float segtot = warp_segment_total<ESIZE, kDrawResidual>(c);
-        if (lane == 0) {
-            a.rseg[(static_cast<long long>(b) * C + chunk) * kDrawWarps + warp] = segtot;
-            __threadfence();
-        }
+        float *tb = a.rtbl + static_cast<long long>(b) * a.nsub;
+        residual_subranges<ESIZE>(c, chunk, part, a.U, tb);
         __syncthreads();
         if (tid == 0) {
+            __threadfence();
             const int done = atomicAdd(&a.rcnt[b], 1) + 1;
             __threadfence();
-            ds.last = (done == C);
+            ds.last = (done == C * kResidParts);
         }
         __syncthreads();
         if (!ds.last) return;
-        if (tid < C) {
-            float t = 0.f;
-            for (int g = 0; g < kDrawWarps; ++g)
-                t += __ldcg(&a.rseg[(static_cast<long long>(b) * C + tid) * kDrawWarps + g]);
-            ds.cm[tid] = t;
+        if (warp == 0) {
+            bool zero = false, fbw = false;
+            const int nsub = max(1, (c.gt.n16 + kSubUnits - 1) / kSubUnits);
+            int sel;
+            float dsel;
+            scan_table(tb, nsub, r.u, &sel, &dsel, &zero, &fbw);
+            int yw = -1;
+            if (!zero && sel >= 0) {
+                DrawCtx cs = c;
+                cs.ubody0 = sel * kSubUnits;
+                cs.nbody = max(0, min(kSubUnits, c.gt.n16 - cs.ubody0));
+                cs.has_head = (sel == 0) && c.gt.head > 0;
+                cs.has_tail = (sel == nsub - 1) && c.gt.tail > 0;
+                yw = locate_in_subrange<ESIZE, kDrawResidual>(cs, dsel, &fbw);
+            }
+            if (lane == 0) {
+                ds.ysel = yw;
+                ds.gsel = zero ? 1 : 0;
+                ds.lastpos = fbw ? 1 : 0;
+            }
         }
         __syncthreads();
-        if (tid == 0) {
-            float dd = 0.f;
-            int cs = select_chunk(ds.cm, C, r.u, &dd);
-            int m = kDrawResidual;
-            if (cs < 0) {
-                // The residual vanished to rounding (p_j == q_j): draw from p_j.
-                m = kDrawP;
+        if (ds.gsel == 0) {
+            y = ds.ysel;
+            fb = ds.lastpos != 0;
+            csel = -1;
+        } else {
+            // The residual vanished to rounding (p_j == q_j): draw from p_j.
+            if (tid == 0) {
+                float dd = 0.f;
                 note |= SV_NOTE_ZERO_RESIDUAL;
                 chunk_masses_serial(a, b, j, r.mt, r.k, ds.cm);
-                cs = select_chunk(ds.cm, C, r.u, &dd);
+                ds.gsel = select_chunk(ds.cm, C, r.u, &dd);
+                ds.dsel = dd;
             }
-            ds.gsel = cs;
-            ds.dsel = dd;
-            ds.lastpos = m;
-        }
-        __syncthreads();
-        csel = ds.gsel;
-        d = ds.dsel;
-        if (ds.lastpos == kDrawP) {
+            __syncthreads();
+            csel = ds.gsel;
+            d = ds.dsel;
             c.mode = kDrawP;
             c.ct = 0.f;
-        } else {
-            have_segments = true;
         }
     }
-    int y = -1;
-    bool fb = false;
     if (csel >= 0) {
         set_chunk(csel);
-        if (have_segments) {
-            if (tid < kDrawWarps)
-                ds.wsum[tid] =
-                    __ldcg(&a.rseg[(static_cast<long long>(b) * C + csel) * kDrawWarps + tid]);
-        } else {
-            const float segtot = segment_total_any<ESIZE>(c);
-            if (lane == 0) ds.wsum[warp] = segtot;
-        }
+        const float segtot = segment_total_any<ESIZE>(c);
+        if (lane == 0) ds.wsum[warp] = segtot;
         __syncthreads();
         y = chunk_locate_any<ESIZE>(c, d, ds, &fb);
     }
@@ -1374,7 +1636,9 @@ template <int ESIZE> static const void *stream_kernel_ptr() {
 // ---------------------------------------------------------------------------
 struct Plan {
     int C, U, S;
-    size_t off_rcnt, off_leff, off_rowj, off_pcnt, off_lvloff, off_lvlrow, off_part, off_rseg,
+    int nsub;
+    size_t off_rcnt, off_leff, off_rowj, off_pcnt, off_lvloff, off_lvlrow, off_part, off_rtbl,
+        off_work,
         off_rec, bytes;
 };
 
@@ -1387,7 +1651,8 @@ static bool make_plan(int B, int K, int V, sv_dtype dtype, Plan *p) {
     int C = static_cast<int>((n16 + kMaxUnitsPerItem - 1) / kMaxUnitsPerItem);
     if (C < 1) C = 1;
     if (C > kMaxChunks) return false;
-    const int U = static_cast<int>((n16 + C - 1) / C);
+    int U = static_cast<int>((n16 + C - 1) / C);
+    U = (U + kSubUnits - 1) / kSubUnits * kSubUnits;   // chunks hold whole sub-ranges
     const int S = 2 * K + 1;
     const long long items = static_cast<long long>(B) * S * C;
     if (items >= INT_MAX / 2 || static_cast<long long>(B) * C >= INT_MAX / 2) return false;
@@ -1402,7 +1667,10 @@ static bool make_plan(int B, int K, int V, sv_dtype dtype, Plan *p) {
     p->off_lvloff = off; off = align16(off + sizeof(int) * static_cast<size_t>(K + 2));
     p->off_lvlrow = off; off = align16(off + sizeof(int) * static_cast<size_t>(K + 1) * (B + 1));
     p->off_part = off;   off = align16(off + sizeof(float4) * static_cast<size_t>(items));
-    p->off_rseg = off;   off = align16(off + sizeof(float) * static_cast<size_t>(B) * C * kDrawWarps);
+    p->nsub = static_cast<int>((n16 + kSubUnits - 1) / kSubUnits);
+    if (p->nsub < 1) p->nsub = 1;
+    p->off_rtbl = off;   off = align16(off + sizeof(float) * static_cast<size_t>(B) * p->nsub);
+    p->off_work = off;   off = align16(off + sizeof(int) * static_cast<size_t>(B) * C * kResidParts);
     p->off_rec = off;    off = align16(off + sizeof(DrawRecord) * static_cast<size_t>(B));
     p->bytes = off;
     return true;
@@ -1462,7 +1730,9 @@ static sv_status verify_impl(const void *zt, const void *zd, sv_dtype dtype, int
     a.lvl_off = reinterpret_cast<int *>(w + p.off_lvloff);
     a.lvl_row = reinterpret_cast<int *>(w + p.off_lvlrow);
     a.part = reinterpret_cast<float4 *>(w + p.off_part);
-    a.rseg = reinterpret_cast<float *>(w + p.off_rseg);
+    a.rtbl = reinterpret_cast<float *>(w + p.off_rtbl);
+    a.nsub = p.nsub;
+    a.work = reinterpret_cast<int *>(w + p.off_work);
     a.rec = reinterpret_cast<DrawRecord *>(w + p.off_rec);
 
     const int grid = stream_grid(es, static_cast<long long>(B) * p.S * p.C);
@@ -1479,7 +1749,7 @@ static sv_status verify_impl(const void *zt, const void *zd, sv_dtype dtype, int
                   : launch_pdl(stream_kernel<2>, dim3(grid), dim3(kBlock), kRingBytes, st, a);
     if (e != cudaSuccess) return note_cuda(e);
     profile_mark_end(st);
-    const unsigned draw_grid = static_cast<unsigned>(B) * static_cast<unsigned>(p.C);
+    const unsigned draw_grid = static_cast<unsigned>(B) * static_cast<unsigned>(p.C) * kResidParts;
     if (es == 4) {
         e = launch_pdl(accept_kernel<4>, dim3(B), dim3(kDrawThreads), 0, st, a);
         if (e == cudaSuccess)
