@@ -57,6 +57,8 @@ def lib():
         L.oracle_schedule_admit.argtypes = [vp, i32, i32, vp, i32, vp, vp, vp]
         L.oracle_schedule_admit.restype = i32
         L.oracle_ndiag.restype = i32
+        L.oracle_sts_fit.argtypes = [vp, vp, i32, i32, dbl, dbl, vp, vp]
+        L.oracle_sts_fit.restype = ctypes.c_long
         assert L.oracle_ndiag() == NDIAG
         _lib = L
     return _lib
@@ -199,3 +201,21 @@ def default_threads() -> int:
         return len(os.sched_getaffinity(0))
     except AttributeError:  # pragma: no cover
         return os.cpu_count() or 1
+
+
+def sts_fit(logits, accept, tmin=1e-2, tmax=1e2):
+    """Per-position temperature scaling of the confidence head on held-out
+    blocks: logits [N, K] float32 (confidence = sigmoid), accepted lengths
+    [N] int32 (position i observed iff i <= a, survived iff i < a; a < 0
+    skips the block).  Returns (T [K] fp64, (ece_before, ece_after),
+    observed count)."""
+    l = np.ascontiguousarray(logits, dtype=np.float32)
+    N, K = l.shape
+    a = np.ascontiguousarray(accept, dtype=np.int32).reshape(-1)
+    T = np.zeros(K, dtype=np.float64)
+    ece = np.zeros(2, dtype=np.float64)
+    n = lib().oracle_sts_fit(_p(l), _p(a), N, K, ctypes.c_double(tmin), ctypes.c_double(tmax),
+                             _p(T), _p(ece))
+    if n < 0:
+        raise ValueError("bad arguments")
+    return T, (float(ece[0]), float(ece[1])), int(n)

@@ -520,3 +520,119 @@ int oracle_schedule_admit(const float *conf, int B, int K, const float *speed, i
     free(c);
     return k;
 }
+
+/* ------------------------------------------------------------------------
+ * Per-position temperature scaling of the confidence head.
+ *
+ * umans.ai, "DeepSeek V4 Pro DSpark: the model isn't ready, the
+ * architecture is", section "What DSpark adds", item "2. Verify smarter":
+ * the head's raw confidences are overconfident (3-8% expected calibration
+ * error) and a per-position temperature fitted on held-out data brings
+ * them to about 1%.  zhichai.net DSpark topic, "Under the hood": the head
+ * is calibrated by Sequential Temperature Scaling.
+ *
+ * Held-out data: N draft blocks, the head's logits l[n, i] (confidence =
+ * sigmoid(l)) for positions i = 0..K-1, and the accepted length a[n] in
+ * [0, K] seen when the block was verified (a[n] < 0 skips the block).  The
+ * head predicts survival given that every earlier position survived, so
+ * position i of block n is observed iff i <= a[n], and survived iff
+ * i < a[n]: each position is fitted on the blocks that reached it.
+ *
+ * T_i minimises the binary negative log-likelihood of the observed outcomes
+ * at position i under confidence sigmoid(l / T).  With beta = 1/T and
+ * s = +1 (survived) or -1,
+ *     NLL(beta)  = sum log(1 + exp(-s beta l))           (convex in beta)
+ *     NLL'(beta) = sum -s l sigmoid(-s beta l)           (non-decreasing)
+ * The minimiser over [1/tmax, 1/tmin] is the end point where NLL' does not
+ * change sign there, else the root of NLL' found by bisection (80
+ * halvings, past fp64 resolution).  No observed sample, or NLL' zero at both
+ * ends (every observed l is 0), gives T = 1.
+ *
+ * ECE over every observed (n, i), 15 equal-width confidence bins (the last
+ * one closed): ECE = sum over bins |sum (y - conf)| / (observed count), for
+ * conf = sigmoid(l) (ece[0]) and conf = sigmoid(l / T_i) (ece[1]).
+ * Returns the number of observed (n, i), or -1 on bad arguments.
+ * ------------------------------------------------------------------------ */
+static double sts_sigmoid(double x)
+{
+    if (x >= 0.0) return 1.0 / (1.0 + exp(-x));
+    double e = exp(x);
+    return e / (1.0 + e);
+}
+
+static double sts_deriv(const float *l, const int32_t *a, int N, int K, int i, double beta,
+                        long *count)
+{
+    double g = 0.0;
+    long c = 0;
+    for (int n = 0; n < N; ++n) {
+        if (a[n] < 0 || i > a[n]) continue;
+        double s = (i < a[n]) ? 1.0 : -1.0;
+        double x = (double)l[(size_t)n * K + i];
+        g += -s * x * sts_sigmoid(-s * beta * x);
+        ++c;
+    }
+    *count = c;
+    return g;
+}
+
+#define STS_BINS 15
+
+static void sts_ece(const float *l, const int32_t *a, int N, int K, const double *T,
+                    double *out)
+{
+    double diff[STS_BINS];
+    long cnt = 0;
+    for (int m = 0; m < STS_BINS; ++m) diff[m] = 0.0;
+    for (int n = 0; n < N; ++n) {
+        if (a[n] < 0) continue;
+        for (int i = 0; i < K && i <= a[n]; ++i) {
+            double conf = sts_sigmoid((double)l[(size_t)n * K + i] / (T ? T[i] : 1.0));
+            int m = (int)(conf * STS_BINS);
+            if (m >= STS_BINS) m = STS_BINS - 1;
+            diff[m] += ((i < a[n]) ? 1.0 : 0.0) - conf;
+            ++cnt;
+        }
+    }
+    double e = 0.0;
+    for (int m = 0; m < STS_BINS; ++m) e += fabs(diff[m]);
+    *out = cnt > 0 ? e / (double)cnt : 0.0;
+}
+
+long oracle_sts_fit(const float *l, const int32_t *a, int N, int K, double tmin, double tmax,
+                    double *T, double *ece)
+{
+    if (!l || !a || !T || N < 0 || K < 1 || !(tmin > 0.0) || !(tmax > tmin)) return -1;
+    long total = 0;
+    for (int n = 0; n < N; ++n)
+        if (a[n] >= 0) total += (a[n] < K ? a[n] + 1 : K);
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int i = 0; i < K; ++i) {
+        long c = 0;
+        const double lo0 = 1.0 / tmax, hi0 = 1.0 / tmin;
+        double glo = sts_deriv(l, a, N, K, i, lo0, &c);
+        if (c == 0) { T[i] = 1.0; continue; }
+        double ghi = sts_deriv(l, a, N, K, i, hi0, &c);
+        double beta;
+        if (glo == 0.0 && ghi == 0.0) {
+            beta = 1.0;
+        } else if (glo >= 0.0) {
+            beta = lo0;
+        } else if (ghi <= 0.0) {
+            beta = hi0;
+        } else {
+            double lo = lo0, hi = hi0;
+            for (int it = 0; it < 80; ++it) {
+                double mid = 0.5 * (lo + hi);
+                if (sts_deriv(l, a, N, K, i, mid, &c) < 0.0) lo = mid; else hi = mid;
+            }
+            beta = 0.5 * (lo + hi);
+        }
+        T[i] = 1.0 / beta;
+    }
+    if (ece) {
+        sts_ece(l, a, N, K, NULL, &ece[0]);
+        sts_ece(l, a, N, K, T, &ece[1]);
+    }
+    return total;
+}
