@@ -294,6 +294,33 @@ def run_ours(args, rank, world, local_rank):
                  "candidates": B * K, "admitted": int(adm_len.sum().item()),
                  "tau": round(float(adm_tau.item()), 6), "bound": "latency (one CTA)"}
 
+    # ---- confidence-head calibration (per-position temperature scaling) on
+    # synthetic held-out blocks: the fit that produces the confidences -------
+    calib = None
+    if rank == 0:
+        hl, ha = workloads.sts_heldout(262144, K, seed=17)
+        hlt = torch.from_numpy(hl).to(dev)
+        hat = torch.from_numpy(ha).to(dev)
+        hT = torch.empty(K, dtype=torch.float32, device=dev)
+        hece = torch.empty(2, dtype=torch.float32, device=dev)
+        hws = torch.empty(sv.sv_sts_workspace_bytes(262144, K), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            sv.sv_sts_fit(hlt, hat, hT, hece, hws)
+        torch.cuda.synchronize()
+        n_fit = max(1, min(args.steps, 10))
+        e0.record(stream)
+        for _ in range(n_fit):
+            sv.sv_sts_fit(hlt, hat, hT, hece, hws)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        calib = {"kernel": "sv::sts_eval_kernel + sts_final_kernel",
+                 "us_per_call": round(e0.elapsed_time(e1) / n_fit * 1e3, 2),
+                 "blocks": 262144, "positions": K,
+                 "ece_before": round(float(hece[0].item()), 5),
+                 "ece_after": round(float(hece[1].item()), 5),
+                 "bound": "latency (43 dependent launches)"}
+        del hlt, hat, hws
+
     # ---- end-to-end through host buffers ------------------------------------
     e2e = None
     if not args.no_e2e:
@@ -390,6 +417,7 @@ def run_ours(args, rank, world, local_rank):
                "e2e": e2e, "gpu_launches": args.steps * (sv.sv_verify_launches()
                                                          + (1 if fixed is None else 0)),
                "roofline": roofline, "cpu_baseline": cpu, "clocks": clk, "admission": admit,
+               "calibration": calib,
                "device_status": st, "impl": "ours"}
         print(json.dumps(out), flush=True)
     del batch

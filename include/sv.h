@@ -129,6 +129,55 @@ sv_status sv_schedule_admit(const float *conf, int B, int K, const float *speed,
                             int32_t *lengths, float *tau_out, void *stream);
 
 /*
+ * sv_sts_fit -- per-position temperature of the confidence head, fitted on
+ * held-out blocks (the calibration that feeds sv_schedule / sv_schedule_admit).
+ *
+ * Defined by: umans.ai, "DeepSeek V4 Pro DSpark: the model isn't ready, the
+ * architecture is", section "What DSpark adds", item "2. Verify smarter"
+ * (the head's raw confidence is overconfident by 3-8% expected calibration
+ * error; a per-position temperature fitted on held-out data brings it to
+ * about 1%); zhichai.net DSpark topic, "Under the hood" (Sequential
+ * Temperature Scaling).
+ *
+ * The head predicts survival of position i given that every earlier
+ * position survived, so position i of block n is observed iff
+ * i <= accept_len[n] and survived iff i < accept_len[n] (blocks with
+ * accept_len < 0 are skipped).  T_i = 1/beta_i minimises
+ * sum over observed n of log(1 + exp(-s beta logits[n, i])), s = +1 survived,
+ * -1 not, over beta in [1/tmax, 1/tmin] (convex in beta; fp64 sums).  A
+ * position that no block reached, or whose observed logits are all 0, gets
+ * T = 1.  The expected calibration error uses 15 equal-width bins over every
+ * observed (n, i): sum over bins |sum (y - conf)| / count.
+ *
+ *   logits       device float32 [N, K], read only: the head's logits
+ *                (confidence = sigmoid(logit)).
+ *   accept_len   device int32 [N], read only: accepted length of each
+ *                held-out block (e.g. out_accept_len of sv_verify).
+ *   N, K         1 <= N, 1 <= K <= SV_MAX_K.
+ *   tmin, tmax   0 < tmin < tmax, finite: the temperature range.
+ *   temperature  device float32 [K], written.
+ *   ece          device float32 [2], nullable: calibration error before
+ *                (T = 1) and after the fit.
+ *   workspace    device scratch of sv_sts_workspace_bytes(N, K) bytes,
+ *                16-byte aligned, owned by the caller.
+ * Returns SV_OK, SV_ERR_ARG, SV_ERR_SHAPE, SV_ERR_WORKSPACE or SV_ERR_CUDA.
+ * Enqueues 43 launches and one memset on `stream`; never synchronises.
+ */
+size_t sv_sts_workspace_bytes(int N, int K);
+sv_status sv_sts_fit(const float *logits, const int32_t *accept_len, int N, int K, float tmin,
+                     float tmax, float *temperature, float *ece, void *workspace,
+                     size_t workspace_bytes, void *stream);
+
+/*
+ * sv_sts_apply -- calibrated confidences conf[n, i] = sigmoid(logits[n, i] /
+ * temperature[i]) (same passages as sv_sts_fit), ready for sv_schedule.
+ *   logits [N, K], temperature [K] read only; conf_out [N, K] written; all
+ *   device float32.  Returns SV_OK, SV_ERR_ARG, SV_ERR_SHAPE or SV_ERR_CUDA.
+ */
+sv_status sv_sts_apply(const float *logits, const float *temperature, int N, int K,
+                       float *conf_out, void *stream);
+
+/*
  * sv_verify_workspace_bytes -- device scratch that sv_verify needs for
  * (B, K, V, dtype): per-row work counters, per-row work offsets and the
  * per-chunk softmax partials.  Returns 0 for unsupported sizes.

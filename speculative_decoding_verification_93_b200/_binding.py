@@ -46,6 +46,11 @@ def lib():
                              ctypes.c_size_t)
     L.sv_schedule.argtypes = [vp, i32, i32, ctypes.c_float, vp, vp]
     L.sv_schedule_admit.argtypes = [vp, i32, i32, vp, i32, vp, vp, vp]
+    L.sv_sts_workspace_bytes.argtypes = [i32, i32]
+    L.sv_sts_workspace_bytes.restype = sz
+    L.sv_sts_fit.argtypes = [vp, vp, i32, i32, ctypes.c_float, ctypes.c_float, vp, vp, vp, sz,
+                             vp]
+    L.sv_sts_apply.argtypes = [vp, vp, i32, i32, vp, vp]
     L.sv_verify_workspace_bytes.argtypes = [i32, i32, i32, i32]
     L.sv_verify_workspace_bytes.restype = sz
     L.sv_verify.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, u64, i64, vp, vp, vp, sz, vp,
@@ -61,7 +66,8 @@ def lib():
     L.sv_profile_read.restype = i32
     L.sv_status_string.argtypes = [i32]
     L.sv_status_string.restype = ctypes.c_char_p
-    for name in ("sv_schedule", "sv_schedule_admit", "sv_verify", "sv_verify_debug", "sv_verify_noalloc",
+    for name in ("sv_schedule", "sv_schedule_admit", "sv_sts_fit", "sv_sts_apply", "sv_verify",
+                 "sv_verify_debug", "sv_verify_noalloc",
                  "sv_philox_uniforms",
                  "sv_philox4x32_10", "sv_profile_begin"):
         getattr(L, name).restype = i32
@@ -119,6 +125,35 @@ def sv_schedule_admit(conf: torch.Tensor, speed: torch.Tensor, lengths: torch.Te
     _check("sv_schedule_admit", lib().sv_schedule_admit(
         _ptr(conf), B, K, _ptr(speed), speed.numel(), _ptr(lengths), _ptr(tau_out),
         _stream(stream, conf)))
+
+
+def sv_sts_workspace_bytes(N: int, K: int) -> int:
+    return int(lib().sv_sts_workspace_bytes(N, K))
+
+
+def sv_sts_fit(logits: torch.Tensor, accept_len: torch.Tensor, temperature: torch.Tensor,
+               ece: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+               tmin: float = 1e-2, tmax: float = 1e2, stream=None) -> None:
+    _need(logits, torch.float32, "logits")
+    _need(accept_len, torch.int32, "accept_len")
+    _need(temperature, torch.float32, "temperature")
+    N, K = logits.shape
+    if workspace is None:
+        workspace = torch.empty(sv_sts_workspace_bytes(N, K), dtype=torch.uint8,
+                                device=logits.device)
+    _check("sv_sts_fit", lib().sv_sts_fit(
+        _ptr(logits), _ptr(accept_len), N, K, float(tmin), float(tmax), _ptr(temperature),
+        _ptr(ece), _ptr(workspace), workspace.numel(), _stream(stream, logits)))
+
+
+def sv_sts_apply(logits: torch.Tensor, temperature: torch.Tensor, conf_out: torch.Tensor,
+                 stream=None) -> None:
+    _need(logits, torch.float32, "logits")
+    _need(temperature, torch.float32, "temperature")
+    _need(conf_out, torch.float32, "conf_out")
+    N, K = logits.shape
+    _check("sv_sts_apply", lib().sv_sts_apply(_ptr(logits), _ptr(temperature), N, K,
+                                              _ptr(conf_out), _stream(stream, logits)))
 
 
 def sv_verify_workspace_bytes(B: int, K: int, V: int, dtype: int) -> int:

@@ -213,3 +213,20 @@ def to_host_logits(t: torch.Tensor) -> np.ndarray:
     if t.dtype == torch.float32:
         return t.numpy()
     raise TypeError(t.dtype)
+
+
+def sts_heldout(N: int, K: int, seed: int = 0, kappa=(1.3, 2.2), mu: float = 1.8,
+                sigma: float = 1.0):
+    """Synthetic held-out blocks for the confidence head's calibration: a
+    true survival logit l* ~ N(mu, sigma^2) per (block, position); survival
+    drawn left to right from sigmoid(l*) until the first failure (the
+    accepted length a); the head reports l = kappa_i * l*, overconfident by
+    a factor kappa_i spread evenly over `kappa` along the block.  Returns
+    (logits [N, K] float32, accept [N] int32), numpy."""
+    rng = np.random.default_rng(seed)
+    lstar = rng.normal(mu, sigma, size=(N, K))
+    kap = np.linspace(kappa[0], kappa[1], K)
+    logits = (lstar * kap).astype(np.float32)
+    survive = rng.random((N, K)) < 1.0 / (1.0 + np.exp(-lstar))
+    accept = np.where(survive.all(axis=1), K, np.argmin(survive, axis=1)).astype(np.int32)
+    return logits, accept

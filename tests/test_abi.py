@@ -96,3 +96,27 @@ def test_python_binding_marshals_only():
     with pytest.raises(TypeError):
         sv.sv_verify(zt.double(), None, torch.zeros(2, 2, dtype=torch.int32),
                      torch.zeros(2, dtype=torch.int32), torch.zeros(2), 0, None, None, None)
+
+
+def test_sts_arguments_rejected_on_host():
+    L = sv.lib()
+    v = ctypes.c_void_p
+    big = 1 << 30
+    ok = dict(l=1 << 20, a=1 << 21, N=100, K=4, tmin=0.01, tmax=100.0, T=1 << 22, ws=1 << 23,
+              wsb=big)
+
+    def call(**kw):
+        d = dict(ok)
+        d.update(kw)
+        return L.sv_sts_fit(v(d["l"]) if d["l"] else None, v(d["a"]) if d["a"] else None,
+                            d["N"], d["K"], ctypes.c_float(d["tmin"]), ctypes.c_float(d["tmax"]),
+                            v(d["T"]) if d["T"] else None, None, v(d["ws"]) if d["ws"] else None,
+                            d["wsb"], None)
+    assert call(l=0) == 1 and call(a=0) == 1 and call(T=0) == 1 and call(ws=0) == 1
+    assert call(tmin=0.0) == 1 and call(tmax=0.005) == 1 and call(tmax=float("inf")) == 1
+    assert call(K=65) == 2 and call(K=0) == 2 and call(N=0) == 2
+    assert call(wsb=16) == 4
+    assert call(ws=(1 << 23) + 4) == 1
+    assert sv.sv_sts_workspace_bytes(100, 4) > 0 and sv.sv_sts_workspace_bytes(100, 65) == 0
+    assert L.sv_sts_apply(None, v(1), 1, 1, v(1), None) == 1
+    assert L.sv_sts_apply(v(1), v(1), 1, 65, v(1), None) == 2
