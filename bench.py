@@ -313,12 +313,12 @@ def run_ours(args, rank, world, local_rank):
             sv.sv_sts_fit(hlt, hat, hT, hece, hws)
         e1.record(stream)
         torch.cuda.synchronize()
-        calib = {"kernel": "sv::sts_eval_kernel + sts_final_kernel",
+        calib = {"kernel": "sv::sts_fit_kernel",
                  "us_per_call": round(e0.elapsed_time(e1) / n_fit * 1e3, 2),
                  "blocks": 262144, "positions": K,
                  "ece_before": round(float(hece[0].item()), 5),
                  "ece_after": round(float(hece[1].item()), 5),
-                 "bound": "latency (43 dependent launches)"}
+                 "bound": "fp64 sigmoid per observed (block, position) and pass; grid barriers"}
         del hlt, hat, hws
 
     # ---- end-to-end through host buffers ------------------------------------

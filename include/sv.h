@@ -161,7 +161,8 @@ sv_status sv_schedule_admit(const float *conf, int B, int K, const float *speed,
  *   workspace    device scratch of sv_sts_workspace_bytes(N, K) bytes,
  *                16-byte aligned, owned by the caller.
  * Returns SV_OK, SV_ERR_ARG, SV_ERR_SHAPE, SV_ERR_WORKSPACE or SV_ERR_CUDA.
- * Enqueues 43 launches and one memset on `stream`; never synchronises.
+ * Enqueues one memset and one cooperative launch (all CTAs resident, a
+ * bounded grid barrier between passes) on `stream`; never synchronises.
  */
 size_t sv_sts_workspace_bytes(int N, int K);
 sv_status sv_sts_fit(const float *logits, const int32_t *accept_len, int N, int K, float tmin,

@@ -14,18 +14,22 @@
 // negative log-likelihood NLL(beta) = sum log(1 + exp(-s beta l)), s = +1
 // survived, -1 not, over beta in [1/tmax, 1/tmin].  NLL is convex in beta.
 //
-// Kernels (every sum in fp64 with a fixed order, so results do not depend on
-// scheduling):
-//   sts_eval_kernel, grid (chunks, K): each CTA sums, over its chunk of
-//   blocks, NLL'(beta) and NLL''(beta) at its position's current beta (the
-//   first launch: the observed count and NLL' at both ends of the
-//   interval).  The last CTA of a position (atomic counter, no waiting)
-//   adds the chunk partials in chunk order and updates the position: end
-//   points and degenerate cases first, then safeguarded Newton steps on
-//   NLL' inside the bracket where it changes sign (bisection whenever a
-//   Newton step leaves the bracket), until the step is below 1e-13.
-//   sts_final_kernel, grid (chunks): T, and the 15-bin calibration error of
-//   sigmoid(l) and sigmoid(l / T_i) over every observed (block, position).
+// Kernel: one persistent grid, launched cooperatively so that every CTA is
+// resident, with a grid barrier between passes (bounded in wall time: on
+// timeout the temperatures come out NaN instead of the kernel hanging).
+// Every sum is in fp64 with a fixed order, so results do not depend on
+// scheduling.
+//   1. Init pass: per (position, chunk of 2048 blocks), the observed count
+//      and NLL' at both ends of the interval; the CTA owning a position adds
+//      the chunk partials in order and settles end points and degenerate
+//      cases.
+//   2. Newton passes: NLL'(beta) and NLL''(beta) of every unconverged
+//      position; its owner takes a safeguarded Newton step inside the bracket
+//      where NLL' changes sign (bisection whenever the step would leave it),
+//      until the step is below 1e-10 of beta (the rounding noise of the sums
+//      sets the floor; the output is fp32).
+//   3. Final pass: T, and the 15-bin calibration error of sigmoid(l) and
+//      sigmoid(l / T_i) over every observed (block, position).
 #include <cmath>
 #include <cstdint>
 
@@ -38,7 +42,6 @@ namespace sv {
 constexpr int kStsThreads = 256;
 constexpr int kStsChunk = 2048;          // blocks per CTA
 constexpr int kStsBins = 15;
-constexpr int kStsNewtonLaunches = 40;   // a position that has converged skips the rest
 
 struct StsState {
     double beta, lo, hi;
@@ -53,7 +56,7 @@ struct StsArgs {
     double lo0, hi0;     // 1/tmax, 1/tmin
     StsState *st;        // [K]
     double *part;        // [K, nchunk, 3]
-    int *arrive;         // [K] (first K ints) + [1] for the final kernel
+    int *bar;            // [0] arrivals, [1] generation
     double *epart;       // [nchunk, 2 * kStsBins + 1]
     float *T;            // [K] out
     float *ece;          // [2] out, nullable
@@ -82,18 +85,46 @@ __device__ __forceinline__ void block_sum3(double &x, double &y, double &z) {
     __syncthreads();
 }
 
-// First launch (`init`): partials (count, NLL'(lo), NLL'(hi)); later launches:
-// (NLL'(beta), NLL''(beta), 0).
-__global__ void __launch_bounds__(kStsThreads) sts_eval_kernel(StsArgs s, int init) {
-    const int i = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x;
-    griddep_wait();
-    griddep_launch_dependents();
-    StsState *ps = s.st + i;
-    if (!init && __ldcg(&ps->done)) return;
-    const double beta = init ? 0.0 : __ldcg(&ps->beta);
+__device__ __forceinline__ int ld_acquire_i32(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Grid barrier (sense by generation).  Every CTA of the cooperative launch
+// is resident, so a wait ends as soon as the last CTA arrives; the wait is
+// still bounded in wall time.  Returns false (in every thread) on timeout.
+__device__ bool grid_barrier(int *bar, int nblocks) {
+    __shared__ int ok;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const int gen = ld_acquire_i32(&bar[1]);
+        __threadfence();
+        int good = 1;
+        if (atomicAdd(&bar[0], 1) + 1 == nblocks) {
+            bar[0] = 0;
+            __threadfence();
+            atomicAdd(&bar[1], 1);
+        } else {
+            const uint64_t t0 = global_ns();
+            while (ld_acquire_i32(&bar[1]) == gen) {
+                if (global_ns() - t0 > 1000000000ull) { good = 0; break; }
+                __nanosleep(64);
+            }
+        }
+        __threadfence();
+        ok = good;
+    }
+    __syncthreads();
+    return ok != 0;
+}
+
+// Partial sums of one (position, chunk) unit at `beta`; init: (count,
+// NLL'(lo), NLL'(hi)), else (NLL'(beta), NLL''(beta), 0).
+__device__ void sts_unit(const StsArgs &s, int i, int chunk, bool init, double beta) {
     double x = 0.0, y = 0.0, z = 0.0;
     const int n0 = chunk * kStsChunk, n1 = min(n0 + kStsChunk, s.N);
-    for (int n = n0 + tid; n < n1; n += kStsThreads) {
+    for (int n = n0 + static_cast<int>(threadIdx.x); n < n1; n += kStsThreads) {
         const int an = __ldg(&s.a[n]);
         if (an < 0 || i > an) continue;
         const double sg = (i < an) ? 1.0 : -1.0;
@@ -109,22 +140,20 @@ __global__ void __launch_bounds__(kStsThreads) sts_eval_kernel(StsArgs s, int in
         }
     }
     block_sum3(x, y, z);
-    __shared__ int last;
-    double *pp = s.part + (static_cast<long long>(i) * s.nchunk + chunk) * 3;
-    if (tid == 0) {
+    if (threadIdx.x == 0) {
+        double *pp = s.part + (static_cast<long long>(i) * s.nchunk + chunk) * 3;
         pp[0] = x; pp[1] = y; pp[2] = z;
-        __threadfence();
-        last = atomicAdd(&s.arrive[i], 1) + 1 == s.nchunk;
-        if (last) __threadfence();
     }
-    __syncthreads();
-    if (!last || tid != 0) return;
-    s.arrive[i] = 0;   // every CTA of this launch has arrived
+}
+
+// The owner of position i adds its chunk partials in order and updates it.
+__device__ void sts_update(const StsArgs &s, int i, bool init) {
     double X = 0.0, Y = 0.0, Z = 0.0;
     for (int c = 0; c < s.nchunk; ++c) {
         const double *q = s.part + (static_cast<long long>(i) * s.nchunk + c) * 3;
         X += __ldcg(q); Y += __ldcg(q + 1); Z += __ldcg(q + 2);
     }
+    StsState *ps = s.st + i;
     if (init) {
         StsState st;
         st.lo = s.lo0; st.hi = s.hi0; st.pad = 0; st.done = 1;
@@ -145,66 +174,101 @@ __global__ void __launch_bounds__(kStsThreads) sts_eval_kernel(StsArgs s, int in
     const double g = X, h = Y;
     if (g == 0.0) { st.done = 1; *ps = st; return; }
     if (g < 0.0) st.lo = st.beta; else st.hi = st.beta;
+    // A converged Newton step ends the search before the bracket test: at
+    // the root the step lands on the bracket end just moved to beta.
+    if (h > 0.0 && fabs(g / h) <= 1e-10 * st.beta) {
+        st.beta = fmin(fmax(st.beta - g / h, st.lo), st.hi);
+        st.done = 1;
+        *ps = st;
+        return;
+    }
     double nb = st.beta - g / h;
-    if (!(h > 0.0) || !(nb > st.lo && nb < st.hi)) nb = 0.5 * (st.lo + st.hi);
-    if (fabs(nb - st.beta) <= 1e-13 * st.beta || st.hi - st.lo <= 1e-13 * st.hi) st.done = 1;
+    if (!(h > 0.0) || !(nb >= st.lo && nb <= st.hi)) nb = 0.5 * (st.lo + st.hi);
+    if (fabs(nb - st.beta) <= 1e-10 * st.beta || st.hi - st.lo <= 1e-10 * st.hi) st.done = 1;
     st.beta = nb;
     *ps = st;
 }
 
-__global__ void __launch_bounds__(kStsThreads) sts_final_kernel(StsArgs s) {
-    const int chunk = blockIdx.x, tid = threadIdx.x;
-    griddep_wait();
-    griddep_launch_dependents();
+constexpr int kStsMaxIter = 64;    // safeguarded Newton; bisection alone needs < 40
+
+__global__ void __launch_bounds__(kStsThreads) sts_fit_kernel(StsArgs s) {
+    const int tid = threadIdx.x;
+    const int G = gridDim.x, g = blockIdx.x;
+    const int units = s.K * s.nchunk;
+    bool ok = true;
+    // 1. init pass
+    for (int u = g; u < units; u += G) sts_unit(s, u / s.nchunk, u % s.nchunk, true, 0.0);
+    ok = grid_barrier(s.bar, G);
+    if (ok && tid == 0)
+        for (int i = g; i < s.K; i += G) sts_update(s, i, true);
+    if (ok) ok = grid_barrier(s.bar, G);
+    // 2. Newton passes
+    __shared__ int s_open;
+    for (int it = 0; ok && it < kStsMaxIter; ++it) {
+        if (tid == 0) {
+            int open = 0;
+            for (int i = 0; i < s.K; ++i) open |= !__ldcg(&s.st[i].done);
+            s_open = open;
+        }
+        __syncthreads();
+        if (!s_open) break;   // every CTA reads the same states after the barrier
+        for (int u = g; u < units; u += G) {
+            const int i = u / s.nchunk;
+            if (__ldcg(&s.st[i].done)) continue;
+            sts_unit(s, i, u % s.nchunk, false, __ldcg(&s.st[i].beta));
+        }
+        ok = grid_barrier(s.bar, G);
+        if (ok && tid == 0)
+            for (int i = g; i < s.K; i += G)
+                if (!__ldcg(&s.st[i].done)) sts_update(s, i, false);
+        if (ok) ok = grid_barrier(s.bar, G);
+    }
+    // 3. outputs
     __shared__ double invT[SV_MAX_K];
     for (int i = tid; i < s.K; i += kStsThreads) {
-        invT[i] = __ldcg(&s.st[i].beta);
-        if (chunk == 0) s.T[i] = static_cast<float>(1.0 / invT[i]);
+        invT[i] = ok ? __ldcg(&s.st[i].beta) : __longlong_as_double(0x7ff8000000000000ll);
+        if (g == 0) s.T[i] = static_cast<float>(1.0 / invT[i]);
     }
     __syncthreads();
-    if (!s.ece) return;
-    // Per thread: sum of (y - conf) per bin before and after, and the count.
+    if (!s.ece || !ok) return;
     double d0[kStsBins], d1[kStsBins];
+    for (int chunk = g; chunk < s.nchunk; chunk += G) {
 #pragma unroll
-    for (int m = 0; m < kStsBins; ++m) d0[m] = d1[m] = 0.0;
-    double cnt = 0.0;
-    const int n0 = chunk * kStsChunk, n1 = min(n0 + kStsChunk, s.N);
-    for (int n = n0 + tid; n < n1; n += kStsThreads) {
-        const int an = __ldg(&s.a[n]);
-        if (an < 0) continue;
-        for (int i = 0; i < s.K && i <= an; ++i) {
-            const double v = static_cast<double>(__ldg(&s.l[static_cast<long long>(n) * s.K + i]));
-            const double y = (i < an) ? 1.0 : 0.0;
-            const double c0 = sts_sigmoid(v), c1 = sts_sigmoid(v * invT[i]);
-            const int m0 = min(static_cast<int>(c0 * kStsBins), kStsBins - 1);
-            const int m1 = min(static_cast<int>(c1 * kStsBins), kStsBins - 1);
+        for (int m = 0; m < kStsBins; ++m) d0[m] = d1[m] = 0.0;
+        double cnt = 0.0;
+        const int n0 = chunk * kStsChunk, n1 = min(n0 + kStsChunk, s.N);
+        for (int n = n0 + tid; n < n1; n += kStsThreads) {
+            const int an = __ldg(&s.a[n]);
+            if (an < 0) continue;
+            for (int i = 0; i < s.K && i <= an; ++i) {
+                const double v =
+                    static_cast<double>(__ldg(&s.l[static_cast<long long>(n) * s.K + i]));
+                const double y = (i < an) ? 1.0 : 0.0;
+                const double c0 = sts_sigmoid(v), c1 = sts_sigmoid(v * invT[i]);
+                const int m0 = min(static_cast<int>(c0 * kStsBins), kStsBins - 1);
+                const int m1 = min(static_cast<int>(c1 * kStsBins), kStsBins - 1);
 #pragma unroll
-            for (int m = 0; m < kStsBins; ++m) {
-                d0[m] += (m == m0) ? y - c0 : 0.0;
-                d1[m] += (m == m1) ? y - c1 : 0.0;
+                for (int m = 0; m < kStsBins; ++m) {
+                    d0[m] += (m == m0) ? y - c0 : 0.0;
+                    d1[m] += (m == m1) ? y - c1 : 0.0;
+                }
+                cnt += 1.0;
             }
-            cnt += 1.0;
+        }
+        double *pp = s.epart + static_cast<long long>(chunk) * (2 * kStsBins + 1);
+#pragma unroll
+        for (int m = 0; m < kStsBins; ++m) {
+            double x = d0[m], y = d1[m], z = (m == 0) ? cnt : 0.0;
+            block_sum3(x, y, z);
+            if (tid == 0) {
+                pp[m] = x;
+                pp[kStsBins + m] = y;
+                if (m == 0) pp[2 * kStsBins] = z;
+            }
         }
     }
-    double *pp = s.epart + static_cast<long long>(chunk) * (2 * kStsBins + 1);
-    for (int m = 0; m < kStsBins; m += 1) {
-        double x = d0[m], y = d1[m], z = (m == 0) ? cnt : 0.0;
-        block_sum3(x, y, z);
-        if (tid == 0) {
-            pp[m] = x;
-            pp[kStsBins + m] = y;
-            if (m == 0) pp[2 * kStsBins] = z;
-        }
-    }
-    __shared__ int last;
-    if (tid == 0) {
-        __threadfence();
-        last = atomicAdd(&s.arrive[s.K], 1) + 1 == s.nchunk;
-        if (last) __threadfence();
-    }
-    __syncthreads();
-    if (!last || tid != 0) return;
-    s.arrive[s.K] = 0;
+    if (!grid_barrier(s.bar, G)) return;
+    if (g != 0 || tid != 0) return;
     double e0 = 0.0, e1 = 0.0, c = 0.0;
     for (int m = 0; m < kStsBins; ++m) {
         double x = 0.0, y = 0.0;
@@ -235,7 +299,7 @@ __global__ void sts_apply_kernel(const float *__restrict__ l, const float *__res
 
 struct StsPlan {
     int nchunk;
-    size_t off_st, off_part, off_arrive, off_epart, bytes;
+    size_t off_st, off_part, off_bar, off_epart, bytes;
 };
 
 static bool sts_plan(int N, int K, StsPlan *p) {
@@ -245,7 +309,7 @@ static bool sts_plan(int N, int K, StsPlan *p) {
     size_t off = 0;
     p->off_st = off;     off = align16(off + sizeof(StsState) * K);
     p->off_part = off;   off = align16(off + sizeof(double) * 3 * static_cast<size_t>(K) * p->nchunk);
-    p->off_arrive = off; off = align16(off + sizeof(int) * (K + 1));
+    p->off_bar = off;    off = align16(off + sizeof(int) * 2);
     p->off_epart = off;  off = align16(off + sizeof(double) * (2 * kStsBins + 1) * p->nchunk);
     p->bytes = off;
     return true;
@@ -275,19 +339,35 @@ extern "C" sv_status sv_sts_fit(const float *logits, const int32_t *accept_len, 
     s.hi0 = 1.0 / static_cast<double>(tmin);
     s.st = reinterpret_cast<sv::StsState *>(w + p.off_st);
     s.part = reinterpret_cast<double *>(w + p.off_part);
-    s.arrive = reinterpret_cast<int *>(w + p.off_arrive);
+    s.bar = reinterpret_cast<int *>(w + p.off_bar);
     s.epart = reinterpret_cast<double *>(w + p.off_epart);
     s.T = temperature; s.ece = ece;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // The arrival counters start at zero; each launch's last CTA resets its own.
-    cudaError_t e = cudaMemsetAsync(s.arrive, 0, sizeof(int) * (K + 1), st);
-    if (e != cudaSuccess) return sv::note_cuda(e);
-    const dim3 grid(p.nchunk, K);
-    e = sv::launch_pdl(sv::sts_eval_kernel, grid, dim3(sv::kStsThreads), 0, st, s, 1);
-    for (int it = 0; it < sv::kStsNewtonLaunches && e == cudaSuccess; ++it)
-        e = sv::launch_pdl(sv::sts_eval_kernel, grid, dim3(sv::kStsThreads), 0, st, s, 0);
+    int dev = 0, sms = 0, per = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess)
-        e = sv::launch_pdl(sv::sts_final_kernel, dim3(p.nchunk), dim3(sv::kStsThreads), 0, st, s);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, sv::sts_fit_kernel,
+                                                          sv::kStsThreads, 0);
+    if (e != cudaSuccess) return sv::note_cuda(e);
+    const long long units = static_cast<long long>(K) * p.nchunk;
+    const long long cap = static_cast<long long>(sms) * (per > 0 ? per : 1);
+    const int grid = static_cast<int>(units < cap ? units : cap);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // The barrier words start at zero; the kernel leaves them at zero again.
+    e = cudaMemsetAsync(s.bar, 0, sizeof(int) * 2, st);
+    if (e != cudaSuccess) return sv::note_cuda(e);
+    // Cooperative launch: every CTA resident, which the grid barrier needs.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(sv::kStsThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, sv::sts_fit_kernel, s);
     if (e != cudaSuccess) return sv::note_cuda(e);
     return sv::note_cuda(cudaGetLastError());
 }
