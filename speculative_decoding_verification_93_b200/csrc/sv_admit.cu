@@ -18,12 +18,17 @@
 // so each row's admitted candidates form a prefix.  S is the fp64 running
 // product of the clamped confidences (NaN counts as 0).
 //
-// Kernel: per-row products in fp64 in the same order as the definition,
-// bitonic sort in shared memory, an fp64 block prefix scan for E(k), and a
-// block-wide minimum for the first k at which f stops rising.
+// Kernel (one CTA): per-row products in fp64 in the same order as the
+// definition; a stable block radix sort of (S, candidate index) pairs,
+// descending in S (candidates enter in index order, so ties stay in index
+// order); an fp64 block scan of the sorted S for E(k); and a block-wide
+// minimum for the first k at which f stops rising.
 #include <cfloat>
 #include <climits>
 #include <cstdint>
+
+#include <cub/block/block_radix_sort.cuh>
+#include <cub/block/block_scan.cuh>
 
 #include "sv.h"
 #include "sv_device.cuh"
@@ -31,128 +36,142 @@
 
 namespace sv {
 
-constexpr int kAdmitThreads = 1024;
-constexpr int kAdmitMax = SV_MAX_ADMIT;   // candidates (B * K) sorted in shared memory
+constexpr int kAdmitMax = SV_MAX_ADMIT;     // B * K candidates in one CTA
 
-// a precedes b in admission order
-__device__ __forceinline__ bool admit_before(double ka, int ia, double kb, int ib) {
-    return ka > kb || (ka == kb && ia < ib);
-}
+template <int THREADS, int kAdmitItems>
+struct AdmitSort {
+    using Sort = cub::BlockRadixSort<double, THREADS, kAdmitItems, int, 5>;
+    using Scan = cub::BlockScan<double, THREADS>;
+    union Storage {
+        typename Sort::TempStorage sort;
+        typename Scan::TempStorage scan;
+    };
+};
 
-__global__ void __launch_bounds__(kAdmitThreads) admit_kernel(const float *__restrict__ conf,
-                                                              int B, int K,
-                                                              const float *__restrict__ speed,
-                                                              int n_speed, int32_t *lengths,
-                                                              float *tau_out) {
+template <int THREADS, int kAdmitItems>
+__global__ void __launch_bounds__(THREADS) admit_kernel(const float *__restrict__ conf, int B,
+                                                        int K, const float *__restrict__ speed,
+                                                        int n_speed, int32_t *lengths,
+                                                        float *tau_out) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    auto &tmp = *reinterpret_cast<typename AdmitSort<THREADS, kAdmitItems>::Storage *>(smem_raw);
+    __shared__ int s_stop;
+    __shared__ double s_last;
+    const int tid = threadIdx.x;
     griddep_wait();
     griddep_launch_dependents();
     const int n = B * K;
-    int N = 1;
-    while (N < n) N <<= 1;
-    double *key = reinterpret_cast<double *>(smem_raw);        // [N]
-    int *idx = reinterpret_cast<int *>(key + N);                // [N]
-    __shared__ double s_wsum[kAdmitThreads / 32];
-    __shared__ int s_stop;
 
-    // 1. Prefix survival of every candidate.
-    for (int b = tid; b < B; b += kAdmitThreads) {
-        double S = 1.0;
-        for (int i = 0; i < K; ++i) {
-            double c = static_cast<double>(__ldg(conf + static_cast<long long>(b) * K + i));
-            c = isnan(c) ? 0.0 : fmin(fmax(c, 0.0), 1.0);
-            S = S * c;
-            key[b * K + i] = S;
-            idx[b * K + i] = b * K + i;
-        }
+    // 1. Prefix survival of every candidate; thread t holds candidates
+    //    t * 8 .. t * 8 + 7 (index order).  Padding sorts last (key -1).
+    double key[kAdmitItems];
+    int idx[kAdmitItems];
+#pragma unroll
+    for (int q = 0; q < kAdmitItems; ++q) {
+        key[q] = -1.0;
+        idx[q] = INT_MAX;
     }
-    for (int q = n + tid; q < N; q += kAdmitThreads) { key[q] = -1.0; idx[q] = INT_MAX; }
-    __syncthreads();
-
-    // 2. Bitonic sort into admission order.
-    for (int k = 2; k <= N; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int i = tid; i < N; i += kAdmitThreads) {
-                const int p = i ^ j;
-                if (p > i) {
-                    const double ki = key[i], kp = key[p];
-                    const int ii = idx[i], ip = idx[p];
-                    const bool asc = (i & k) == 0;   // segment in admission order
-                    const bool swap = asc ? admit_before(kp, ip, ki, ii) : admit_before(ki, ii, kp, ip);
-                    if (swap) {
-                        key[i] = kp; key[p] = ki;
-                        idx[i] = ip; idx[p] = ii;
-                    }
+    {
+        // survival products need the row's earlier positions: a thread walks
+        // each row that its candidates touch from the row start.
+        const int c0 = tid * kAdmitItems;
+        if (c0 < n) {
+            int b = c0 / K, i = c0 - b * K;
+            double S = 1.0;
+            for (int j = 0; j < i; ++j) {
+                double c = static_cast<double>(__ldg(conf + static_cast<long long>(b) * K + j));
+                c = isnan(c) ? 0.0 : fmin(fmax(c, 0.0), 1.0);
+                S = S * c;
+            }
+#pragma unroll
+            for (int q = 0; q < kAdmitItems; ++q) {
+                const int cq = c0 + q;
+                if (cq < n) {
+                    if (i == K) { ++b; i = 0; S = 1.0; }
+                    double c = static_cast<double>(__ldg(conf + cq));
+                    c = isnan(c) ? 0.0 : fmin(fmax(c, 0.0), 1.0);
+                    S = S * c;
+                    key[q] = S;
+                    idx[q] = cq;
+                    ++i;
                 }
             }
-            __syncthreads();
         }
     }
-
-    // 3. Exclusive prefix sums of the sorted survivals (per-thread runs of
-    //    consecutive candidates, then a block scan of the run totals).
-    const int per = N / kAdmitThreads > 0 ? N / kAdmitThreads : 1;
-    const int r0 = tid * per;
-    double run = 0.0;
-    for (int q = 0; q < per; ++q)
-        if (r0 + q < n) run += key[r0 + q];
-    double x = run;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const double y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) s_wsum[warp] = x;
     if (tid == 0) s_stop = INT_MAX;
-    __syncthreads();
-    if (warp == 0) {
-        double y = s_wsum[lane];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const double z = __shfl_up_sync(0xffffffffu, y, o);
-            if (lane >= o) y += z;
-        }
-        s_wsum[lane] = y;
-    }
-    __syncthreads();
-    const double xprev = __shfl_up_sync(0xffffffffu, x, 1);
-    double pre = (lane ? xprev : 0.0) + (warp ? s_wsum[warp - 1] : 0.0);   // sum before this run
 
-    // 4. First k whose admission does not raise f (or runs out of table).
-    //    Each thread tests the candidates of its run: k = r0 + q.
+    // 2. Admission order: S descending, ties by index (stable sort).
+    typename AdmitSort<THREADS, kAdmitItems>::Sort(tmp.sort).SortDescending(key, idx);
+    __syncthreads();
+
+    // 3. Exclusive prefix of the sorted survivals: thread totals, then a
+    //    block scan.
+    double run = 0.0;
+#pragma unroll
+    for (int q = 0; q < kAdmitItems; ++q)
+        if (key[q] >= 0.0) run += key[q];
+    double pre;
+    typename AdmitSort<THREADS, kAdmitItems>::Scan(tmp.scan).ExclusiveSum(run, pre);
+
+    // 4. First k whose admission does not raise f (or leaves the table).
+    const int r0 = tid * kAdmitItems;
     int stop = INT_MAX;
-    for (int q = 0; q < per; ++q) {
+#pragma unroll
+    for (int q = 0; q < kAdmitItems; ++q) {
         const int k = r0 + q;
-        if (k > n || r0 + q >= N + 1) break;
-        const double Ek = static_cast<double>(B) + pre;
-        bool fail;
-        if (k >= n || B + k + 1 >= n_speed) {
-            fail = true;
-        } else {
-            const double fk = Ek * static_cast<double>(__ldg(speed + B + k));
-            const double f1 = (Ek + key[k]) * static_cast<double>(__ldg(speed + B + k + 1));
-            fail = !(f1 > fk);
+        if (stop == INT_MAX && k <= n) {
+            bool fail;
+            if (k >= n || B + k + 1 >= n_speed) {
+                fail = true;
+            } else {
+                const double Ek = static_cast<double>(B) + pre;
+                const double fk = Ek * static_cast<double>(__ldg(speed + B + k));
+                const double f1 = (Ek + key[q]) * static_cast<double>(__ldg(speed + B + k + 1));
+                fail = !(f1 > fk);
+            }
+            if (fail) stop = k;
+            else pre += key[q];
         }
-        if (fail) { stop = k; break; }
-        pre += key[k];
     }
     if (stop != INT_MAX) atomicMin(&s_stop, stop);
     __syncthreads();
     int admitted = s_stop;
-    if (admitted == INT_MAX) admitted = n;   // every candidate admitted (N == n case)
+    if (admitted == INT_MAX) admitted = n;   // every candidate admitted
     if (B >= n_speed) admitted = 0;
 
     // 5. Per-row counts and the threshold.
-    for (int b = tid; b < B; b += kAdmitThreads) lengths[b] = 0;
+    for (int b = tid; b < B; b += THREADS) lengths[b] = 0;
     __syncthreads();
-    for (int q = tid; q < admitted; q += kAdmitThreads) atomicAdd(&lengths[idx[q] / K], 1);
+#pragma unroll
+    for (int q = 0; q < kAdmitItems; ++q) {
+        const int k = r0 + q;
+        if (k < admitted) atomicAdd(&lengths[idx[q] / K], 1);
+        if (k == admitted - 1) s_last = key[q];
+    }
+    __syncthreads();
     if (tid == 0 && tau_out)
-        *tau_out = admitted > 0 ? static_cast<float>(key[admitted - 1])
-                                : __int_as_float(0x7f800000);
+        *tau_out = admitted > 0 ? static_cast<float>(s_last) : __int_as_float(0x7f800000);
 }
 
 }  // namespace sv
+
+template <int THREADS, int ITEMS>
+static sv_status launch_admit(const float *conf, int B, int K, const float *speed, int n_speed,
+                              int32_t *lengths, float *tau_out, cudaStream_t st) {
+    constexpr size_t smem = sizeof(typename sv::AdmitSort<THREADS, ITEMS>::Storage);
+    static bool attr_set[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return sv::note_cuda(e);
+    if (!attr_set[dev & 63]) {
+        e = cudaFuncSetAttribute(sv::admit_kernel<THREADS, ITEMS>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return sv::note_cuda(e);
+        attr_set[dev & 63] = true;
+    }
+    return sv::note_cuda(sv::launch_pdl(sv::admit_kernel<THREADS, ITEMS>, dim3(1), dim3(THREADS), smem, st,
+                                        conf, B, K, speed, n_speed, lengths, tau_out));
+}
 
 extern "C" sv_status sv_schedule_admit(const float *conf, int B, int K, const float *speed,
                                        int n_speed, int32_t *lengths, float *tau_out,
@@ -161,20 +180,8 @@ extern "C" sv_status sv_schedule_admit(const float *conf, int B, int K, const fl
     if (B < 1 || K < 1 || K > SV_MAX_K || static_cast<long long>(B) * K > sv::kAdmitMax ||
         n_speed < 1)
         return SV_ERR_SHAPE;
-    int N = 1;
-    while (N < B * K) N <<= 1;
-    const size_t smem = static_cast<size_t>(N) * (sizeof(double) + sizeof(int));
-    static bool attr_set[64];
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return sv::note_cuda(e);
-    if (!attr_set[dev & 63]) {
-        e = cudaFuncSetAttribute(sv::admit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(sv::kAdmitMax * (sizeof(double) + sizeof(int))));
-        if (e != cudaSuccess) return sv::note_cuda(e);
-        attr_set[dev & 63] = true;
-    }
-    return sv::note_cuda(sv::launch_pdl(sv::admit_kernel, dim3(1), dim3(sv::kAdmitThreads), smem,
-                                        static_cast<cudaStream_t>(stream), conf, B, K, speed,
-                                        n_speed, lengths, tau_out));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (B * K <= 256 * 8)
+        return launch_admit<256, 8>(conf, B, K, speed, n_speed, lengths, tau_out, st);
+    return launch_admit<512, 16>(conf, B, K, speed, n_speed, lengths, tau_out, st);
 }
