@@ -180,8 +180,11 @@ sv_status sv_sts_apply(const float *logits, const float *temperature, int N, int
 
 /*
  * sv_verify_workspace_bytes -- device scratch that sv_verify needs for
- * (B, K, V, dtype): per-row work counters, per-row work offsets and the
- * per-chunk softmax partials.  Returns 0 for unsupported sizes.
+ * (B, K, V, dtype): work counters, per-row state (length, first rejection
+ * found so far, per-position completion counts), the position-major work
+ * list, the per-chunk softmax partials, the residual draw table and the
+ * resample work list.  Linear in B * K * V / 64K.  Returns 0 for
+ * unsupported sizes.
  */
 size_t sv_verify_workspace_bytes(int B, int K, int V, sv_dtype dtype);
 

@@ -18,27 +18,33 @@
 //
 // Design.  Everything a row needs is a set of logit vectors (target
 // positions 0..L, draft positions 0..L-1 for sampled rows).  Every vector is
-// cut into C equal chunks of 16-byte units, and one *item* is one chunk.
-//   1. prologue_kernel (1 CTA): validates rows, counts items per row, writes
-//      the exclusive prefix of item counts (the work list is implicit in it)
-//      and resets the per-row counters.
-//   2. stream_kernel (persistent, 2 CTAs/SM, warp-specialised): one HBM pass
-//      over every scheduled vector.  A producer warp takes items from a
-//      global atomic counter, decodes them and streams their bytes into a
-//      6-stage shared-memory ring with bulk copies (cp.async.bulk, mbarrier
-//      completion), running ahead of the math across item boundaries.  Eight
-//      consumer warps reduce each stage -- packed bf16x2 max, one exp2 per
-//      element against the running max -- and publish one (max, sum) partial
-//      per item (greedy rows: max and first argmax).  Every mbarrier wait is
-//      bounded in wall time and reports SV_NOTE_TIMEOUT instead of hanging.
-//   3. draw_kernel (one CTA per row and chunk): merges the partials into the
-//      normalisers, runs the accept test with Philox uniforms, and draws the
-//      final token by inverse CDF in two steps: over chunks, then inside the
-//      chosen chunk.  Chunk masses of p_j (bonus, greedy drafter) come from
-//      the stream partials without touching the logits again; the residual
-//      max(0, p_j - q_j) is summed chunk by chunk by the row's CTAs in
-//      parallel, and the last of them (atomic counter, no waiting) locates
-//      the token.  Only position j of a rejecting row is read a second time.
+// cut into C chunks of 16-byte units, and one *item* is one chunk.
+//   1. prologue_kernel (1 CTA): validates rows, resets the per-row state
+//      and writes the position-major work list, implicit in per-level row
+//      prefixes: every row's position 0 comes before any row's position 1.
+//   2. stream_kernel (persistent, 3 CTAs/SM, warp-specialised): a producer
+//      thread claims items from a global counter, skips an item whose row
+//      has already rejected an earlier position, and streams the others
+//      into a 4-stage shared-memory ring with bulk copies (cp.async.bulk,
+//      mbarrier completion), abandoning an item between stages once it is
+//      known to be unneeded.  Eight consumer warps reduce each stage --
+//      packed bf16x2 max, one exp2 per element against the running max --
+//      into (max, sum) partials (greedy rows: max and first argmax).  A
+//      publisher warp merges each item's warp partials, publishes one
+//      partial per item, counts finished items per (row, position), and
+//      runs the accept test of a position as soon as it is complete,
+//      lowering the row's first-rejection marker on a rejection.  Every
+//      mbarrier wait is bounded in wall time and reports SV_NOTE_TIMEOUT.
+//   3. accept_kernel (one CTA per row): settles j = first rejection (or L),
+//      merges the normalisers of positions 0..j, writes greedy rows, sets up
+//      each sampled row's final draw (for p-mass draws the chunk is chosen
+//      from the stream partials) and appends the resample work list.
+//   4. resample_kernel (one CTA per work entry): residual draws sum
+//      max(0, p_j - q_j) over their chunk by 64-unit sub-ranges; the last
+//      chunk CTA of the row (atomic counter, no waiting) picks the sub-range
+//      from the row's table and the token inside it.  p-mass draws locate
+//      the token inside the chosen chunk.  Only position j of a rejecting
+//      row is read a second time.
 #include <climits>
 #include <cstdint>
 #include <cstdio>
@@ -59,7 +65,6 @@ constexpr int kRingBytes = kStages * kStageUnits * 16;
 constexpr int kMaxUnitsPerItem = 4 * kStageUnits; // an item spans up to 4 stages
 constexpr int kMaxSlots = 2 * SV_MAX_K + 1;
 constexpr int kMaxChunks = 64;                    // V <= SV_MAX_V keeps C within this
-constexpr int kPartsPerItem = 1;                  // one merged softmax partial per item
 constexpr int kPrologueThreads = 1024;
 
 struct VerifyArgs {
@@ -1086,40 +1091,23 @@ __device__ __forceinline__ int select_chunk(const float *cm, int C, float u, flo
 // Same masses, computed by a single thread (rare fallback paths).
 __device__ __forceinline__ void chunk_masses_serial(const VerifyArgs &a, int b, int j, float mj,
                                                     float k, float *cm) {
-    const long long base = (static_cast<long long>(b) * a.S + j) * a.C * kPartsPerItem;
+    const long long base = (static_cast<long long>(b) * a.S + j) * a.C;
     for (int cc = 0; cc < a.C; ++cc) {
-        float t = 0.f;
-        for (int w = 0; w < kPartsPerItem; ++w) {
-            const float4 p = __ldcg(&a.part[base + cc * kPartsPerItem + w]);
-            if (p.x != kNegInf) t += p.y * ex2((p.x - mj) * k);
-        }
-        cm[cc] = t;
+        const float4 p = __ldcg(&a.part[base + cc]);
+        cm[cc] = (p.x != kNegInf) ? p.y * ex2((p.x - mj) * k) : 0.f;
     }
 }
 
 // Mass of p_j per chunk, in units of 2^((z - m_j) k), from the stream
-// partials (sum over the chunk's warp partials).  Thread-parallel over the
-// C * kPartsPerItem partials; the result lands in cm[0..C).
+// partials (one per chunk).  Thread-parallel; the result lands in cm[0..C).
 __device__ __forceinline__ void chunk_masses(const VerifyArgs &a, int b, int j, float mj, float k,
                                              float *cm) {
-    const int tid = threadIdx.x;
-    const long long base = (static_cast<long long>(b) * a.S + j) * a.C * kPartsPerItem;
-    const int n = a.C * kPartsPerItem;
-    const int lane = tid & 31;
-    for (int q0 = tid - lane; q0 < n; q0 += blockDim.x) {   // warp-uniform trip count
-        const int q = q0 + lane;
-        float t = 0.f;
-        if (q < n) {
-            const float4 p = __ldcg(&a.part[base + q]);
-            if (p.x != kNegInf) t = p.y * ex2((p.x - mj) * k);
-        }
-        // kPartsPerItem (8) consecutive lanes hold one chunk
-#pragma unroll
-        for (int o = 1; o < kPartsPerItem; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-        if (q < n && (q & (kPartsPerItem - 1)) == 0) cm[q / kPartsPerItem] = t;
+    const long long base = (static_cast<long long>(b) * a.S + j) * a.C;
+    for (int q = threadIdx.x; q < a.C; q += blockDim.x) {
+        const float4 p = __ldcg(&a.part[base + q]);
+        cm[q] = (p.x != kNegInf) ? p.y * ex2((p.x - mj) * k) : 0.f;
     }
 }
-
 
 // ---------------------------------------------------------------------------
 // Residual draw by sub-ranges of kSubUnits units.
