@@ -62,11 +62,11 @@ typedef enum { SV_F32 = 0, SV_BF16 = 1 } sv_dtype;
  *
  * Defined by: umans.ai, "DeepSeek V4 Pro DSpark: the model isn't ready, the
  * architecture is", section "What DSpark adds", item "2. Verify smarter"
- * (a confidence head gives, per draft position, the probability that the
- * token survives given that every earlier one survived; multiplying along the
- * block gives the survival probability of every prefix length); aiweekly.co
- * alert (verify length from estimated prefix survival and system load);
- * en.5iter.com article, section "What DSpark changed is how to generate a
+ * (for each draft position a confidence head estimates the chance that the
+ * token is kept once every token before it was kept; the running product
+ * along the block is then the chance that each prefix is kept); aiweekly.co
+ * alert (the verify length follows the estimated survival of each prefix
+ * and the current load); en.5iter.com article, section "What DSpark changed is how to generate a
  * draft", and techvisionai "DeepSeek-V4: Breaking the Efficiency Barrier",
  * Ch. 7 "Confidence-Scheduled Verification" (verify longer when idle, only
  * the confident prefix when busy).
@@ -95,10 +95,11 @@ sv_status sv_schedule(const float *conf, int B, int K, float load,
  *
  * Defined by: umans.ai, "DeepSeek V4 Pro DSpark: the model isn't ready, the
  * architecture is", section "What DSpark adds", item "2. Verify smarter"
- * (profile the engine's steps per second as a function of batch size; every
- * step, sort every candidate token of every request by survival
- * probability, admit them one at a time, and stop the moment expected
- * accepted tokens times the speed at that batch size stops rising);
+ * (the engine's verification rate is measured once for each batch size;
+ * at each step the candidates of all requests are ranked by their survival
+ * chance and taken in that order for as long as the expected number of
+ * accepted tokens, multiplied by the measured rate at the resulting batch
+ * size, keeps growing);
  * techvisionai "DeepSeek-V4: Breaking the Efficiency Barrier", Ch. 7
  * "Hardware-Aware Scheduling"; zhichai.net DSpark topic, "Under the hood".
  *
@@ -135,8 +136,8 @@ sv_status sv_schedule_admit(const float *conf, int B, int K, const float *speed,
  * Defined by: umans.ai, "DeepSeek V4 Pro DSpark: the model isn't ready, the
  * architecture is", section "What DSpark adds", item "2. Verify smarter"
  * (the head's raw confidence is overconfident by 3-8% expected calibration
- * error; a per-position temperature fitted on held-out data brings it to
- * about 1%); zhichai.net DSpark topic, "Under the hood" (Sequential
+ * error; a temperature for each position, chosen on blocks kept aside,
+ * lowers that to about 1%); zhichai.net DSpark topic, "Under the hood" (Sequential
  * Temperature Scaling).
  *
  * The head predicts survival of position i given that every earlier

@@ -26,9 +26,9 @@
  * The pages state the rule in words only: the target accepts the prefix it
  * agrees with plus one token of its own [P1 "Speculative decoding, briefly"],
  * by rejection sampling on the target/draft probability ratio [P3 "Why LLMs
- * speak so slowly"], so that accepted tokens follow the target distribution
- * exactly [P1]; a rejected token is replaced by one the target would produce
- * [P1].  Written out in symbols (the standard speculative-sampling rule):
+ * speak so slowly"], which leaves the accepted tokens distributed exactly as
+ * the target's own [P1]; a rejected token gives way to one of the target's
+ * choosing [P1].  Written out in symbols (the standard speculative-sampling rule):
  *   accept x_i with probability min(1, p_i(x_i) / q_i(x_i)); at the first
  *   rejection j emit a draw from norm(max(0, p_j - q_j)); if all L drafts
  *   survive emit a bonus draw from p_L.
@@ -457,11 +457,10 @@ int oracle_ndiag(void) { return OR_NDIAG; }
 /* ---------------------------------------------------------------------------
  * Hardware-aware admission [P1 "What DSpark adds", item "2. Verify
  * smarter"; P3 "Under the hood"; P4 Ch.7 "Hardware-Aware Scheduling"]: the
- * engine's speed (verification steps per second) is profiled once as a
- * function of the verify batch size; every step the candidate draft tokens of
- * all rows are sorted by prefix survival, admitted one at a time, and
- * admission stops the moment expected system throughput -- expected accepted
- * tokens times the speed at that batch size -- stops rising.
+ * verification rate (steps per second) is measured once per verify batch
+ * size; at each step the candidate draft tokens of all rows are ranked by
+ * prefix survival and taken one by one while the expected accepted tokens,
+ * multiplied by the measured rate at the resulting batch size, still grows.
  *
  * Reading: row b always verifies its final position, so the batch holds
  * n = B + k tokens after k admissions; expected emitted tokens are
@@ -527,8 +526,8 @@ int oracle_schedule_admit(const float *conf, int B, int K, const float *speed, i
  * umans.ai, "DeepSeek V4 Pro DSpark: the model isn't ready, the
  * architecture is", section "What DSpark adds", item "2. Verify smarter":
  * the head's raw confidences are overconfident (3-8% expected calibration
- * error) and a per-position temperature fitted on held-out data brings
- * them to about 1%.  zhichai.net DSpark topic, "Under the hood": the head
+ * error), and dividing each position's logit by its own temperature,
+ * chosen on blocks kept aside from training, lowers that to about 1%.  zhichai.net DSpark topic, "Under the hood": the head
  * is calibrated by Sequential Temperature Scaling.
  *
  * Held-out data: N draft blocks, the head's logits l[n, i] (confidence =

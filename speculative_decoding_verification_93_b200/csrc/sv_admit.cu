@@ -2,11 +2,11 @@
 //
 // Method (cited as page title + section): umans.ai, "DeepSeek V4 Pro DSpark:
 // the model isn't ready, the architecture is", section "What DSpark adds",
-// item "2. Verify smarter" -- the engine's speed is profiled once as a
-// function of batch size; every step, expected system throughput is expected
-// accepted tokens times the speed at that batch size; every candidate token
-// of every active request is sorted by survival probability, admitted one at
-// a time, and admission stops the moment the product stops rising.
+// item "2. Verify smarter" -- the engine's verification rate is measured
+// once per batch size; at each step the candidates of all live requests are
+// ranked by survival chance and taken one by one while the expected number
+// of accepted tokens times the measured rate at the resulting batch size
+// still grows.
 // zhichai.net DSpark topic, "Under the hood" and techvisionai Ch. 7
 // "Hardware-Aware Scheduling" describe the same scheduler.
 //

@@ -3,8 +3,8 @@
 // Method (cited as page title + section): umans.ai, "DeepSeek V4 Pro DSpark:
 // the model isn't ready, the architecture is", section "What DSpark adds",
 // item "2. Verify smarter" -- the head's raw confidences are overconfident
-// (3-8% expected calibration error) and a per-position temperature fitted on
-// held-out data brings them to about 1%; zhichai.net DSpark topic, "Under
+// (3-8% expected calibration error), and a temperature for each position,
+// chosen on blocks kept aside, lowers that to about 1%; zhichai.net DSpark topic, "Under
 // the hood": the head is calibrated by Sequential Temperature Scaling.
 //
 // Reading: the head predicts survival of position i given that every

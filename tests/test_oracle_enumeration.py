@@ -1,8 +1,8 @@
 """Losslessness pin for the oracle by exact interval enumeration.
 
 What the pages fix: verification is rejection sampling on the target/draft
-probability ratio and "accepted tokens follow the target model's distribution
-exactly" (umans.ai "DeepSeek V4 Pro DSpark: the model isn't ready, the
+probability ratio, and the tokens it emits are distributed exactly as the
+target's own (umans.ai "DeepSeek V4 Pro DSpark: the model isn't ready, the
 architecture is", section "Speculative decoding, briefly"; zhichai.net DSpark
 topic, section "Why LLMs speak so slowly").  So, for every position i <= L,
 given that positions 0..i-1 were emitted as accepted drafts, the token

@@ -1,6 +1,6 @@
 """Pins for the oracle's per-position temperature scaling of the confidence
-head (umans.ai page, "What DSpark adds", item "2. Verify smarter": a
-per-position temperature fitted on held-out data; zhichai.net topic, "Under
+head (umans.ai page, "What DSpark adds", item "2. Verify smarter": one
+temperature for each draft position, chosen on blocks kept aside; zhichai.net topic, "Under
 the hood": Sequential Temperature Scaling).
 
 Each pin comes from outside the oracle's code: a closed form for a constant
