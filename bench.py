@@ -197,6 +197,78 @@ def workload_config(batch, lengths_np, esize):
             "data_seed": s.data_seed}
 
 
+def vocab_parallel_probe(batch, lengths, V, esize, sched_bytes, seed, steps, peak):
+    """Vocabulary-parallel verification of the same batch, split over n = 1
+    and n = 8 ranks: the time one rank spends in its three kernels
+    (sv_vp_stats, sv_vp_decide, sv_vp_draw) for its slice, and the stats
+    kernel's roofline.  One GPU stands in for the ranks: every slice's
+    statistics are computed once to fill the gathered buffers, then rank 0's
+    kernels are timed alone (collectives excluded: they need n GPUs).  L2 is
+    flushed before every timed launch (an eighth of the logits fits in L2)."""
+    from speculative_decoding_verification_93_b200.vocab_parallel import shard_vocab
+    dev = batch.zt.device
+    B, K1, _ = batch.zt.shape
+    K = K1 - 1
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    res = {}
+    for n in (1, 8):
+        sl = []
+        for r in range(n):
+            v0, v1 = shard_vocab(V, n, r)
+            zt_r = batch.zt[:, :, v0:v1].contiguous() if n > 1 else batch.zt
+            zd_r = batch.zd[:, :, v0:v1].contiguous() if n > 1 else batch.zd
+            sl.append((zt_r, zd_r, sv.vp_slice(zt_r, zd_r, V, v0, n, r)))
+        nst = sv.sv_vp_stats_bytes(sl[0][2])
+        stats_all = torch.empty(n * nst, dtype=torch.uint8, device=dev)
+        stats_local = torch.empty(nst, dtype=torch.uint8, device=dev)
+        mass_all = torch.empty(n * B, 2, dtype=torch.float32, device=dev)
+        mass_local = torch.empty(B, 2, dtype=torch.float32, device=dev)
+        ws = torch.empty(sv.sv_vp_workspace_bytes(sl[0][2]), dtype=torch.uint8, device=dev)
+        ot = torch.empty(B, K1, dtype=torch.int32, device=dev)
+        oa = torch.empty(B, dtype=torch.int32, device=dev)
+        for r, (_, _, d) in enumerate(sl):
+            sv.sv_vp_stats(d, batch.tokens, lengths, batch.temperature,
+                           stats_all[r * nst:(r + 1) * nst])
+        for r, (_, _, d) in enumerate(sl):
+            sv.sv_vp_decide(d, stats_all, batch.tokens, lengths, batch.temperature, seed, ot, oa,
+                            mass_all[r * B:(r + 1) * B], ws)
+        d0 = sl[0][2]
+        t_stats, t_step = [], []
+        for i in range(steps + 3):
+            flush.zero_()
+            a0 = torch.cuda.Event(enable_timing=True)
+            a1 = torch.cuda.Event(enable_timing=True)
+            a2 = torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            sv.sv_vp_stats(d0, batch.tokens, lengths, batch.temperature, stats_local)
+            a1.record(stream)
+            sv.sv_vp_decide(d0, stats_all, batch.tokens, lengths, batch.temperature, seed + i, ot,
+                            oa, mass_local, ws)
+            sv.sv_vp_draw(d0, mass_all, ot, ws)
+            a2.record(stream)
+            torch.cuda.synchronize()
+            if i >= 3:
+                t_stats.append(a0.elapsed_time(a1))
+                t_step.append(a0.elapsed_time(a2))
+        ms_stats = sum(t_stats) / len(t_stats)
+        ms_step = sum(t_step) / len(t_step)
+        v0, v1 = shard_vocab(V, n, 0)
+        bytes_rank = sched_bytes * (v1 - v0) / V
+        gbs = bytes_rank / (ms_stats / 1e3) / 1e9
+        res[f"n{n}"] = {"slice_tokens": v1 - v0, "rank_ms_per_step": round(ms_step, 5),
+                        "stats_kernel_ms": round(ms_stats, 5),
+                        "stats_bytes_per_launch": int(bytes_rank),
+                        "stats_gbs": round(gbs, 1), "stats_frac": round(gbs / peak, 4),
+                        "exchange_bytes_per_rank": int(nst + B * 8 + B * K1 * 4)}
+        del sl, stats_all
+    res["note"] = ("one rank's kernels per step with the vocabulary split n ways; the three "
+                   "collectives between them are not in these times (one GPU)")
+    res["kernel"] = "sv::vp::vp_stats_kernel"
+    res["launches_per_step"] = 3
+    return res
+
+
 def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -403,6 +475,11 @@ def run_ours(args, rank, world, local_rank):
                 "kernel_timing": "CUDA events around each stream-kernel launch over a second "
                                  "timed pass of the same steps"}
 
+    vocab = None
+    if rank == 0 and world == 1 and not args.no_vocab:
+        vocab = vocab_parallel_probe(batch, ln_buf, V, esize, sched_bytes, args.seed,
+                                     min(args.steps, 20), peak)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = oracle_sample(batch, lengths_np, args.cpu_seconds)
@@ -417,7 +494,7 @@ def run_ours(args, rank, world, local_rank):
                "e2e": e2e, "gpu_launches": args.steps * (sv.sv_verify_launches()
                                                          + (1 if fixed is None else 0)),
                "roofline": roofline, "cpu_baseline": cpu, "clocks": clk, "admission": admit,
-               "calibration": calib,
+               "calibration": calib, "vocab_parallel": vocab,
                "device_status": st, "impl": "ours"}
         print(json.dumps(out), flush=True)
     del batch
@@ -481,6 +558,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-vocab", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-rows", type=int, default=64)
     args = ap.parse_args()

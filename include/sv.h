@@ -194,11 +194,11 @@ size_t sv_verify_workspace_bytes(int B, int K, int V, sv_dtype dtype);
  * sv_verify -- batched speculative verification.
  *
  * Defined by: umans.ai page above, section "Speculative decoding, briefly"
- * (the target verifies the whole draft block in one pass, accepts the prefix
- * it agrees with plus a bonus token of its own, and discards the rest; the
- * acceptance rule is rejection sampling under which accepted tokens follow
- * the target distribution exactly, and a rejected token is replaced by one
- * the target would produce); zhichai.net DSpark topic, section "Why LLMs
+ * (one target pass scores the whole draft block; the drafts the target
+ * agrees with are kept, followed by one token of the target's own, and the
+ * rest are dropped; the test is rejection sampling, which leaves the emitted
+ * tokens distributed exactly as the target's, and a rejected draft gives way
+ * to a token of the target's choosing); zhichai.net DSpark topic, section "Why LLMs
  * speak so slowly" (rejection sampling on the target/draft probability
  * ratio; generation restarts from the first error).  In symbols, per row b
  * with verify length L = lengths[b] and temperature T = temperature[b]:
@@ -310,6 +310,124 @@ sv_status sv_verify_noalloc(const void *target_logits, const void *draft_logits,
                             const float *temperature, uint64_t seed, int64_t row_base,
                             int32_t *out_tokens, int32_t *out_accept_len, int32_t *status,
                             void *stream);
+
+/*
+ * Vocabulary-parallel verification: sv_vp_stats, sv_vp_decide, sv_vp_draw.
+ *
+ * The rule is that of sv_verify (the umans.ai and zhichai.net passages cited
+ * there), for a target and drafter whose output heads are split across
+ * ranks by vocabulary, so that each rank holds only a contiguous slice of
+ * both models' logits (zhichai.net DSpark topic, "From paper to running
+ * service in two weeks": the method is served by vLLM and SGLang on 8-GPU
+ * nodes; techvisionai "DeepSeek-V4: Breaking the Efficiency Barrier",
+ * Ch. 7 "Deployment with vLLM").  The pages do not say how the heads are
+ * split; slices ordered by rank that partition [0, V) are the reading taken.
+ *
+ * One verification step on every rank, with the caller's exchanges between:
+ *   sv_vp_stats     partials of this slice           -> stats_local
+ *   all-gather      stats_local of every rank, in rank order -> stats_all
+ *   sv_vp_decide    accept tests, accepted prefix    -> out_tokens, out_accept_len,
+ *                   this slice's draw masses          -> mass_local
+ *   all-gather      mass_local of every rank, in rank order -> mass_all
+ *   sv_vp_draw      the rank whose slice holds the draw writes the drawn token
+ *   all-reduce(max) out_tokens over the ranks
+ * Every rank computes the same normalisers, decisions and uniforms from the
+ * same gathered data, so out_accept_len and the accepted prefix agree on
+ * all ranks without an exchange; before the final all-reduce the drawn
+ * position holds -1 on every rank but one.  Results equal those of
+ * sv_verify on the whole vocabulary up to the rounding of the sums (fp32,
+ * a different summation order); decisions inside the tie windows of
+ * sv_verify may differ.  SV_NOTE_CDF_FALLBACK can be raised on one rank
+ * only (the one that drew); every other bit is raised on every rank.
+ *
+ * sv_vp_slice describes this rank's slice; every call of a step takes the
+ * same description.
+ */
+typedef struct {
+    const void *target_logits;  /* device [B, K+1, Vs] of dtype: this slice of zt */
+    const void *draft_logits;   /* device [B, K, Vs] of dtype, or NULL (greedy drafter) */
+    sv_dtype dtype;
+    int B, K;                   /* 1 <= B, 1 <= K <= SV_MAX_K */
+    int V;                      /* whole vocabulary, 1 <= V <= SV_MAX_V */
+    int v0, Vs;                 /* this slice holds tokens v0 .. v0+Vs-1; 1 <= Vs <= ceil(V / nshards) */
+    int nshards;                /* ranks the vocabulary is split over, 1 <= nshards <= V */
+    int shard;                  /* this rank's place in slice order, 0 .. nshards-1 */
+} sv_vp_slice;
+
+/*
+ * sv_vp_stats_bytes -- bytes of stats_local: B * (2K+1) * C records of 16
+ * bytes, C = ceil(ceil(V / nshards) * elt / 65536) clamped to [1, 64] (the
+ * same on every rank).  stats_all is nshards times that.  0 for an invalid
+ * slice.
+ * sv_vp_workspace_bytes -- per-rank scratch of sv_vp_decide and sv_vp_draw:
+ * a 48-byte draw record per row and two segment tables of the slice (at most
+ * 2 * 512 floats per row).  0 for an invalid slice.
+ */
+size_t sv_vp_stats_bytes(const sv_vp_slice *slice);
+size_t sv_vp_workspace_bytes(const sv_vp_slice *slice);
+
+/*
+ * sv_vp_stats -- per (row, slot, chunk) of the slice: (m, Sigma, z_x, w) with
+ * m = max z, Sigma = sum exp((z - m) / T) over the chunk; in chunk 0, z_x is
+ * the logit of the row's draft token at that position and w = 1 when the
+ * slice holds the token (else z_x = 0, w = 0).  Greedy rows (T == 0): (max,
+ * 0, 0, global index of the first argmax).  Slot i <= K is target position
+ * i, slot K+1+i draft position i; only the slots sv_vp_decide reads
+ * (target 0..L, draft 0..L-1 of sampled rows with draft logits) are written;
+ * rows with a bad length or temperature are skipped.
+ *   draft_tokens, lengths, temperature  as for sv_verify.
+ *   stats_local  device, sv_vp_stats_bytes() bytes, 16-byte aligned, written.
+ * Returns SV_OK, SV_ERR_ARG, SV_ERR_SHAPE, SV_ERR_DTYPE or SV_ERR_CUDA.
+ */
+sv_status sv_vp_stats(const sv_vp_slice *slice, const int32_t *draft_tokens,
+                      const int32_t *lengths, const float *temperature, void *stats_local,
+                      void *stream);
+
+/*
+ * sv_vp_decide -- per row: validates it (as sv_verify: an invalid row gets
+ * -1 everywhere and its SV_ROW_* bit), merges the partials of every rank in
+ * a fixed order, runs the accept tests with u(seed, row, i, 0), writes
+ * out_accept_len[b] = j and out_tokens[b] = x_0 .. x_{j-1}, y, -1 ... where
+ * y is the target argmax for greedy rows and -1 (to be drawn) otherwise,
+ * and sums this slice's draw weights at position j.
+ *   stats_all      device [nshards] x stats_local, rank order, 16-byte aligned.
+ *   seed, row_base as for sv_verify.
+ *   out_tokens     device int32 [B, K+1]; out_accept_len device int32 [B].
+ *   mass_local     device float32 [B, 2], 8-byte aligned, written: the
+ *                  slice's total draw weight and its total unnormalised
+ *                  target weight (the zero-residual fallback); 0 for rows
+ *                  with no draw.
+ *   norm_out       device float32 [B, 2K+1, 2], nullable: the merged
+ *                  (m, Sigma) of every slot read (as sv_verify_debug).
+ *   workspace      device, >= sv_vp_workspace_bytes(), 16-byte aligned,
+ *                  kept for sv_vp_draw of the same step.
+ *   status         device int32, nullable; bits OR-ed in.
+ * Returns SV_OK, SV_ERR_ARG, SV_ERR_SHAPE, SV_ERR_DTYPE, SV_ERR_WORKSPACE or
+ * SV_ERR_CUDA.
+ */
+sv_status sv_vp_decide(const sv_vp_slice *slice, const void *stats_all,
+                       const int32_t *draft_tokens, const int32_t *lengths,
+                       const float *temperature, uint64_t seed, int64_t row_base,
+                       int32_t *out_tokens, int32_t *out_accept_len, float *mass_local,
+                       float *norm_out, void *workspace, size_t workspace_bytes,
+                       int32_t *status, void *stream);
+
+/*
+ * sv_vp_draw -- per row with a draw: R = sum of the slices' masses in rank
+ * order (the unnormalised target weight if the draw's own mass is zero,
+ * raising SV_NOTE_ZERO_RESIDUAL), t = u(seed, row, j, 1) * R; the slice
+ * whose exclusive prefix is <= t < prefix + mass holds the token, and only
+ * that rank writes out_tokens[b, j] = the smallest token of its slice whose
+ * cumulative weight passes t (the last positive one, with
+ * SV_NOTE_CDF_FALLBACK, if rounding leaves t at or past the total).
+ *   mass_all   device float32 [nshards, B, 2], rank order, 8-byte aligned.
+ *   out_tokens as written by sv_vp_decide of this step.
+ *   workspace  the one sv_vp_decide of this step used.
+ * Returns SV_OK, SV_ERR_ARG, SV_ERR_SHAPE, SV_ERR_DTYPE, SV_ERR_WORKSPACE or
+ * SV_ERR_CUDA.
+ */
+sv_status sv_vp_draw(const sv_vp_slice *slice, const float *mass_all, int32_t *out_tokens,
+                     void *workspace, size_t workspace_bytes, int32_t *status, void *stream);
 
 /*
  * sv_philox_uniforms -- the uniforms sv_verify draws, for tests:

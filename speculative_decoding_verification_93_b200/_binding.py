@@ -59,6 +59,14 @@ def lib():
                                   sz, vp, vp, vp]
     L.sv_verify_noalloc.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, u64, i64, vp, vp, vp,
                                     vp]
+    sp = ctypes.POINTER(sv_vp_slice)
+    L.sv_vp_stats_bytes.argtypes = [sp]
+    L.sv_vp_stats_bytes.restype = sz
+    L.sv_vp_workspace_bytes.argtypes = [sp]
+    L.sv_vp_workspace_bytes.restype = sz
+    L.sv_vp_stats.argtypes = [sp, vp, vp, vp, vp, vp]
+    L.sv_vp_decide.argtypes = [sp, vp, vp, vp, vp, u64, i64, vp, vp, vp, vp, vp, sz, vp, vp]
+    L.sv_vp_draw.argtypes = [sp, vp, vp, vp, sz, vp, vp]
     L.sv_philox_uniforms.argtypes = [u64, vp, vp, vp, i32, vp, vp]
     L.sv_philox4x32_10.argtypes = [vp, vp, i32, vp, vp]
     L.sv_profile_begin.argtypes = [i32]
@@ -67,7 +75,8 @@ def lib():
     L.sv_status_string.argtypes = [i32]
     L.sv_status_string.restype = ctypes.c_char_p
     for name in ("sv_schedule", "sv_schedule_admit", "sv_sts_fit", "sv_sts_apply", "sv_verify",
-                 "sv_verify_debug", "sv_verify_noalloc",
+                 "sv_verify_debug", "sv_verify_noalloc", "sv_vp_stats", "sv_vp_decide",
+                 "sv_vp_draw",
                  "sv_philox_uniforms",
                  "sv_philox4x32_10", "sv_profile_begin"):
         getattr(L, name).restype = i32
@@ -76,6 +85,31 @@ def lib():
     L.sv_verify_launches.restype = i32
     _lib = L
     return L
+
+
+class sv_vp_slice(ctypes.Structure):
+    """This rank's slice of the vocabulary (``sv_vp_slice`` in include/sv.h)."""
+    _fields_ = [("target_logits", ctypes.c_void_p), ("draft_logits", ctypes.c_void_p),
+                ("dtype", ctypes.c_int), ("B", ctypes.c_int), ("K", ctypes.c_int),
+                ("V", ctypes.c_int), ("v0", ctypes.c_int), ("Vs", ctypes.c_int),
+                ("nshards", ctypes.c_int), ("shard", ctypes.c_int)]
+
+
+def vp_slice(target_logits, draft_logits, V: int, v0: int, nshards: int,
+             shard: int) -> sv_vp_slice:
+    """Describe a slice from its logits: target [B, K+1, Vs], draft [B, K, Vs]
+    or None, holding tokens v0 .. v0+Vs-1 of a vocabulary of V."""
+    B, K1, Vs = target_logits.shape
+    dt = _dtype(target_logits)
+    if not target_logits.is_contiguous():
+        raise TypeError("target_logits must be contiguous")
+    if draft_logits is not None and (draft_logits.dtype != target_logits.dtype
+                                     or not draft_logits.is_contiguous()
+                                     or tuple(draft_logits.shape) != (B, K1 - 1, Vs)):
+        raise TypeError("draft_logits must be a contiguous [B, K, Vs] tensor of the target dtype")
+    return sv_vp_slice(target_logits.data_ptr(),
+                       None if draft_logits is None else draft_logits.data_ptr(),
+                       dt, B, K1 - 1, int(V), int(v0), Vs, int(nshards), int(shard))
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -208,6 +242,44 @@ def sv_verify_noalloc(target_logits, draft_logits, draft_tokens, lengths, temper
         _ptr(target_logits), _ptr(draft_logits), dt, B, K, V, _ptr(draft_tokens), _ptr(lengths),
         _ptr(temperature), ctypes.c_uint64(seed & (2**64 - 1)), int(row_base), _ptr(out_tokens),
         _ptr(out_accept_len), _ptr(status), _stream(stream, target_logits)))
+
+
+def sv_vp_stats_bytes(slice_: sv_vp_slice) -> int:
+    return int(lib().sv_vp_stats_bytes(ctypes.byref(slice_)))
+
+
+def sv_vp_workspace_bytes(slice_: sv_vp_slice) -> int:
+    return int(lib().sv_vp_workspace_bytes(ctypes.byref(slice_)))
+
+
+def sv_vp_stats(slice_: sv_vp_slice, draft_tokens, lengths, temperature, stats_local,
+                stream=None) -> None:
+    _need(draft_tokens, torch.int32, "draft_tokens")
+    _need(lengths, torch.int32, "lengths")
+    _need(temperature, torch.float32, "temperature")
+    _check("sv_vp_stats", lib().sv_vp_stats(
+        ctypes.byref(slice_), _ptr(draft_tokens), _ptr(lengths), _ptr(temperature),
+        _ptr(stats_local), _stream(stream, lengths)))
+
+
+def sv_vp_decide(slice_: sv_vp_slice, stats_all, draft_tokens, lengths, temperature, seed: int,
+                 out_tokens, out_accept_len, mass_local, workspace, status=None, norm_out=None,
+                 row_base: int = 0, stream=None) -> None:
+    _need(draft_tokens, torch.int32, "draft_tokens")
+    _need(lengths, torch.int32, "lengths")
+    _need(temperature, torch.float32, "temperature")
+    _check("sv_vp_decide", lib().sv_vp_decide(
+        ctypes.byref(slice_), _ptr(stats_all), _ptr(draft_tokens), _ptr(lengths),
+        _ptr(temperature), ctypes.c_uint64(seed & (2**64 - 1)), int(row_base), _ptr(out_tokens),
+        _ptr(out_accept_len), _ptr(mass_local), _ptr(norm_out), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream, lengths)))
+
+
+def sv_vp_draw(slice_: sv_vp_slice, mass_all, out_tokens, workspace, status=None,
+               stream=None) -> None:
+    _check("sv_vp_draw", lib().sv_vp_draw(
+        ctypes.byref(slice_), _ptr(mass_all), _ptr(out_tokens), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream, out_tokens)))
 
 
 def sv_philox_uniforms(seed: int, row, pos, draw, out, stream=None) -> None:

@@ -217,81 +217,6 @@ __global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(VerifyArgs a
 // ---------------------------------------------------------------------------
 constexpr int kGroup = kConsumers;   // threads of the consumer group
 
-// Online (max, sum) update with a batch of units.  The batch max is a
-// balanced tree of packed bf16x2 (or f32) max operations; the running sum is
-// rescaled once if the max grew; then one exp2 per element with the
-// argument formed by one packed FMA, z * k + c with c = RN(-m * k).  The
-// rounding of c is exact to recover, -m * k = c + e with e = fma(-m, k, -c),
-// and common to the batch, so the batch sum is multiplied by 2^e
-// (= 1 + e ln 2 to far below fp32 resolution, |e| < 1e-6).  Two packed
-// accumulators halve the add chain.
-template <int ESIZE, int N>
-__device__ __forceinline__ void lse_update(const uint4 (&v)[N], float k, float &m, float &s) {
-    float bm;
-    if (ESIZE == 2) {
-        uint32_t t[N];
-#pragma unroll
-        for (int j = 0; j < N; ++j) t[j] = bmax2(bmax2(v[j].x, v[j].y), bmax2(v[j].z, v[j].w));
-#pragma unroll
-        for (int w = 1; w < N; w <<= 1)
-#pragma unroll
-            for (int j = 0; j + w < N; j += 2 * w) t[j] = bmax2(t[j], t[j + w]);
-        bm = fmaxf(bf16_lo(t[0]), bf16_hi(t[0]));
-    } else {
-        float t[N];
-#pragma unroll
-        for (int j = 0; j < N; ++j)
-            t[j] = fmaxf(fmaxf(__uint_as_float(v[j].x), __uint_as_float(v[j].y)),
-                         fmaxf(__uint_as_float(v[j].z), __uint_as_float(v[j].w)));
-#pragma unroll
-        for (int w = 1; w < N; w <<= 1)
-#pragma unroll
-            for (int j = 0; j + w < N; j += 2 * w) t[j] = fmaxf(t[j], t[j + w]);
-        bm = t[0];
-    }
-    if (bm == kNegInf) return;              // nothing but padding / -inf
-    if (bm > m) {
-        s = (m == kNegInf) ? 0.f : s * ex2((m - bm) * k);
-        m = bm;
-    }
-    const float c = -m * k;
-    const float e = fmaf(-m, k, -c);
-    const float2 cc = make_float2(c, c), kk = make_float2(k, k);
-    float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int j = 0; j < N; ++j) {
-        const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
-        if (ESIZE == 2) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float2 z = make_float2(bf16_lo(w[q]), bf16_hi(w[q]));
-                const float2 d = __ffma2_rn(z, kk, cc);
-                const float2 e = make_float2(ex2(d.x), ex2(d.y));
-                if (q & 1) acc1 = __fadd2_rn(acc1, e); else acc0 = __fadd2_rn(acc0, e);
-            }
-        } else {
-#pragma unroll
-            for (int q = 0; q < 4; q += 2) {
-                const float2 z = make_float2(__uint_as_float(w[q]), __uint_as_float(w[q + 1]));
-                const float2 d = __ffma2_rn(z, kk, cc);
-                const float2 e = make_float2(ex2(d.x), ex2(d.y));
-                if (q & 2) acc1 = __fadd2_rn(acc1, e); else acc0 = __fadd2_rn(acc0, e);
-            }
-        }
-    }
-    s = fmaf((acc0.x + acc0.y) + (acc1.x + acc1.y), fmaf(e, 0.69314718055994531f, 1.f), s);
-}
-
-template <int ESIZE>
-__device__ __forceinline__ void consider_unit(const uint4 &u, int first, float &best, int &bidx) {
-    constexpr int kPer = 16 / ESIZE;
-#pragma unroll
-    for (int e = 0; e < kPer; ++e) {
-        const float x = unit_elem<ESIZE>(u, e);
-        if (x > best) { best = x; bidx = first + e; }
-    }
-}
-
 struct __align__(16) StageDesc {
     int b;        // row; -1 = no more work
     int slot;

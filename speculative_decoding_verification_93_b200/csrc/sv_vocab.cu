@@ -1,0 +1,757 @@
+// sv_vocab.cu -- verification with the vocabulary split across ranks (sm_100a).
+//
+// Method: the rule of sv_verify -- umans.ai, "DeepSeek V4 Pro DSpark: the
+// model isn't ready, the architecture is", section "Speculative decoding,
+// briefly"; zhichai.net DSpark topic, section "Why LLMs speak so slowly" --
+// evaluated where each rank holds only a contiguous slice [v0, v0 + Vs) of
+// both models' logits, as a multi-GPU serving engine whose output heads are
+// split by vocabulary produces them (zhichai.net topic, "From paper to
+// running service in two weeks": the method runs inside vLLM and SGLang on
+// 8-GPU nodes; techvisionai "DeepSeek-V4: Breaking the Efficiency Barrier",
+// Ch. 7 "Deployment with vLLM").
+//
+// Three local steps; the caller runs an exchange after each of the first two
+// and one at the end:
+//   1. vp_stats_kernel, one CTA per (row, slot, chunk) of the slice: the
+//      online (max, sum of exp2) of the chunk (greedy rows: max and first
+//      argmax), plus -- in chunk 0 -- the logit of the row's draft token when
+//      the token falls in the slice.  Exchange: all-gather, rank order.
+//   2. vp_decide_kernel, one CTA per row: merges every rank's partials in a
+//      fixed order, so every rank holds the same normalisers and takes the
+//      same decisions; runs the accept tests; writes the accepted prefix and
+//      the accept length; then sums the draw weights of its own slice at the
+//      final position, by segments of 16-byte units, into a table.
+//      Exchange: all-gather of the per-row slice totals, rank order.
+//   3. vp_draw_kernel, one warp per row: every rank scans the slice totals in
+//      rank order and finds the slice that holds the CDF target; only that
+//      rank locates the token, from its segment table and then inside one
+//      segment.  Other ranks leave -1 there.  Exchange: all-reduce (max) of
+//      out_tokens, after which every rank holds the same result.
+// Every sum runs in a fixed order; nothing waits on another CTA.
+#include <climits>
+#include <cstdint>
+
+#include "sv.h"
+#include "sv_device.cuh"
+#include "sv_host.h"
+
+namespace sv {
+namespace vp {
+
+constexpr int kStatsThreads = 256;
+constexpr int kStatsWarps = kStatsThreads / 32;
+constexpr int kBatch = 8;                      // 16-byte units per thread per load batch
+constexpr int kChunkBytes = 64 * 1024;         // target bytes per stats chunk
+constexpr int kMaxChunks = 64;
+constexpr int kDecideThreads = 256;
+constexpr int kDecideWarps = kDecideThreads / 32;
+constexpr int kMaxSlots = 2 * SV_MAX_K + 1;
+constexpr int kMaxSeg = 512;                   // segments per slice vector
+constexpr int kModeDone = -1, kModeP = 0, kModeResidual = 1, kModeOneHot = 2;
+
+struct __align__(16) Record {
+    int j;        // draw position
+    int mode;     // kModeDone (outputs complete), kModeP, kModeResidual, kModeOneHot
+    int xl;       // one-hot mode: slice-local index of x_j, or -1 if outside the slice
+    int pad0;
+    float u, k;   // draw uniform; log2(e) / T
+    float mt, ct, md, cd;   // weight offsets, as in sv_verify
+    int pad1[2];
+};
+
+struct Args {
+    const char *zt, *zd;    // slices [B, K+1, Vs], [B, K, Vs]
+    int B, K, V, v0, Vs, S, C, nshards, shard;
+    int SU, G;              // units per segment, segments per table
+    const int32_t *tokens, *lengths;
+    const float *temp;
+    uint64_t seed;
+    int64_t row_base;
+    float4 *stats_local;        // [B, S, C]
+    const float4 *stats_all;    // [nshards, B, S, C]
+    float2 *mass_local;         // [B]: (mode mass, p mass)
+    const float2 *mass_all;     // [nshards, B]
+    int32_t *out_tokens, *out_accept, *status;
+    float *norm;                // nullable [B, S, 2]
+    Record *rec;                // [B]
+    float *seg;                 // [B, 2, G]
+};
+
+__device__ __forceinline__ bool bad_temperature(float T) {
+    return !(T >= 0.f) || isinf(T) || (T > 0.f && T < 1e-6f);
+}
+
+template <int ESIZE>
+__device__ __forceinline__ const char *tgt_vec(const Args &a, int b, int i) {
+    return a.zt + ((static_cast<long long>(b) * (a.K + 1) + i) * a.Vs) * ESIZE;
+}
+template <int ESIZE>
+__device__ __forceinline__ const char *dft_vec(const Args &a, int b, int i) {
+    return a.zd + ((static_cast<long long>(b) * a.K + i) * a.Vs) * ESIZE;
+}
+
+// ---------------------------------------------------------------------------
+// 1. Slice statistics.
+// ---------------------------------------------------------------------------
+template <int ESIZE>
+__global__ void __launch_bounds__(kStatsThreads, 4) vp_stats_kernel(Args a) {
+    constexpr int kPer = 16 / ESIZE;
+    griddep_wait();
+    griddep_launch_dependents();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int c = static_cast<int>(blockIdx.x % a.C);
+    const int bs = static_cast<int>(blockIdx.x / a.C);
+    const int slot = bs % a.S, b = bs / a.S;
+    const int L = __ldg(&a.lengths[b]);
+    const float T = __ldg(&a.temp[b]);
+    if (L < 0 || L > a.K || bad_temperature(T)) return;   // the decide step marks the row
+    const bool greedy = !(T > 0.f);
+    const float k = greedy ? 0.f : kLog2e / T;
+    int i;
+    const char *base;
+    if (slot <= a.K) {
+        i = slot;
+        if (i > L) return;
+        base = tgt_vec<ESIZE>(a, b, i);
+    } else {
+        i = slot - a.K - 1;
+        if (greedy || a.zd == nullptr || i >= L) return;
+        base = dft_vec<ESIZE>(a, b, i);
+    }
+    const VecGeom g = vec_geom<ESIZE>(base, a.Vs);
+    const int U = (g.n16 + a.C - 1) / a.C;
+    const int u0 = min(c * U, g.n16), u1 = min(u0 + U, g.n16);
+    const uint32_t pw = neg_inf_word<ESIZE>();
+    const uint4 pad = make_uint4(pw, pw, pw, pw);
+
+    float m = kNegInf, s = 0.f;
+    int idx = INT_MAX;
+    // Head elements (chunk 0, thread 0) precede every body element.
+    if (c == 0 && tid == 0 && g.head > 0) {
+        const uint4 hu = ld_partial_unit<ESIZE>(g.base, 0, g.head);
+        if (greedy) {
+            consider_unit<ESIZE>(hu, 0, m, idx);
+        } else {
+            const uint4 h1[1] = {hu};
+            lse_update<ESIZE, 1>(h1, k, m, s);
+        }
+    }
+    for (int ub = u0; ub < u1; ub += kBatch * kStatsThreads) {
+        uint4 v[kBatch];
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+            const int u = ub + q * kStatsThreads + tid;
+            v[q] = u < u1 ? ld_stream(g.body + static_cast<long long>(u) * 16) : pad;
+        }
+        if (greedy) {
+#pragma unroll
+            for (int q = 0; q < kBatch; ++q)
+                consider_unit<ESIZE>(v[q], g.head + (ub + q * kStatsThreads + tid) * kPer, m, idx);
+        } else {
+            lse_update<ESIZE, kBatch>(v, k, m, s);
+        }
+    }
+    // Tail elements (last chunk, thread 1) follow every body element.
+    if (c == a.C - 1 && tid == 1 && g.tail > 0) {
+        const int first = g.head + g.n16 * kPer;
+        const uint4 tu = ld_partial_unit<ESIZE>(g.base, first, g.tail);
+        if (greedy) {
+            consider_unit<ESIZE>(tu, first, m, idx);
+        } else {
+            const uint4 t1[1] = {tu};
+            lse_update<ESIZE, 1>(t1, k, m, s);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+        const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+        const int i2 = __shfl_xor_sync(0xffffffffu, idx, o);
+        if (greedy) {
+            if (m2 > m || (m2 == m && i2 < idx)) { m = m2; idx = i2; }
+        } else {
+            lse_merge(m, s, m2, s2, k);
+        }
+    }
+    __shared__ float4 wp[kStatsWarps];
+    if (lane == 0) wp[warp] = make_float4(m, s, 0.f, __int_as_float(idx));
+    __syncthreads();
+    if (tid != 0) return;
+    float rm = wp[0].x, rs = wp[0].y;
+    int ri = __float_as_int(wp[0].w);
+    for (int w = 1; w < kStatsWarps; ++w) {
+        const float4 p = wp[w];
+        const int i2 = __float_as_int(p.w);
+        if (greedy) {
+            if (p.x > rm || (p.x == rm && i2 < ri)) { rm = p.x; ri = i2; }
+        } else {
+            lse_merge(rm, rs, p.x, p.y, k);
+        }
+    }
+    float4 out;
+    if (greedy) {
+        // Slice-local argmax made global.
+        out = make_float4(rm, 0.f, 0.f, __int_as_float(ri == INT_MAX ? INT_MAX : a.v0 + ri));
+    } else {
+        // Chunk 0 carries the draft token's logit when the slice holds it.
+        float zx = 0.f;
+        int own = 0;
+        if (c == 0 && i < L) {
+            const int xl = __ldg(&a.tokens[static_cast<long long>(b) * a.K + i]) - a.v0;
+            if (xl >= 0 && xl < a.Vs) { zx = ld_elem<ESIZE>(g.base, xl); own = 1; }
+        }
+        out = make_float4(rm, rs, zx, __int_as_float(own));
+    }
+    a.stats_local[(static_cast<long long>(b) * a.S + slot) * a.C + c] = out;
+}
+
+// ---------------------------------------------------------------------------
+// Draw weights of one 16-byte unit of the slice at the draw position.
+// Local unit lu: 0 = head, 1..n16 = body units, n16+1 = tail.
+// ---------------------------------------------------------------------------
+struct DrawCtx {
+    VecGeom gt, gd;
+    bool aligned;     // target and draft slices share their 16-byte phase
+    int mode, xl, NU;
+    float k, mt, ct, md, cd;
+};
+
+template <int ESIZE>
+__device__ __forceinline__ void load_unit(const DrawCtx &c, int lu, bool want_draft, uint4 &t,
+                                          uint4 &d, int &first, int &count) {
+    constexpr int kPer = 16 / ESIZE;
+    const uint32_t pw = neg_inf_word<ESIZE>();
+    d = make_uint4(pw, pw, pw, pw);
+    if (lu == 0) {
+        first = 0; count = c.gt.head;
+        t = ld_partial_unit<ESIZE>(c.gt.base, 0, count);
+    } else if (lu <= c.gt.n16) {
+        first = c.gt.head + (lu - 1) * kPer; count = kPer;
+        t = ld_reuse(c.gt.body + static_cast<long long>(lu - 1) * 16);
+    } else {
+        first = c.gt.head + c.gt.n16 * kPer; count = c.gt.tail;
+        t = ld_partial_unit<ESIZE>(c.gt.base, first, count);
+    }
+    if (want_draft && c.aligned) {
+        if (lu >= 1 && lu <= c.gt.n16) d = ld_reuse(c.gd.body + static_cast<long long>(lu - 1) * 16);
+        else d = ld_partial_unit<ESIZE>(c.gd.base, first, count);
+    }
+}
+
+// Weights of the elements of a loaded unit: table 0 is the draw's own
+// weight (p, p without x_j, or max(0, p - q)), table 1 the unnormalised p
+// that a zero residual falls back to.  Elements past `count` weigh 0.
+template <int ESIZE>
+__device__ __forceinline__ float elem_weight(const DrawCtx &c, int table, const uint4 &t,
+                                             const uint4 &d, int first, int count, int e) {
+    if (e >= count) return 0.f;
+    const float z = unit_elem<ESIZE>(t, e);
+    if (table == 1 || c.mode == kModeP) return ex2((z - c.mt) * c.k);
+    if (c.mode == kModeOneHot) return (first + e == c.xl) ? 0.f : ex2((z - c.mt) * c.k);
+    const float zd = c.aligned ? unit_elem<ESIZE>(d, e) : ld_elem<ESIZE>(c.gd.base, first + e);
+    const float p = ex2(fmaf(z - c.mt, c.k, -c.ct));
+    const float q = ex2(fmaf(zd - c.md, c.k, -c.cd));
+    return fmaxf(p - q, 0.f);
+}
+
+template <int ESIZE>
+__device__ __forceinline__ float unit_weight(const DrawCtx &c, int table, const uint4 &t,
+                                             const uint4 &d, int first, int count) {
+    constexpr int kPer = 16 / ESIZE;
+    float w = 0.f;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) w += elem_weight<ESIZE>(c, table, t, d, first, count, e);
+    return w;
+}
+
+template <int ESIZE>
+__device__ __forceinline__ DrawCtx draw_ctx(const Args &a, int b, const Record &r) {
+    DrawCtx c;
+    c.gt = vec_geom<ESIZE>(tgt_vec<ESIZE>(a, b, r.j), a.Vs);
+    const bool resid = r.mode == kModeResidual;
+    c.gd = resid ? vec_geom<ESIZE>(dft_vec<ESIZE>(a, b, r.j), a.Vs) : c.gt;
+    c.aligned = !resid || c.gd.head == c.gt.head;
+    c.mode = r.mode;
+    c.xl = r.xl;
+    c.NU = c.gt.n16 + 2;
+    c.k = r.k; c.mt = r.mt; c.ct = r.ct; c.md = r.md; c.cd = r.cd;
+    return c;
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// ---------------------------------------------------------------------------
+// 2. Decide: merge, accept tests, outputs, slice draw masses.
+// ---------------------------------------------------------------------------
+struct DecideSmem {
+    float m[kMaxSlots], s[kMaxSlots], zx[kMaxSlots];
+    int arg[kMaxSlots];
+    int bits, L, j;
+    Record rec;
+};
+
+template <int ESIZE>
+__global__ void __launch_bounds__(kDecideThreads) vp_decide_kernel(Args a) {
+    __shared__ DecideSmem sm;
+    griddep_wait();
+    griddep_launch_dependents();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int b = blockIdx.x, K = a.K, S = a.S;
+    const float T = __ldg(&a.temp[b]);
+    if (tid == 0) {
+        const int L = __ldg(&a.lengths[b]);
+        int bits = 0;
+        if (L < 0 || L > K) bits |= SV_ROW_BAD_LENGTH;
+        if (bad_temperature(T)) bits |= SV_ROW_BAD_TEMPERATURE;
+        if (!(bits & SV_ROW_BAD_LENGTH))
+            for (int i = 0; i < L; ++i) {
+                const int x = __ldg(&a.tokens[static_cast<long long>(b) * K + i]);
+                if (x < 0 || x >= a.V) { bits |= SV_ROW_BAD_TOKEN; break; }
+            }
+        sm.bits = bits;
+        sm.L = L;
+    }
+    __syncthreads();
+    if (sm.bits) {
+        for (int t = tid; t <= K; t += kDecideThreads)
+            a.out_tokens[static_cast<long long>(b) * (K + 1) + t] = -1;
+        if (tid == 0) {
+            a.out_accept[b] = -1;
+            if (a.status) atomicOr(a.status, sm.bits);
+            a.rec[b].mode = kModeDone;
+            a.mass_local[b] = make_float2(0.f, 0.f);
+        }
+        return;
+    }
+    const int L = sm.L;
+    const bool greedy = !(T > 0.f);
+    const bool has_draft = a.zd != nullptr && !greedy;
+    const float k = greedy ? 0.f : kLog2e / T;
+
+    // Normalisers: target slots 0..L and draft slots 0..L-1, each merged
+    // over (rank, chunk) in a fixed order by one warp.
+    const int nslot = L + 1 + (has_draft ? L : 0);
+    const int nparts = a.nshards * a.C;
+    for (int q = warp; q < nslot; q += kDecideWarps) {
+        const int slot = q <= L ? q : K + 1 + (q - L - 1);
+        float m = kNegInf, s = 0.f, zx = 0.f;
+        int idx = INT_MAX, own = 0;
+        for (int p = lane; p < nparts; p += 32) {
+            const int r = p / a.C, c = p - r * a.C;
+            const float4 v =
+                __ldg(&a.stats_all[((static_cast<long long>(r) * a.B + b) * S + slot) * a.C + c]);
+            const int w = __float_as_int(v.w);
+            if (greedy) {
+                if (v.x > m || (v.x == m && w < idx)) { m = v.x; idx = w; }
+            } else {
+                lse_merge(m, s, v.x, v.y, k);
+                if (w && !own) { zx = v.z; own = 1; }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+            const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+            const int i2 = __shfl_xor_sync(0xffffffffu, idx, o);
+            const float z2 = __shfl_xor_sync(0xffffffffu, zx, o);
+            const int o2 = __shfl_xor_sync(0xffffffffu, own, o);
+            if (greedy) {
+                if (m2 > m || (m2 == m && i2 < idx)) { m = m2; idx = i2; }
+            } else {
+                lse_merge(m, s, m2, s2, k);
+                if (o2 && !own) { zx = z2; own = 1; }
+            }
+        }
+        if (lane == 0) {
+            sm.m[slot] = m;
+            sm.s[slot] = greedy ? 1.f : s;
+            sm.zx[slot] = own ? zx : kNegInf;
+            sm.arg[slot] = idx == INT_MAX ? 0 : idx;
+            if (a.norm) {
+                a.norm[(static_cast<long long>(b) * S + slot) * 2 + 0] = m;
+                a.norm[(static_cast<long long>(b) * S + slot) * 2 + 1] = greedy ? 1.f : s;
+            }
+        }
+    }
+    __syncthreads();
+
+    // Accept tests in position order (the same rule as sv_verify).
+    const uint64_t row = static_cast<uint64_t>(a.row_base) + static_cast<uint64_t>(b);
+    if (tid == 0) {
+        int j = L;
+        for (int i = 0; i < L; ++i) {
+            const int x = __ldg(&a.tokens[static_cast<long long>(b) * K + i]);
+            bool acc;
+            if (greedy) {
+                acc = x == sm.arg[i];
+            } else {
+                const float lp = fmaf(sm.zx[i] - sm.m[i], k, -log2f(sm.s[i]));
+                float lq = 0.f;
+                if (has_draft)
+                    lq = fmaf(sm.zx[K + 1 + i] - sm.m[K + 1 + i], k, -log2f(sm.s[K + 1 + i]));
+                const float u = uniform24(a.seed, row, static_cast<uint32_t>(i), 0u);
+                if (lp == kNegInf) acc = false;
+                else if (lq == kNegInf) acc = true;
+                else acc = (lp >= lq) || (u < exp2f(lp - lq));
+            }
+            if (!acc) { j = i; break; }
+        }
+        sm.j = j;
+        Record r;
+        r.j = j;
+        r.pad0 = 0; r.pad1[0] = r.pad1[1] = 0;
+        r.k = k;
+        r.u = greedy ? 0.f : uniform24(a.seed, row, static_cast<uint32_t>(j), 1u);
+        r.mt = sm.m[j];
+        const bool resid = has_draft && j < L;
+        r.mode = greedy ? kModeDone : (j == L ? kModeP : (resid ? kModeResidual : kModeOneHot));
+        r.ct = resid ? log2f(sm.s[j]) : 0.f;
+        r.md = resid ? sm.m[K + 1 + j] : 0.f;
+        r.cd = resid ? log2f(sm.s[K + 1 + j]) : 0.f;
+        r.xl = -1;
+        if (r.mode == kModeOneHot) {
+            const int xl = __ldg(&a.tokens[static_cast<long long>(b) * K + j]) - a.v0;
+            r.xl = (xl >= 0 && xl < a.Vs) ? xl : -1;
+        }
+        sm.rec = r;
+        a.rec[b] = r;
+        a.out_accept[b] = j;
+    }
+    __syncthreads();
+    const int j = sm.j;
+    for (int t = tid; t <= K; t += kDecideThreads) {
+        int v = -1;
+        if (t < j) v = __ldg(&a.tokens[static_cast<long long>(b) * K + t]);
+        else if (t == j && greedy) v = sm.arg[j];
+        a.out_tokens[static_cast<long long>(b) * (K + 1) + t] = v;
+    }
+    if (greedy) {
+        if (tid == 0) a.mass_local[b] = make_float2(0.f, 0.f);
+        return;
+    }
+
+    // Slice draw masses at position j by segments of SU units: rounds of 32
+    // units, each round's warp sum added to the segment in round order.
+    const DrawCtx c = draw_ctx<ESIZE>(a, b, sm.rec);
+    const bool want_draft = c.mode == kModeResidual;
+    float *tb = a.seg + static_cast<long long>(b) * 2 * a.G;
+    for (int g = warp; g < a.G; g += kDecideWarps) {
+        const int e0 = min(g * a.SU, c.NU), e1 = min(e0 + a.SU, c.NU);
+        float s0 = 0.f, s1 = 0.f;
+        for (int r0 = e0; r0 < e1; r0 += 32) {
+            const int lu = r0 + lane;
+            float w0 = 0.f, w1 = 0.f;
+            if (lu < e1) {
+                uint4 t, d;
+                int first, count;
+                load_unit<ESIZE>(c, lu, want_draft, t, d, first, count);
+                w0 = unit_weight<ESIZE>(c, 0, t, d, first, count);
+                w1 = unit_weight<ESIZE>(c, 1, t, d, first, count);
+            }
+            s0 += warp_sum(w0);
+            s1 += warp_sum(w1);
+        }
+        if (lane == 0) { tb[g] = s0; tb[a.G + g] = s1; }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        float W0 = 0.f, W1 = 0.f;
+        for (int g = 0; g < a.G; ++g) { W0 += tb[g]; W1 += tb[a.G + g]; }
+        a.mass_local[b] = make_float2(W0, W1);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 3. Draw: owner slice by the slice totals in rank order; the owner locates
+//    the token.
+// ---------------------------------------------------------------------------
+template <int ESIZE>
+__global__ void __launch_bounds__(32) vp_draw_kernel(Args a) {
+    constexpr int kPer = 16 / ESIZE;
+    griddep_wait();
+    griddep_launch_dependents();
+    const int lane = threadIdx.x, b = blockIdx.x;
+    const Record r = a.rec[b];
+    if (r.mode == kModeDone) return;
+    int owner = 0, table = 0, note = 0;
+    float tl = 0.f;
+    if (lane == 0) {
+        float R = 0.f;
+        for (int q = 0; q < a.nshards; ++q) R += a.mass_all[static_cast<long long>(q) * a.B + b].x;
+        if (!(R > 0.f)) {
+            // A rejection that left no residual mass: draw from p_j.
+            if (r.mode != kModeP) note |= SV_NOTE_ZERO_RESIDUAL;
+            table = 1;
+            R = 0.f;
+            for (int q = 0; q < a.nshards; ++q)
+                R += a.mass_all[static_cast<long long>(q) * a.B + b].y;
+        }
+        const float t = r.u * R;
+        float cum = 0.f;
+        owner = -1;
+        int last = 0;
+        for (int q = 0; q < a.nshards; ++q) {
+            const float2 mq = a.mass_all[static_cast<long long>(q) * a.B + b];
+            const float w = table ? mq.y : mq.x;
+            if (w > 0.f) last = q;
+            if (owner < 0 && cum + w > t) { owner = q; tl = t - cum; }
+            if (owner < 0) cum += w;
+        }
+        if (owner < 0) {
+            // Rounding left the target at or past the total: the last slice
+            // with positive weight, and inside it the last positive element.
+            owner = last;
+            tl = __int_as_float(0x7f800000);   // +inf: falls through every scan
+            note |= SV_NOTE_CDF_FALLBACK;
+        }
+        if (note && a.status) atomicOr(a.status, note);
+    }
+    owner = __shfl_sync(0xffffffffu, owner, 0);
+    if (owner != a.shard) return;
+    table = __shfl_sync(0xffffffffu, table, 0);
+    tl = __shfl_sync(0xffffffffu, tl, 0);
+
+    // Segment: sequential scan of the table in the order its total was formed.
+    const float *tb = a.seg + static_cast<long long>(b) * 2 * a.G + (table ? a.G : 0);
+    int gsel = 0;
+    float tg = 0.f;
+    bool fb = false;
+    if (lane == 0) {
+        float cum = 0.f;
+        int last = 0;
+        gsel = -1;
+        for (int g = 0; g < a.G; ++g) {
+            const float w = tb[g];
+            if (w > 0.f) last = g;
+            if (gsel < 0 && cum + w > tl) { gsel = g; tg = tl - cum; }
+            if (gsel < 0) cum += w;
+        }
+        if (gsel < 0) { gsel = last; fb = true; }
+    }
+    gsel = __shfl_sync(0xffffffffu, gsel, 0);
+    tg = __shfl_sync(0xffffffffu, tg, 0);
+    fb = __shfl_sync(0xffffffffu, fb ? 1 : 0, 0) != 0;
+
+    // Inside the segment: rounds of 32 units, running sum of the round warp
+    // sums exactly as the segment total was formed; the lane whose inclusive
+    // prefix first passes the target scans its unit's elements.
+    const DrawCtx c = draw_ctx<ESIZE>(a, b, r);
+    const bool want_draft = c.mode == kModeResidual && table == 0;
+    const int e0 = min(gsel * a.SU, c.NU), e1 = min(e0 + a.SU, c.NU);
+    float running = 0.f;
+    int y = -1, ylast = -1;
+    for (int r0 = e0; r0 < e1 && y < 0; r0 += 32) {
+        const int lu = r0 + lane;
+        uint4 t = make_uint4(0, 0, 0, 0), d = make_uint4(0, 0, 0, 0);
+        int first = 0, count = 0;
+        float w = 0.f;
+        if (lu < e1) {
+            load_unit<ESIZE>(c, lu, want_draft, t, d, first, count);
+            w = unit_weight<ESIZE>(c, table, t, d, first, count);
+        }
+        // Last positive element of this round (fallback).
+        const unsigned pos = __ballot_sync(0xffffffffu, w > 0.f);
+        if (pos) {
+            const int hl = 31 - __clz(pos);
+            int le = -1;
+            if (lane == hl)
+                for (int e = 0; e < kPer; ++e)
+                    if (elem_weight<ESIZE>(c, table, t, d, first, count, e) > 0.f) le = first + e;
+            ylast = __shfl_sync(0xffffffffu, le, hl);
+        }
+        const float tot = warp_sum(w);
+        if (!fb && running + tot > tg) {
+            float incl = w;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            const unsigned hit = __ballot_sync(0xffffffffu, running + incl > tg);
+            if (hit) {
+                const int hl = __ffs(hit) - 1;
+                int ye = -1;
+                if (lane == hl) {
+                    float cc = running + (incl - w);
+                    int lp = -1;
+                    for (int e = 0; e < kPer && ye < 0; ++e) {
+                        const float we = elem_weight<ESIZE>(c, table, t, d, first, count, e);
+                        if (we > 0.f) lp = first + e;
+                        cc += we;
+                        if (cc > tg && we > 0.f) ye = first + e;
+                    }
+                    if (ye < 0) ye = lp;   // rounding inside the unit
+                }
+                y = __shfl_sync(0xffffffffu, ye, hl);
+                if (y < 0) y = ylast;
+            } else {
+                y = ylast;            // rounding inside the round
+            }
+            if (y >= 0) break;
+        }
+        running += tot;
+    }
+    if (y < 0) y = ylast >= 0 ? ylast : 0;
+    if (lane == 0) a.out_tokens[static_cast<long long>(b) * (a.K + 1) + r.j] = a.v0 + y;
+}
+
+// ---------------------------------------------------------------------------
+// Host side.
+// ---------------------------------------------------------------------------
+struct Plan {
+    int es, S, C, SU, G;
+    size_t stats_bytes, off_seg, ws_bytes;
+};
+
+static bool make_plan(const sv_vp_slice *s, Plan *p) {
+    if (s->B < 1 || s->K < 1 || s->K > SV_MAX_K || s->V < 1 || s->V > SV_MAX_V) return false;
+    if (s->nshards < 1 || s->nshards > s->V || s->shard < 0 || s->shard >= s->nshards) return false;
+    const int vmax = (s->V + s->nshards - 1) / s->nshards;
+    if (s->Vs < 1 || s->Vs > vmax || s->v0 < 0 || s->v0 > s->V - s->Vs) return false;
+    if (s->dtype != SV_F32 && s->dtype != SV_BF16) return false;
+    p->es = s->dtype == SV_F32 ? 4 : 2;
+    p->S = 2 * s->K + 1;
+    // Chunks from the largest slice, so that every rank uses the same count.
+    const long long vbytes = static_cast<long long>(vmax) * p->es;
+    p->C = static_cast<int>((vbytes + kChunkBytes - 1) / kChunkBytes);
+    if (p->C < 1) p->C = 1;
+    if (p->C > kMaxChunks) p->C = kMaxChunks;
+    const long long blocks = static_cast<long long>(s->B) * p->S * p->C;
+    if (blocks >= INT_MAX) return false;
+    const long long nu = static_cast<long long>(s->Vs) * p->es / 16 + 2;   // >= any vector's n16 + 2
+    const long long per = (nu + kMaxSeg - 1) / kMaxSeg;
+    p->SU = static_cast<int>((per + 31) / 32 * 32);
+    p->G = static_cast<int>((nu + p->SU - 1) / p->SU);
+    p->stats_bytes = sizeof(float4) * static_cast<size_t>(blocks);
+    const size_t rec = sizeof(Record) * static_cast<size_t>(s->B);
+    p->off_seg = (rec + 15) & ~static_cast<size_t>(15);
+    p->ws_bytes = p->off_seg + sizeof(float) * 2 * static_cast<size_t>(p->G) * s->B;
+    return true;
+}
+
+static sv_status check_slice(const sv_vp_slice *s, Plan *p) {
+    if (!s || !s->target_logits) return SV_ERR_ARG;
+    if (s->dtype != SV_F32 && s->dtype != SV_BF16) return SV_ERR_DTYPE;
+    if (!make_plan(s, p)) return SV_ERR_SHAPE;
+    if ((reinterpret_cast<uintptr_t>(s->target_logits) % p->es) ||
+        (s->draft_logits && (reinterpret_cast<uintptr_t>(s->draft_logits) % p->es)))
+        return SV_ERR_ARG;
+    return SV_OK;
+}
+
+static Args base_args(const sv_vp_slice *s, const Plan &p) {
+    Args a = {};
+    a.zt = static_cast<const char *>(s->target_logits);
+    a.zd = static_cast<const char *>(s->draft_logits);
+    a.B = s->B; a.K = s->K; a.V = s->V; a.v0 = s->v0; a.Vs = s->Vs;
+    a.S = p.S; a.C = p.C; a.nshards = s->nshards; a.shard = s->shard;
+    a.SU = p.SU; a.G = p.G;
+    return a;
+}
+
+static bool aligned16(const void *q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; }
+
+}  // namespace vp
+}  // namespace sv
+
+using sv::vp::Plan;
+
+extern "C" size_t sv_vp_stats_bytes(const sv_vp_slice *s) {
+    Plan p;
+    if (!s || !sv::vp::make_plan(s, &p)) return 0;
+    return p.stats_bytes;
+}
+
+extern "C" size_t sv_vp_workspace_bytes(const sv_vp_slice *s) {
+    Plan p;
+    if (!s || !sv::vp::make_plan(s, &p)) return 0;
+    return p.ws_bytes;
+}
+
+extern "C" sv_status sv_vp_stats(const sv_vp_slice *s, const int32_t *draft_tokens,
+                                 const int32_t *lengths, const float *temperature,
+                                 void *stats_local, void *stream) {
+    Plan p;
+    const sv_status st0 = sv::vp::check_slice(s, &p);
+    if (st0 != SV_OK) return st0;
+    if (!draft_tokens || !lengths || !temperature || !stats_local) return SV_ERR_ARG;
+    if (!sv::vp::aligned16(stats_local)) return SV_ERR_ARG;
+    sv::vp::Args a = sv::vp::base_args(s, p);
+    a.tokens = draft_tokens; a.lengths = lengths; a.temp = temperature;
+    a.stats_local = static_cast<float4 *>(stats_local);
+    const unsigned grid = static_cast<unsigned>(s->B) * static_cast<unsigned>(p.S * p.C);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    sv::profile_mark_begin(st);
+    const cudaError_t e =
+        p.es == 4 ? sv::launch_pdl(sv::vp::vp_stats_kernel<4>, dim3(grid),
+                                   dim3(sv::vp::kStatsThreads), 0, st, a)
+                  : sv::launch_pdl(sv::vp::vp_stats_kernel<2>, dim3(grid),
+                                   dim3(sv::vp::kStatsThreads), 0, st, a);
+    if (e != cudaSuccess) return sv::note_cuda(e);
+    sv::profile_mark_end(st);
+    return sv::note_cuda(cudaGetLastError());
+}
+
+extern "C" sv_status sv_vp_decide(const sv_vp_slice *s, const void *stats_all,
+                                  const int32_t *draft_tokens, const int32_t *lengths,
+                                  const float *temperature, uint64_t seed, int64_t row_base,
+                                  int32_t *out_tokens, int32_t *out_accept_len, float *mass_local,
+                                  float *norm_out, void *workspace, size_t workspace_bytes,
+                                  int32_t *status, void *stream) {
+    Plan p;
+    const sv_status st0 = sv::vp::check_slice(s, &p);
+    if (st0 != SV_OK) return st0;
+    if (!stats_all || !draft_tokens || !lengths || !temperature || !out_tokens ||
+        !out_accept_len || !mass_local || !workspace)
+        return SV_ERR_ARG;
+    if (row_base < 0 || !sv::vp::aligned16(stats_all) || !sv::vp::aligned16(workspace) ||
+        (reinterpret_cast<uintptr_t>(mass_local) & 7))
+        return SV_ERR_ARG;
+    if (workspace_bytes < p.ws_bytes) return SV_ERR_WORKSPACE;
+    sv::vp::Args a = sv::vp::base_args(s, p);
+    a.tokens = draft_tokens; a.lengths = lengths; a.temp = temperature;
+    a.seed = seed; a.row_base = row_base;
+    a.stats_all = static_cast<const float4 *>(stats_all);
+    a.mass_local = reinterpret_cast<float2 *>(mass_local);
+    a.out_tokens = out_tokens; a.out_accept = out_accept_len; a.status = status;
+    a.norm = norm_out;
+    char *w = static_cast<char *>(workspace);
+    a.rec = reinterpret_cast<sv::vp::Record *>(w);
+    a.seg = reinterpret_cast<float *>(w + p.off_seg);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const cudaError_t e =
+        p.es == 4 ? sv::launch_pdl(sv::vp::vp_decide_kernel<4>, dim3(s->B),
+                                   dim3(sv::vp::kDecideThreads), 0, st, a)
+                  : sv::launch_pdl(sv::vp::vp_decide_kernel<2>, dim3(s->B),
+                                   dim3(sv::vp::kDecideThreads), 0, st, a);
+    if (e != cudaSuccess) return sv::note_cuda(e);
+    return sv::note_cuda(cudaGetLastError());
+}
+
+extern "C" sv_status sv_vp_draw(const sv_vp_slice *s, const float *mass_all, int32_t *out_tokens,
+                                void *workspace, size_t workspace_bytes, int32_t *status,
+                                void *stream) {
+    Plan p;
+    const sv_status st0 = sv::vp::check_slice(s, &p);
+    if (st0 != SV_OK) return st0;
+    if (!mass_all || !out_tokens || !workspace) return SV_ERR_ARG;
+    if (!sv::vp::aligned16(workspace) || (reinterpret_cast<uintptr_t>(mass_all) & 7))
+        return SV_ERR_ARG;
+    if (workspace_bytes < p.ws_bytes) return SV_ERR_WORKSPACE;
+    sv::vp::Args a = sv::vp::base_args(s, p);
+    a.mass_all = reinterpret_cast<const float2 *>(mass_all);
+    a.out_tokens = out_tokens; a.status = status;
+    char *w = static_cast<char *>(workspace);
+    a.rec = reinterpret_cast<sv::vp::Record *>(w);
+    a.seg = reinterpret_cast<float *>(w + p.off_seg);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const cudaError_t e =
+        p.es == 4 ? sv::launch_pdl(sv::vp::vp_draw_kernel<4>, dim3(s->B), dim3(32), 0, st, a)
+                  : sv::launch_pdl(sv::vp::vp_draw_kernel<2>, dim3(s->B), dim3(32), 0, st, a);
+    if (e != cudaSuccess) return sv::note_cuda(e);
+    return sv::note_cuda(cudaGetLastError());
+}

@@ -120,3 +120,47 @@ def test_sts_arguments_rejected_on_host():
     assert sv.sv_sts_workspace_bytes(100, 4) > 0 and sv.sv_sts_workspace_bytes(100, 65) == 0
     assert L.sv_sts_apply(None, v(1), 1, 1, v(1), None) == 1
     assert L.sv_sts_apply(v(1), v(1), 1, 65, v(1), None) == 2
+
+
+def test_vocab_parallel_arguments_rejected_on_host():
+    L = sv.lib()
+    v = ctypes.c_void_p
+    big = 1 << 30
+
+    def sl(**kw):
+        d = dict(t=1 << 20, d=1 << 21, dtype=sv.SV_BF16, B=4, K=4, V=1000, v0=0, Vs=500, n=2, r=0)
+        d.update(kw)
+        return sv.sv_vp_slice(d["t"], d["d"], d["dtype"], d["B"], d["K"], d["V"], d["v0"],
+                              d["Vs"], d["n"], d["r"])
+    ok = sl()
+    assert sv.sv_vp_stats_bytes(ok) == 4 * 9 * 1 * 16
+    assert sv.sv_vp_workspace_bytes(ok) > 0
+    # largest slice sets the chunk count on every rank: 129280 bf16 / 1 rank
+    assert sv.sv_vp_stats_bytes(sl(V=129280, Vs=129280, n=1)) == 4 * 9 * 4 * 16
+    for bad in (sl(Vs=501), sl(v0=501), sl(r=2), sl(n=1001, Vs=1), sl(K=65), sl(K=0), sl(B=0),
+                sl(V=0), sl(dtype=7), sl(Vs=0), sl(v0=-1), sl(V=(1 << 20) + 1)):
+        assert sv.sv_vp_stats_bytes(bad) == 0 and sv.sv_vp_workspace_bytes(bad) == 0
+    p = v(1 << 22)
+    R = ctypes.byref
+    assert L.sv_vp_stats(None, p, p, p, p, None) == 1
+    assert L.sv_vp_stats(R(sl(t=0)), p, p, p, p, None) == 1
+    assert L.sv_vp_stats(R(ok), None, p, p, p, None) == 1
+    assert L.sv_vp_stats(R(ok), p, p, p, v((1 << 22) + 8), None) == 1
+    assert L.sv_vp_stats(R(sl(dtype=5)), p, p, p, p, None) == 3
+    assert L.sv_vp_stats(R(sl(Vs=600)), p, p, p, p, None) == 2
+    assert L.sv_vp_stats(R(sl(t=(1 << 20) + 1)), p, p, p, p, None) == 1
+
+    def decide(s=ok, stats=p, ws=p, wsb=big, row_base=0, mass=p):
+        return L.sv_vp_decide(R(s), stats, p, p, p, ctypes.c_uint64(0), row_base, p, p, mass,
+                              None, ws, wsb, None, None)
+    assert decide(wsb=16) == 4
+    assert decide(row_base=-1) == 1
+    assert decide(stats=v((1 << 22) + 4)) == 1
+    assert decide(ws=v((1 << 22) + 8)) == 1
+    assert decide(mass=v((1 << 22) + 4)) == 1
+    assert decide(stats=None) == 1
+    assert decide(s=sl(K=65)) == 2
+    assert L.sv_vp_draw(R(ok), p, p, p, 16, None, None) == 4
+    assert L.sv_vp_draw(R(ok), v((1 << 22) + 4), p, p, big, None, None) == 1
+    assert L.sv_vp_draw(R(ok), None, p, p, big, None, None) == 1
+    assert L.sv_vp_draw(R(sl(r=-1)), p, p, p, big, None, None) == 2
