@@ -360,8 +360,9 @@ typedef struct {
  * same on every rank).  stats_all is nshards times that.  0 for an invalid
  * slice.
  * sv_vp_workspace_bytes -- per-rank scratch of sv_vp_decide and sv_vp_draw:
- * a 48-byte draw record per row and two segment tables of the slice (at most
- * 2 * 512 floats per row).  0 for an invalid slice.
+ * a 48-byte draw record, two segment tables of the slice (at most 2 * 512
+ * floats), their part sums (at most 2 * 32 floats) and a counter per row.
+ * 0 for an invalid slice.
  */
 size_t sv_vp_stats_bytes(const sv_vp_slice *slice);
 size_t sv_vp_workspace_bytes(const sv_vp_slice *slice);
@@ -403,7 +404,8 @@ sv_status sv_vp_stats(const sv_vp_slice *slice, const int32_t *draft_tokens,
  *                  kept for sv_vp_draw of the same step.
  *   status         device int32, nullable; bits OR-ed in.
  * Returns SV_OK, SV_ERR_ARG, SV_ERR_SHAPE, SV_ERR_DTYPE, SV_ERR_WORKSPACE or
- * SV_ERR_CUDA.
+ * SV_ERR_CUDA.  Two launches: the decisions (one CTA per row), then the
+ * slice masses (up to 32 CTAs per row).
  */
 sv_status sv_vp_decide(const sv_vp_slice *slice, const void *stats_all,
                        const int32_t *draft_tokens, const int32_t *lengths,

@@ -19,8 +19,10 @@
 //   2. vp_decide_kernel, one CTA per row: merges every rank's partials in a
 //      fixed order, so every rank holds the same normalisers and takes the
 //      same decisions; runs the accept tests; writes the accepted prefix and
-//      the accept length; then sums the draw weights of its own slice at the
-//      final position, by segments of 16-byte units, into a table.
+//      the accept length.  vp_mass_kernel, several CTAs per row: sums the
+//      draw weights of this slice at the final position by segments of
+//      16-byte units, the segments by parts, the parts into the slice total
+//      (the row's last CTA, found by an atomic count).
 //      Exchange: all-gather of the per-row slice totals, rank order.
 //   3. vp_draw_kernel, one warp per row: every rank scans the slice totals in
 //      rank order and finds the slice that holds the CDF target; only that
@@ -47,6 +49,11 @@ constexpr int kDecideThreads = 256;
 constexpr int kDecideWarps = kDecideThreads / 32;
 constexpr int kMaxSlots = 2 * SV_MAX_K + 1;
 constexpr int kMaxSeg = 512;                   // segments per slice vector
+constexpr int kSegPerPart = 32;                // segments per mass CTA (a part)
+constexpr int kMassThreads = 256;
+constexpr int kMassWarps = kMassThreads / 32;
+static_assert(kSegPerPart == 32, "the draw loads one part's segment sums, one per lane");
+static_assert(kMaxSeg / kSegPerPart <= 32, "the draw loads the part sums, one per lane");
 constexpr int kModeDone = -1, kModeP = 0, kModeResidual = 1, kModeOneHot = 2;
 
 struct __align__(16) Record {
@@ -55,14 +62,14 @@ struct __align__(16) Record {
     int xl;       // one-hot mode: slice-local index of x_j, or -1 if outside the slice
     int pad0;
     float u, k;   // draw uniform; log2(e) / T
-    float mt, ct, md, cd;   // weight offsets, as in sv_verify
+    float mt, ist, md, isd; // maxima and reciprocal sums: p = 2^((z - mt) k) * ist
     int pad1[2];
 };
 
 struct Args {
     const char *zt, *zd;    // slices [B, K+1, Vs], [B, K, Vs]
     int B, K, V, v0, Vs, S, C, nshards, shard;
-    int SU, G;              // units per segment, segments per table
+    int SU, G, P;           // units per segment, segments per table, parts per table
     const int32_t *tokens, *lengths;
     const float *temp;
     uint64_t seed;
@@ -74,7 +81,9 @@ struct Args {
     int32_t *out_tokens, *out_accept, *status;
     float *norm;                // nullable [B, S, 2]
     Record *rec;                // [B]
-    float *seg;                 // [B, 2, G]
+    float *seg;                 // [B, 2, G] segment sums (draw weight, p weight)
+    float *part;                // [B, 2, P] part sums: kSegPerPart segments each, in order
+    int *cnt;                   // [B] mass CTAs of the row finished
 };
 
 __device__ __forceinline__ bool bad_temperature(float T) {
@@ -213,7 +222,7 @@ struct DrawCtx {
     VecGeom gt, gd;
     bool aligned;     // target and draft slices share their 16-byte phase
     int mode, xl, NU;
-    float k, mt, ct, md, cd;
+    float k, mt, ist, md, isd;
 };
 
 template <int ESIZE>
@@ -239,29 +248,49 @@ __device__ __forceinline__ void load_unit(const DrawCtx &c, int lu, bool want_dr
 }
 
 // Weights of the elements of a loaded unit: table 0 is the draw's own
-// weight (p, p without x_j, or max(0, p - q)), table 1 the unnormalised p
-// that a zero residual falls back to.  Elements past `count` weigh 0.
+// weight (p, p without x_j, or max(0, p - q) with p and q normalised),
+// table 1 the unnormalised p that a zero residual falls back to.  Elements
+// past `count` weigh 0.  One exp2 per element and model: the normalised p
+// is the unnormalised one times 1 / Sigma.
+template <int ESIZE>
+__device__ __forceinline__ float2 elem_weights(const DrawCtx &c, const uint4 &t, const uint4 &d,
+                                               int first, int count, int e) {
+    if (e >= count) return make_float2(0.f, 0.f);
+    const float pu = ex2((unit_elem<ESIZE>(t, e) - c.mt) * c.k);
+    if (c.mode == kModeP) return make_float2(pu, pu);
+    if (c.mode == kModeOneHot) return make_float2(first + e == c.xl ? 0.f : pu, pu);
+    const float zd = c.aligned ? unit_elem<ESIZE>(d, e) : ld_elem<ESIZE>(c.gd.base, first + e);
+    const float q = ex2((zd - c.md) * c.k) * c.isd;
+    return make_float2(fmaxf(fmaf(pu, c.ist, -q), 0.f), pu);
+}
+
 template <int ESIZE>
 __device__ __forceinline__ float elem_weight(const DrawCtx &c, int table, const uint4 &t,
                                              const uint4 &d, int first, int count, int e) {
-    if (e >= count) return 0.f;
-    const float z = unit_elem<ESIZE>(t, e);
-    if (table == 1 || c.mode == kModeP) return ex2((z - c.mt) * c.k);
-    if (c.mode == kModeOneHot) return (first + e == c.xl) ? 0.f : ex2((z - c.mt) * c.k);
-    const float zd = c.aligned ? unit_elem<ESIZE>(d, e) : ld_elem<ESIZE>(c.gd.base, first + e);
-    const float p = ex2(fmaf(z - c.mt, c.k, -c.ct));
-    const float q = ex2(fmaf(zd - c.md, c.k, -c.cd));
-    return fmaxf(p - q, 0.f);
+    const float2 w = elem_weights<ESIZE>(c, t, d, first, count, e);
+    return table ? w.y : w.x;
+}
+
+// Both tables' weight of a unit, each summed in element order.
+template <int ESIZE>
+__device__ __forceinline__ float2 unit_weights(const DrawCtx &c, const uint4 &t, const uint4 &d,
+                                               int first, int count) {
+    constexpr int kPer = 16 / ESIZE;
+    float w0 = 0.f, w1 = 0.f;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) {
+        const float2 w = elem_weights<ESIZE>(c, t, d, first, count, e);
+        w0 += w.x;
+        w1 += w.y;
+    }
+    return make_float2(w0, w1);
 }
 
 template <int ESIZE>
 __device__ __forceinline__ float unit_weight(const DrawCtx &c, int table, const uint4 &t,
                                              const uint4 &d, int first, int count) {
-    constexpr int kPer = 16 / ESIZE;
-    float w = 0.f;
-#pragma unroll
-    for (int e = 0; e < kPer; ++e) w += elem_weight<ESIZE>(c, table, t, d, first, count, e);
-    return w;
+    const float2 w = unit_weights<ESIZE>(c, t, d, first, count);
+    return table ? w.y : w.x;
 }
 
 template <int ESIZE>
@@ -274,7 +303,7 @@ __device__ __forceinline__ DrawCtx draw_ctx(const Args &a, int b, const Record &
     c.mode = r.mode;
     c.xl = r.xl;
     c.NU = c.gt.n16 + 2;
-    c.k = r.k; c.mt = r.mt; c.ct = r.ct; c.md = r.md; c.cd = r.cd;
+    c.k = r.k; c.mt = r.mt; c.ist = r.ist; c.md = r.md; c.isd = r.isd;
     return c;
 }
 
@@ -290,7 +319,8 @@ __device__ __forceinline__ float warp_sum(float x) {
 struct DecideSmem {
     float m[kMaxSlots], s[kMaxSlots], zx[kMaxSlots];
     int arg[kMaxSlots];
-    int bits, L, j;
+    int tok[SV_MAX_K];
+    int j;
     Record rec;
 };
 
@@ -301,33 +331,31 @@ __global__ void __launch_bounds__(kDecideThreads) vp_decide_kernel(Args a) {
     griddep_launch_dependents();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = blockIdx.x, K = a.K, S = a.S;
+    // Row checks, with the row's draft tokens loaded in parallel.
+    const int L = __ldg(&a.lengths[b]);
     const float T = __ldg(&a.temp[b]);
-    if (tid == 0) {
-        const int L = __ldg(&a.lengths[b]);
-        int bits = 0;
-        if (L < 0 || L > K) bits |= SV_ROW_BAD_LENGTH;
-        if (bad_temperature(T)) bits |= SV_ROW_BAD_TEMPERATURE;
-        if (!(bits & SV_ROW_BAD_LENGTH))
-            for (int i = 0; i < L; ++i) {
-                const int x = __ldg(&a.tokens[static_cast<long long>(b) * K + i]);
-                if (x < 0 || x >= a.V) { bits |= SV_ROW_BAD_TOKEN; break; }
-            }
-        sm.bits = bits;
-        sm.L = L;
+    int bits = 0;
+    if (L < 0 || L > K) bits |= SV_ROW_BAD_LENGTH;
+    if (bad_temperature(T)) bits |= SV_ROW_BAD_TEMPERATURE;
+    int x = 0;
+    if (tid < K) {
+        x = __ldg(&a.tokens[static_cast<long long>(b) * K + tid]);
+        sm.tok[tid] = x;
     }
-    __syncthreads();
-    if (sm.bits) {
+    const bool bad_tok = !(bits & SV_ROW_BAD_LENGTH) && tid < L && (x < 0 || x >= a.V);
+    if (__syncthreads_or(bad_tok)) bits |= SV_ROW_BAD_TOKEN;
+    if (tid == 0) a.cnt[b] = 0;   // the mass kernel of this step counts its CTAs here
+    if (bits) {
         for (int t = tid; t <= K; t += kDecideThreads)
             a.out_tokens[static_cast<long long>(b) * (K + 1) + t] = -1;
         if (tid == 0) {
             a.out_accept[b] = -1;
-            if (a.status) atomicOr(a.status, sm.bits);
+            if (a.status) atomicOr(a.status, bits);
             a.rec[b].mode = kModeDone;
             a.mass_local[b] = make_float2(0.f, 0.f);
         }
         return;
     }
-    const int L = sm.L;
     const bool greedy = !(T > 0.f);
     const bool has_draft = a.zd != nullptr && !greedy;
     const float k = greedy ? 0.f : kLog2e / T;
@@ -379,88 +407,143 @@ __global__ void __launch_bounds__(kDecideThreads) vp_decide_kernel(Args a) {
     }
     __syncthreads();
 
-    // Accept tests in position order (the same rule as sv_verify).
+    // Accept tests (the rule of sv_verify), one position per lane of warp
+    // 0: each depends only on its own position's normalisers and uniform, so
+    // the first rejection is the lowest lane that rejects.
     const uint64_t row = static_cast<uint64_t>(a.row_base) + static_cast<uint64_t>(b);
-    if (tid == 0) {
+    if (warp == 0) {
         int j = L;
-        for (int i = 0; i < L; ++i) {
-            const int x = __ldg(&a.tokens[static_cast<long long>(b) * K + i]);
-            bool acc;
-            if (greedy) {
-                acc = x == sm.arg[i];
-            } else {
-                const float lp = fmaf(sm.zx[i] - sm.m[i], k, -log2f(sm.s[i]));
-                float lq = 0.f;
-                if (has_draft)
-                    lq = fmaf(sm.zx[K + 1 + i] - sm.m[K + 1 + i], k, -log2f(sm.s[K + 1 + i]));
-                const float u = uniform24(a.seed, row, static_cast<uint32_t>(i), 0u);
-                if (lp == kNegInf) acc = false;
-                else if (lq == kNegInf) acc = true;
-                else acc = (lp >= lq) || (u < exp2f(lp - lq));
+        for (int i0 = 0; i0 < L; i0 += 32) {
+            const int i = i0 + lane;
+            bool rej = false;
+            if (i < L) {
+                const int xi = sm.tok[i];
+                if (greedy) {
+                    rej = xi != sm.arg[i];
+                } else {
+                    const float lp = fmaf(sm.zx[i] - sm.m[i], k, -log2f(sm.s[i]));
+                    float lq = 0.f;
+                    if (has_draft)
+                        lq = fmaf(sm.zx[K + 1 + i] - sm.m[K + 1 + i], k,
+                                  -log2f(sm.s[K + 1 + i]));
+                    const float u = uniform24(a.seed, row, static_cast<uint32_t>(i), 0u);
+                    bool acc;
+                    if (lp == kNegInf) acc = false;
+                    else if (lq == kNegInf) acc = true;
+                    else acc = (lp >= lq) || (u < exp2f(lp - lq));
+                    rej = !acc;
+                }
             }
-            if (!acc) { j = i; break; }
+            const unsigned bal = __ballot_sync(0xffffffffu, rej);
+            if (bal) { j = i0 + __ffs(bal) - 1; break; }
         }
-        sm.j = j;
-        Record r;
-        r.j = j;
-        r.pad0 = 0; r.pad1[0] = r.pad1[1] = 0;
-        r.k = k;
-        r.u = greedy ? 0.f : uniform24(a.seed, row, static_cast<uint32_t>(j), 1u);
-        r.mt = sm.m[j];
-        const bool resid = has_draft && j < L;
-        r.mode = greedy ? kModeDone : (j == L ? kModeP : (resid ? kModeResidual : kModeOneHot));
-        r.ct = resid ? log2f(sm.s[j]) : 0.f;
-        r.md = resid ? sm.m[K + 1 + j] : 0.f;
-        r.cd = resid ? log2f(sm.s[K + 1 + j]) : 0.f;
-        r.xl = -1;
-        if (r.mode == kModeOneHot) {
-            const int xl = __ldg(&a.tokens[static_cast<long long>(b) * K + j]) - a.v0;
-            r.xl = (xl >= 0 && xl < a.Vs) ? xl : -1;
+        if (lane == 0) {
+            sm.j = j;
+            Record r;
+            r.j = j;
+            r.pad0 = 0; r.pad1[0] = r.pad1[1] = 0;
+            r.k = k;
+            r.u = greedy ? 0.f : uniform24(a.seed, row, static_cast<uint32_t>(j), 1u);
+            r.mt = sm.m[j];
+            const bool resid = has_draft && j < L;
+            r.mode = greedy ? kModeDone : (j == L ? kModeP : (resid ? kModeResidual : kModeOneHot));
+            r.ist = resid ? 1.f / sm.s[j] : 1.f;
+            r.md = resid ? sm.m[K + 1 + j] : 0.f;
+            r.isd = resid ? 1.f / sm.s[K + 1 + j] : 1.f;
+            r.xl = -1;
+            if (r.mode == kModeOneHot) {
+                const int xl = sm.tok[j] - a.v0;
+                r.xl = (xl >= 0 && xl < a.Vs) ? xl : -1;
+            }
+            sm.rec = r;
+            a.rec[b] = r;
+            a.out_accept[b] = j;
         }
-        sm.rec = r;
-        a.rec[b] = r;
-        a.out_accept[b] = j;
     }
     __syncthreads();
     const int j = sm.j;
     for (int t = tid; t <= K; t += kDecideThreads) {
         int v = -1;
-        if (t < j) v = __ldg(&a.tokens[static_cast<long long>(b) * K + t]);
+        if (t < j) v = sm.tok[t];
         else if (t == j && greedy) v = sm.arg[j];
         a.out_tokens[static_cast<long long>(b) * (K + 1) + t] = v;
     }
-    if (greedy) {
-        if (tid == 0) a.mass_local[b] = make_float2(0.f, 0.f);
-        return;
-    }
+    if (greedy && tid == 0) a.mass_local[b] = make_float2(0.f, 0.f);
+}
 
-    // Slice draw masses at position j by segments of SU units: rounds of 32
-    // units, each round's warp sum added to the segment in round order.
-    const DrawCtx c = draw_ctx<ESIZE>(a, b, sm.rec);
+// ---------------------------------------------------------------------------
+// 2b. Slice draw masses at the draw position: kSegPerPart segments of SU
+//     units per CTA (two per warp), each segment summed in rounds of 32
+//     units with the round's warp sum added in round order; the CTA adds its
+//     segments in order into its part sum; the last CTA of the row (atomic
+//     count, no waiting) adds the parts in order into the slice total.
+// ---------------------------------------------------------------------------
+template <int ESIZE>
+__global__ void __launch_bounds__(kMassThreads, 4) vp_mass_kernel(Args a) {
+    __shared__ float s0v[kSegPerPart], s1v[kSegPerPart];
+    __shared__ int is_last;
+    griddep_wait();
+    griddep_launch_dependents();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int b = static_cast<int>(blockIdx.x / a.P), p = static_cast<int>(blockIdx.x % a.P);
+    const Record r = a.rec[b];
+    if (r.mode == kModeDone) return;   // greedy or invalid row: no draw
+    const DrawCtx c = draw_ctx<ESIZE>(a, b, r);
     const bool want_draft = c.mode == kModeResidual;
     float *tb = a.seg + static_cast<long long>(b) * 2 * a.G;
-    for (int g = warp; g < a.G; g += kDecideWarps) {
-        const int e0 = min(g * a.SU, c.NU), e1 = min(e0 + a.SU, c.NU);
-        float s0 = 0.f, s1 = 0.f;
-        for (int r0 = e0; r0 < e1; r0 += 32) {
-            const int lu = r0 + lane;
-            float w0 = 0.f, w1 = 0.f;
-            if (lu < e1) {
-                uint4 t, d;
-                int first, count;
-                load_unit<ESIZE>(c, lu, want_draft, t, d, first, count);
-                w0 = unit_weight<ESIZE>(c, 0, t, d, first, count);
-                w1 = unit_weight<ESIZE>(c, 1, t, d, first, count);
-            }
-            s0 += warp_sum(w0);
-            s1 += warp_sum(w1);
+    // Warp w holds segments w + 8q, q = 0..3; per round of 32 units the
+    // loads of all four segments are issued before any weight is computed.
+    constexpr int kQ = kSegPerPart / kMassWarps;
+    const int g0 = p * kSegPerPart + warp;
+    float s0[kQ], s1[kQ];
+#pragma unroll
+    for (int q = 0; q < kQ; ++q) { s0[q] = 0.f; s1[q] = 0.f; }
+    for (int r0 = 0; r0 < a.SU; r0 += 32) {
+        uint4 t[kQ], d[kQ];
+        int first[kQ], count[kQ];
+        bool in[kQ];
+#pragma unroll
+        for (int q = 0; q < kQ; ++q) {
+            const int g = g0 + q * kMassWarps;
+            const int e0 = min(g * a.SU, c.NU), e1 = min(e0 + a.SU, c.NU);
+            const int lu = e0 + r0 + lane;
+            in[q] = g < a.G && lu < e1;
+            count[q] = 0;
+            first[q] = 0;
+            if (in[q]) load_unit<ESIZE>(c, lu, want_draft, t[q], d[q], first[q], count[q]);
         }
-        if (lane == 0) { tb[g] = s0; tb[a.G + g] = s1; }
+#pragma unroll
+        for (int q = 0; q < kQ; ++q) {
+            float2 w = make_float2(0.f, 0.f);
+            if (in[q]) w = unit_weights<ESIZE>(c, t[q], d[q], first[q], count[q]);
+            s0[q] += warp_sum(w.x);
+            s1[q] += warp_sum(w.y);
+        }
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int q = 0; q < kQ; ++q) {
+            const int gg = warp + q * kMassWarps, g = g0 + q * kMassWarps;
+            s0v[gg] = s0[q];
+            s1v[gg] = s1[q];
+            if (g < a.G) { tb[g] = s0[q]; tb[a.G + g] = s1[q]; }
+        }
     }
     __syncthreads();
+    float *pt = a.part + static_cast<long long>(b) * 2 * a.P;
     if (tid == 0) {
+        float q0 = 0.f, q1 = 0.f;
+        for (int gg = 0; gg < kSegPerPart; ++gg) { q0 += s0v[gg]; q1 += s1v[gg]; }
+        pt[p] = q0;
+        pt[a.P + p] = q1;
+        __threadfence();
+        is_last = atomicAdd(&a.cnt[b], 1) == a.P - 1;
+    }
+    __syncthreads();
+    if (is_last && tid == 0) {
+        __threadfence();
         float W0 = 0.f, W1 = 0.f;
-        for (int g = 0; g < a.G; ++g) { W0 += tb[g]; W1 += tb[a.G + g]; }
+        for (int q = 0; q < a.P; ++q) { W0 += __ldcg(&pt[q]); W1 += __ldcg(&pt[a.P + q]); }
         a.mass_local[b] = make_float2(W0, W1);
     }
 }
@@ -475,66 +558,93 @@ __global__ void __launch_bounds__(32) vp_draw_kernel(Args a) {
     griddep_wait();
     griddep_launch_dependents();
     const int lane = threadIdx.x, b = blockIdx.x;
+    // Everything that depends only on the row is loaded at once: the record,
+    // this row's slice masses of every rank (32 at a time) and this rank's
+    // part sums of both tables.  The scans below run in the order the totals
+    // were formed, every lane in step, values passed by shuffles.
+    const float *pt = a.part + static_cast<long long>(b) * 2 * a.P;
+    const float pw0 = lane < a.P ? pt[lane] : 0.f;
+    const float pw1 = lane < a.P ? pt[a.P + lane] : 0.f;
+    float2 mw = make_float2(0.f, 0.f);
+    if (lane < a.nshards) mw = a.mass_all[static_cast<long long>(lane) * a.B + b];
     const Record r = a.rec[b];
     if (r.mode == kModeDone) return;
-    int owner = 0, table = 0, note = 0;
-    float tl = 0.f;
-    if (lane == 0) {
-        float R = 0.f;
-        for (int q = 0; q < a.nshards; ++q) R += a.mass_all[static_cast<long long>(q) * a.B + b].x;
-        if (!(R > 0.f)) {
-            // A rejection that left no residual mass: draw from p_j.
-            if (r.mode != kModeP) note |= SV_NOTE_ZERO_RESIDUAL;
-            table = 1;
-            R = 0.f;
-            for (int q = 0; q < a.nshards; ++q)
-                R += a.mass_all[static_cast<long long>(q) * a.B + b].y;
+    int table = 0, note = 0;
+    float R = 0.f;
+    for (int q0 = 0; q0 < a.nshards; q0 += 32) {
+        const float2 m = (q0 == 0) ? mw
+                         : (q0 + lane < a.nshards
+                                ? a.mass_all[static_cast<long long>(q0 + lane) * a.B + b]
+                                : make_float2(0.f, 0.f));
+        for (int q = 0; q < 32 && q0 + q < a.nshards; ++q) R += __shfl_sync(0xffffffffu, m.x, q);
+    }
+    if (!(R > 0.f)) {
+        // A rejection that left no residual mass: draw from p_j.
+        if (r.mode != kModeP) note |= SV_NOTE_ZERO_RESIDUAL;
+        table = 1;
+        R = 0.f;
+        for (int q0 = 0; q0 < a.nshards; q0 += 32) {
+            const float2 m = (q0 == 0) ? mw
+                             : (q0 + lane < a.nshards
+                                    ? a.mass_all[static_cast<long long>(q0 + lane) * a.B + b]
+                                    : make_float2(0.f, 0.f));
+            for (int q = 0; q < 32 && q0 + q < a.nshards; ++q)
+                R += __shfl_sync(0xffffffffu, m.y, q);
         }
-        const float t = r.u * R;
-        float cum = 0.f;
-        owner = -1;
-        int last = 0;
-        for (int q = 0; q < a.nshards; ++q) {
-            const float2 mq = a.mass_all[static_cast<long long>(q) * a.B + b];
-            const float w = table ? mq.y : mq.x;
-            if (w > 0.f) last = q;
-            if (owner < 0 && cum + w > t) { owner = q; tl = t - cum; }
+    }
+    const float tgt = r.u * R;
+    float cum = 0.f, tl = 0.f;
+    int owner = -1, last = 0;
+    for (int q0 = 0; q0 < a.nshards; q0 += 32) {
+        const float2 m = (q0 == 0) ? mw
+                         : (q0 + lane < a.nshards
+                                ? a.mass_all[static_cast<long long>(q0 + lane) * a.B + b]
+                                : make_float2(0.f, 0.f));
+        for (int q = 0; q < 32 && q0 + q < a.nshards; ++q) {
+            const float w = __shfl_sync(0xffffffffu, table ? m.y : m.x, q);
+            if (w > 0.f) last = q0 + q;
+            if (owner < 0 && cum + w > tgt) { owner = q0 + q; tl = tgt - cum; }
             if (owner < 0) cum += w;
         }
-        if (owner < 0) {
-            // Rounding left the target at or past the total: the last slice
-            // with positive weight, and inside it the last positive element.
-            owner = last;
-            tl = __int_as_float(0x7f800000);   // +inf: falls through every scan
-            note |= SV_NOTE_CDF_FALLBACK;
-        }
-        if (note && a.status) atomicOr(a.status, note);
     }
-    owner = __shfl_sync(0xffffffffu, owner, 0);
+    if (owner < 0) {
+        // Rounding left the target at or past the total: the last slice with
+        // positive weight, and inside it the last positive element.
+        owner = last;
+        tl = __int_as_float(0x7f800000);   // +inf: falls through every scan
+        note |= SV_NOTE_CDF_FALLBACK;
+    }
+    if (lane == 0 && note && a.status) atomicOr(a.status, note);
     if (owner != a.shard) return;
-    table = __shfl_sync(0xffffffffu, table, 0);
-    tl = __shfl_sync(0xffffffffu, tl, 0);
 
-    // Segment: sequential scan of the table in the order its total was formed.
+    // Part, then segment inside it.
     const float *tb = a.seg + static_cast<long long>(b) * 2 * a.G + (table ? a.G : 0);
-    int gsel = 0;
-    float tg = 0.f;
+    const float pw = table ? pw1 : pw0;
+    float tp = 0.f;
+    int psel = -1;
     bool fb = false;
-    if (lane == 0) {
-        float cum = 0.f;
-        int last = 0;
-        gsel = -1;
-        for (int g = 0; g < a.G; ++g) {
-            const float w = tb[g];
-            if (w > 0.f) last = g;
-            if (gsel < 0 && cum + w > tl) { gsel = g; tg = tl - cum; }
-            if (gsel < 0) cum += w;
-        }
-        if (gsel < 0) { gsel = last; fb = true; }
+    cum = 0.f;
+    last = 0;
+    for (int q = 0; q < a.P; ++q) {
+        const float w = __shfl_sync(0xffffffffu, pw, q);
+        if (w > 0.f) last = q;
+        if (psel < 0 && cum + w > tl) { psel = q; tp = tl - cum; }
+        if (psel < 0) cum += w;
     }
-    gsel = __shfl_sync(0xffffffffu, gsel, 0);
-    tg = __shfl_sync(0xffffffffu, tg, 0);
-    fb = __shfl_sync(0xffffffffu, fb ? 1 : 0, 0) != 0;
+    if (psel < 0) { psel = last; fb = true; tp = __int_as_float(0x7f800000); }
+    const int g0 = psel * kSegPerPart, g1 = min(g0 + kSegPerPart, a.G);
+    const float sw = g0 + lane < g1 ? tb[g0 + lane] : 0.f;
+    int gsel = -1;
+    float tg = 0.f;
+    cum = 0.f;
+    last = g0;
+    for (int g = g0; g < g1; ++g) {
+        const float w = __shfl_sync(0xffffffffu, sw, g - g0);
+        if (w > 0.f) last = g;
+        if (gsel < 0 && cum + w > tp) { gsel = g; tg = tp - cum; }
+        if (gsel < 0) cum += w;
+    }
+    if (gsel < 0) { gsel = last; fb = true; }
 
     // Inside the segment: rounds of 32 units, running sum of the round warp
     // sums exactly as the segment total was formed; the lane whose inclusive
@@ -603,8 +713,8 @@ __global__ void __launch_bounds__(32) vp_draw_kernel(Args a) {
 // Host side.
 // ---------------------------------------------------------------------------
 struct Plan {
-    int es, S, C, SU, G;
-    size_t stats_bytes, off_seg, ws_bytes;
+    int es, S, C, SU, G, P;
+    size_t stats_bytes, off_seg, off_part, off_cnt, ws_bytes;
 };
 
 static bool make_plan(const sv_vp_slice *s, Plan *p) {
@@ -626,10 +736,13 @@ static bool make_plan(const sv_vp_slice *s, Plan *p) {
     const long long per = (nu + kMaxSeg - 1) / kMaxSeg;
     p->SU = static_cast<int>((per + 31) / 32 * 32);
     p->G = static_cast<int>((nu + p->SU - 1) / p->SU);
+    p->P = (p->G + kSegPerPart - 1) / kSegPerPart;
     p->stats_bytes = sizeof(float4) * static_cast<size_t>(blocks);
-    const size_t rec = sizeof(Record) * static_cast<size_t>(s->B);
-    p->off_seg = (rec + 15) & ~static_cast<size_t>(15);
-    p->ws_bytes = p->off_seg + sizeof(float) * 2 * static_cast<size_t>(p->G) * s->B;
+    auto align16 = [](size_t o) { return (o + 15) & ~static_cast<size_t>(15); };
+    p->off_seg = align16(sizeof(Record) * static_cast<size_t>(s->B));
+    p->off_part = align16(p->off_seg + sizeof(float) * 2 * static_cast<size_t>(p->G) * s->B);
+    p->off_cnt = align16(p->off_part + sizeof(float) * 2 * static_cast<size_t>(p->P) * s->B);
+    p->ws_bytes = align16(p->off_cnt + sizeof(int) * static_cast<size_t>(s->B));
     return true;
 }
 
@@ -649,7 +762,7 @@ static Args base_args(const sv_vp_slice *s, const Plan &p) {
     a.zd = static_cast<const char *>(s->draft_logits);
     a.B = s->B; a.K = s->K; a.V = s->V; a.v0 = s->v0; a.Vs = s->Vs;
     a.S = p.S; a.C = p.C; a.nshards = s->nshards; a.shard = s->shard;
-    a.SU = p.SU; a.G = p.G;
+    a.SU = p.SU; a.G = p.G; a.P = p.P;
     return a;
 }
 
@@ -722,12 +835,20 @@ extern "C" sv_status sv_vp_decide(const sv_vp_slice *s, const void *stats_all,
     char *w = static_cast<char *>(workspace);
     a.rec = reinterpret_cast<sv::vp::Record *>(w);
     a.seg = reinterpret_cast<float *>(w + p.off_seg);
+    a.part = reinterpret_cast<float *>(w + p.off_part);
+    a.cnt = reinterpret_cast<int *>(w + p.off_cnt);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const cudaError_t e =
+    cudaError_t e =
         p.es == 4 ? sv::launch_pdl(sv::vp::vp_decide_kernel<4>, dim3(s->B),
                                    dim3(sv::vp::kDecideThreads), 0, st, a)
                   : sv::launch_pdl(sv::vp::vp_decide_kernel<2>, dim3(s->B),
                                    dim3(sv::vp::kDecideThreads), 0, st, a);
+    if (e != cudaSuccess) return sv::note_cuda(e);
+    const unsigned mgrid = static_cast<unsigned>(s->B) * static_cast<unsigned>(p.P);
+    e = p.es == 4 ? sv::launch_pdl(sv::vp::vp_mass_kernel<4>, dim3(mgrid),
+                                   dim3(sv::vp::kMassThreads), 0, st, a)
+                  : sv::launch_pdl(sv::vp::vp_mass_kernel<2>, dim3(mgrid),
+                                   dim3(sv::vp::kMassThreads), 0, st, a);
     if (e != cudaSuccess) return sv::note_cuda(e);
     return sv::note_cuda(cudaGetLastError());
 }
@@ -748,6 +869,8 @@ extern "C" sv_status sv_vp_draw(const sv_vp_slice *s, const float *mass_all, int
     char *w = static_cast<char *>(workspace);
     a.rec = reinterpret_cast<sv::vp::Record *>(w);
     a.seg = reinterpret_cast<float *>(w + p.off_seg);
+    a.part = reinterpret_cast<float *>(w + p.off_part);
+    a.cnt = reinterpret_cast<int *>(w + p.off_cnt);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const cudaError_t e =
         p.es == 4 ? sv::launch_pdl(sv::vp::vp_draw_kernel<4>, dim3(s->B), dim3(32), 0, st, a)
