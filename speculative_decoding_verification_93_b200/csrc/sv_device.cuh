@@ -169,6 +169,14 @@ __device__ __forceinline__ float unit_elem(const uint4 &u, int e) {
     return (e & 1) ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]);
 }
 
+// Element pair q (elements 2q, 2q+1) of a packed unit, widened to fp32.
+template <int ESIZE>
+__device__ __forceinline__ float2 unit_pair(const uint4 &u, int q) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    if (ESIZE == 2) return make_float2(bf16_lo(w[q]), bf16_hi(w[q]));
+    return make_float2(__uint_as_float(w[2 * q]), __uint_as_float(w[2 * q + 1]));
+}
+
 // Online (max, sum) update with a batch of units.  The batch max is a
 // balanced tree of packed bf16x2 (or f32) max operations; the running sum is
 // rescaled once if the max grew; then one exp2 per element with the

@@ -89,6 +89,7 @@ struct VerifyArgs {
     int *lvl_row;              // [K+1, B+1] per-level exclusive prefix of row item counts
     float4 *part;              // [B, S, C]: (m, s, argmax bits, 0)
     float *rtbl;               // [B, nsub] residual mass per sub-range
+    float *ctot;               // [B, C] residual mass per chunk (its sub-ranges, in scan order)
     int nsub;                  // sub-ranges per row
     int *work;                 // [B * C] (row * C + chunk) of the resample CTAs with work
     struct DrawRecord *rec;    // [B] accept result and draw set-up
@@ -737,14 +738,6 @@ __device__ __forceinline__ float elem_weight(const DrawCtx &c, const UnitData &u
     return fmaxf(p - q, 0.f);
 }
 
-// Element pair q (elements 2q, 2q+1) of a packed unit, widened to fp32.
-template <int ESIZE>
-__device__ __forceinline__ float2 unit_pair(const uint4 &u, int q) {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-    if (ESIZE == 2) return make_float2(bf16_lo(w[q]), bf16_hi(w[q]));
-    return make_float2(__uint_as_float(w[2 * q]), __uint_as_float(w[2 * q + 1]));
-}
-
 // Sum of the draw weights of a unit.  Full body units take a packed path:
 // per element pair, (z - m) by one packed add, (z - m) k - c by one packed
 // FMA, two exp2, and for the residual the same for q, a packed p - q, and
@@ -1040,6 +1033,7 @@ __device__ __forceinline__ void chunk_masses(const VerifyArgs &a, int b, int j, 
 constexpr int kSubUnits = 64;   // units per sub-range; chunk sizes are multiples of it
 constexpr int kRunUnits = 3;    // local units per lane in a located sub-range (66 / 32)
 constexpr int kResidParts = 1;  // resample CTAs per chunk of a residual draw
+static_assert(kResidParts == 1, "each chunk CTA forms its chunk's residual total");
 
 // Draw weight of `count` (< one unit) elements from element `first`,
 // loaded directly (vector head or tail).
@@ -1126,54 +1120,51 @@ __device__ void residual_subranges(const DrawCtx &c, int ch, int part, int U, fl
     }
 }
 
-// Inverse CDF over the sub-range table (one warp): the total R (rounds of
-// 32 entries, a fixed tree per round, rounds in order), then the first
-// entry with positive weight whose running sum exceeds t = u R.  *sel = -1
-// with *zero set when R is 0; if rounding leaves t at or past the end, the
-// last entry with weight is returned with *fb set and an infinite target.
-__device__ void scan_table(const float *tb, int nsub, float u, int *sel_out, float *d_out,
-                           bool *zero, bool *fb) {
+// Sum of n table entries by one warp: rounds of 32 entries in order, a
+// fixed tree inside each round.  table_find walks the entries in the same
+// rounds, so a target below this total always finds its entry.
+__device__ float table_total(const float *tb, int n) {
     constexpr int kRounds = 8;
     const int lane = threadIdx.x & 31;
     float R = 0.f;
-    int lastpos = -1;
     float v[kRounds];
-    for (int base = 0; base < nsub; base += 32 * kRounds) {
+    for (int base = 0; base < n; base += 32 * kRounds) {
 #pragma unroll
         for (int q = 0; q < kRounds; ++q) {
             const int s = base + q * 32 + lane;
-            v[q] = s < nsub ? __ldcg(tb + s) : 0.f;
+            v[q] = s < n ? __ldcg(tb + s) : 0.f;
         }
 #pragma unroll
         for (int q = 0; q < kRounds; ++q) {
-            if (v[q] > 0.f) lastpos = base + q * 32 + lane;
             float r = v[q];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
             R += r;
         }
     }
-    *sel_out = -1;
-    *d_out = 0.f;
-    if (!(R > 0.f)) {
-        *zero = true;
-        return;
-    }
-    const float t = u * R;
-    int sel = -1;
+    return R;
+}
+
+// First entry with positive weight whose running sum exceeds t (one warp);
+// *d_out is t minus the sum before it.  If rounding leaves t at or past the
+// end, the last entry with weight is returned with *fb set and an infinite
+// target.
+__device__ int table_find(const float *tb, int n, float t, float *d_out, bool *fb) {
+    constexpr int kRounds = 8;
+    const int lane = threadIdx.x & 31;
+    int sel = -1, lastpos = -1;
     float dsel = 0.f, cum = 0.f;
-    const bool resident = nsub <= 32 * kRounds;   // pass 1 left the whole table in v
-    for (int base = 0; base < nsub && sel < 0; base += 32 * kRounds) {
-        if (!resident) {
+    float v[kRounds];
+    for (int base = 0; base < n && sel < 0; base += 32 * kRounds) {
 #pragma unroll
-            for (int q = 0; q < kRounds; ++q) {
-                const int s = base + q * 32 + lane;
-                v[q] = s < nsub ? __ldcg(tb + s) : 0.f;
-            }
+        for (int q = 0; q < kRounds; ++q) {
+            const int s = base + q * 32 + lane;
+            v[q] = s < n ? __ldcg(tb + s) : 0.f;
         }
 #pragma unroll
         for (int q = 0; q < kRounds; ++q) {
             if (sel >= 0) break;
+            if (v[q] > 0.f) lastpos = base + q * 32 + lane;
             float incl = v[q];
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -1198,8 +1189,17 @@ __device__ void scan_table(const float *tb, int nsub, float u, int *sel_out, flo
         dsel = __int_as_float(0x7f800000);
         *fb = true;
     }
-    *sel_out = sel;
     *d_out = dsel;
+    return sel;
+}
+
+// Sub-ranges [*s0, *s1) of chunk ch (the head joins sub-range 0 of chunk 0,
+// the tail the last sub-range).
+__device__ __forceinline__ void chunk_subranges(const VecGeom &g, int ch, int U, int *s0, int *s1) {
+    const int u0 = min(ch * U, g.n16), u1 = min((ch + 1) * U, g.n16);
+    *s0 = u0 / kSubUnits;
+    *s1 = (u1 + kSubUnits - 1) / kSubUnits;
+    if (g.n16 == 0 && ch == 0) *s1 = 1;   // head and tail only
 }
 
 // Smallest element of the sub-range described by c (ubody0, nbody, head,
@@ -1469,8 +1469,16 @@ __global__ void __launch_bounds__(kDrawThreads, 3) resample_kernel(VerifyArgs a)
         // row's table and the token inside it.
         set_chunk(chunk);
         float *tb = a.rtbl + static_cast<long long>(b) * a.nsub;
+        float *ct = a.ctot + static_cast<long long>(b) * C;
         residual_subranges<ESIZE>(c, chunk, part, a.U, tb);
         __syncthreads();
+        if (warp == 0) {
+            // This chunk's total, formed as the last CTA's scan will walk it.
+            int s0, s1;
+            chunk_subranges(c.gt, chunk, a.U, &s0, &s1);
+            const float tot = table_total(tb + s0, s1 - s0);
+            if (lane == 0) ct[chunk] = tot;
+        }
         if (tid == 0) {
             __threadfence();
             const int done = atomicAdd(&a.rcnt[b], 1) + 1;
@@ -1480,11 +1488,32 @@ __global__ void __launch_bounds__(kDrawThreads, 3) resample_kernel(VerifyArgs a)
         __syncthreads();
         if (!ds.last) return;
         if (warp == 0) {
+            // Chunk totals in order, then the sub-ranges of the chosen chunk.
             bool zero = false, fbw = false;
             const int nsub = max(1, (c.gt.n16 + kSubUnits - 1) / kSubUnits);
-            int sel;
-            float dsel;
-            scan_table(tb, nsub, r.u, &sel, &dsel, &zero, &fbw);
+            const float w0 = lane < C ? __ldcg(ct + lane) : 0.f;
+            const float w1 = lane + 32 < C ? __ldcg(ct + lane + 32) : 0.f;
+            float R = 0.f;
+            for (int q = 0; q < C; ++q) R += __shfl_sync(0xffffffffu, q < 32 ? w0 : w1, q & 31);
+            int sel = -1;
+            float dsel = 0.f;
+            if (!(R > 0.f)) {
+                zero = true;
+            } else {
+                const float t = r.u * R;
+                float cum = 0.f, tc = 0.f;
+                int cs = -1, clast = 0;
+                for (int q = 0; q < C; ++q) {
+                    const float w = __shfl_sync(0xffffffffu, q < 32 ? w0 : w1, q & 31);
+                    if (w > 0.f) clast = q;
+                    if (cs < 0 && cum + w > t) { cs = q; tc = t - cum; }
+                    if (cs < 0) cum += w;
+                }
+                if (cs < 0) { cs = clast; tc = __int_as_float(0x7f800000); fbw = true; }
+                int s0, s1;
+                chunk_subranges(c.gt, cs, a.U, &s0, &s1);
+                sel = s0 + table_find(tb + s0, s1 - s0, tc, &dsel, &fbw);
+            }
             int yw = -1;
             if (!zero && sel >= 0) {
                 DrawCtx cs = c;
@@ -1550,7 +1579,7 @@ template <int ESIZE> static const void *stream_kernel_ptr() {
 struct Plan {
     int C, U, S;
     int nsub;
-    size_t off_rcnt, off_leff, off_rowj, off_pcnt, off_lvloff, off_lvlrow, off_part, off_rtbl,
+    size_t off_rcnt, off_leff, off_rowj, off_pcnt, off_lvloff, off_lvlrow, off_part, off_rtbl, off_ctot,
         off_work,
         off_rec, bytes;
 };
@@ -1583,6 +1612,7 @@ static bool make_plan(int B, int K, int V, sv_dtype dtype, Plan *p) {
     p->nsub = static_cast<int>((n16 + kSubUnits - 1) / kSubUnits);
     if (p->nsub < 1) p->nsub = 1;
     p->off_rtbl = off;   off = align16(off + sizeof(float) * static_cast<size_t>(B) * p->nsub);
+    p->off_ctot = off;   off = align16(off + sizeof(float) * static_cast<size_t>(B) * C);
     p->off_work = off;   off = align16(off + sizeof(int) * static_cast<size_t>(B) * C * kResidParts);
     p->off_rec = off;    off = align16(off + sizeof(DrawRecord) * static_cast<size_t>(B));
     p->bytes = off;
@@ -1644,6 +1674,7 @@ static sv_status verify_impl(const void *zt, const void *zd, sv_dtype dtype, int
     a.lvl_row = reinterpret_cast<int *>(w + p.off_lvlrow);
     a.part = reinterpret_cast<float4 *>(w + p.off_part);
     a.rtbl = reinterpret_cast<float *>(w + p.off_rtbl);
+    a.ctot = reinterpret_cast<float *>(w + p.off_ctot);
     a.nsub = p.nsub;
     a.work = reinterpret_cast<int *>(w + p.off_work);
     a.rec = reinterpret_cast<DrawRecord *>(w + p.off_rec);

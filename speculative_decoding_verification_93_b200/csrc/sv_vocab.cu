@@ -271,11 +271,45 @@ __device__ __forceinline__ float elem_weight(const DrawCtx &c, int table, const 
     return table ? w.y : w.x;
 }
 
-// Both tables' weight of a unit, each summed in element order.
+// Both tables' weight of a unit.  A full body unit (not holding a
+// one-hot x_j, draft in phase) takes a packed path: per element pair one
+// packed add and one packed multiply form (z - m) k, then two exp2, and for
+// the residual the same for q, a packed multiply by 1/Sigma, a packed FMA
+// and the clamp; the element values equal elem_weights', summed in two
+// interleaved chains.  Other units sum elem_weights in element order.  The
+// mass and draw kernels both call this, so a unit weighs the same in both.
 template <int ESIZE>
 __device__ __forceinline__ float2 unit_weights(const DrawCtx &c, const uint4 &t, const uint4 &d,
                                                int first, int count) {
     constexpr int kPer = 16 / ESIZE;
+    const bool fast = count == kPer && (c.mode != kModeResidual || c.aligned) &&
+                      (c.mode != kModeOneHot || c.xl < first || c.xl >= first + kPer);
+    if (fast) {
+        const float2 kk = make_float2(c.k, c.k), nmt = make_float2(-c.mt, -c.mt);
+        float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+        if (c.mode == kModeResidual) {
+            const float2 nmd = make_float2(-c.md, -c.md);
+            const float2 ist = make_float2(c.ist, c.ist), isd = make_float2(c.isd, c.isd);
+#pragma unroll
+            for (int q = 0; q < kPer / 2; ++q) {
+                const float2 x = __fmul2_rn(__fadd2_rn(unit_pair<ESIZE>(t, q), nmt), kk);
+                const float2 pu = make_float2(ex2(x.x), ex2(x.y));
+                const float2 y = __fmul2_rn(__fadd2_rn(unit_pair<ESIZE>(d, q), nmd), kk);
+                const float2 qn = __fmul2_rn(make_float2(ex2(y.x), ex2(y.y)), isd);
+                const float2 r = __ffma2_rn(pu, ist, make_float2(-qn.x, -qn.y));
+                a0 = __fadd2_rn(a0, make_float2(fmaxf(r.x, 0.f), fmaxf(r.y, 0.f)));
+                a1 = __fadd2_rn(a1, pu);
+            }
+            return make_float2(a0.x + a0.y, a1.x + a1.y);
+        }
+#pragma unroll
+        for (int q = 0; q < kPer / 2; ++q) {
+            const float2 x = __fmul2_rn(__fadd2_rn(unit_pair<ESIZE>(t, q), nmt), kk);
+            a1 = __fadd2_rn(a1, make_float2(ex2(x.x), ex2(x.y)));
+        }
+        const float s1 = a1.x + a1.y;
+        return make_float2(s1, s1);
+    }
     float w0 = 0.f, w1 = 0.f;
 #pragma unroll
     for (int e = 0; e < kPer; ++e) {
