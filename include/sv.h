@@ -3,8 +3,10 @@
  *
  * The library implements the data-parallel hot path of confidence-scheduled
  * speculative decoding: the per-row verify length from the drafter's
- * survival confidences (sv_schedule) and batched draft verification by
- * speculative rejection sampling (sv_verify).
+ * survival confidences (sv_schedule, sv_schedule_admit), batched draft
+ * verification by speculative rejection sampling (sv_verify), the same
+ * verification with the vocabulary split across ranks (sv_vp_*), and the
+ * confidence head's per-position temperature (sv_sts_*).
  *
  * Conventions for every entry point:
  *  - Pointers named as device pointers must be CUDA device memory (or

@@ -218,3 +218,32 @@ def test_c2_full_split(nshards):
     res = compare(g, o, extra_excluded=sched_tie)
     assert g["status"] & ~(sv.SV_NOTE_CDF_FALLBACK | sv.SV_NOTE_ZERO_RESIDUAL) == 0
     assert res["tie_mismatches"] <= max(2, res["rows"] // 50), res
+
+
+@pytest.mark.parametrize("V,dtype,K,B,nshards", [
+    (1000, torch.float32, 4, 16, 40),      # more ranks than a warp holds: masses read 32 at a time
+    (2003, torch.bfloat16, 3, 16, 77),
+    (3000, torch.bfloat16, 40, 12, 3),     # accept tests in two rounds of 32 positions
+    (513, torch.float32, 64, 8, 5),        # the largest K
+])
+def test_many_ranks_and_long_blocks(V, dtype, K, B, nshards):
+    b = _cuda(workloads.random_small(B, K, V, dtype=dtype, seed=V + K, noise=0.05,
+                                     temps=(0.0, 0.8, 1.0)))
+    total = dict(rows=0, tie_mismatches=0)
+    longest = 0
+    for seed in (1, 2):
+        for zd in (b.zd, None):
+            g = vp_emulated(b.zt, zd, b.tokens, b.lengths, b.temperature, seed, nshards)
+            ln = b.lengths.cpu().numpy()
+            o = oracle_verify(b.zt, zd, b.tokens, ln, b.temperature, seed)
+            check_structure(g, b.tokens.cpu().numpy(), ln)
+            r = compare(g, o)
+            total["rows"] += r["rows"]
+            total["tie_mismatches"] += r["tie_mismatches"]
+            if zd is not None:
+                longest = max(longest, int(g["accept"].max()))
+    assert total["tie_mismatches"] <= max(2, total["rows"] // 50)
+    # drafts close to the target (noise 0.05) keep long blocks alive, so the
+    # second round of accept tests (positions 32..) is exercised
+    if K > 32 and b.lengths.max().item() > 33:
+        assert longest > 32
