@@ -247,3 +247,26 @@ def test_many_ranks_and_long_blocks(V, dtype, K, B, nshards):
     # second round of accept tests (positions 32..) is exercised
     if K > 32 and b.lengths.max().item() > 33:
         assert longest > 32
+
+
+def test_verifier_class_single_rank():
+    """VocabParallelVerifier without a process group (one rank, collectives
+    skipped): the public orchestration path, reused across steps."""
+    from speculative_decoding_verification_93_b200.vocab_parallel import VocabParallelVerifier
+    b = _cuda(workloads.random_small(24, 5, 4099, dtype=torch.bfloat16, seed=21,
+                                     temps=(0.0, 0.7, 1.0)))
+    vpv = VocabParallelVerifier(24, 5, 4099, torch.bfloat16, "cuda")
+    assert (vpv.world, vpv.rank, vpv.v0, vpv.Vs) == (1, 0, 0, 4099)
+    ln = b.lengths.cpu().numpy()
+    for seed in (3, 4):
+        ot = torch.full((24, 6), -7, dtype=torch.int32, device="cuda")
+        oa = torch.full((24,), -7, dtype=torch.int32, device="cuda")
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        vpv.step(b.zt, b.zd, b.tokens, b.lengths, b.temperature, seed, ot, oa, status=st)
+        torch.cuda.synchronize()
+        g = dict(tokens=ot.cpu().numpy(), accept=oa.cpu().numpy(), status=int(st.item()))
+        o = oracle_verify(b.zt, b.zd, b.tokens, ln, b.temperature, seed)
+        check_structure(g, b.tokens.cpu().numpy(), ln)
+        compare(g, o)
+    with pytest.raises(ValueError):
+        vpv.slice_of(b.zt[:, :, :100].contiguous(), None)
