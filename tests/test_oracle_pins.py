@@ -225,3 +225,30 @@ def test_invalid_rows_are_marked_not_fatal():
     out, acc, _, st = oracle.verify(zt, zd, np.zeros((5, K), np.int32), np.full(5, 2, np.int32),
                                     T2, seed=1)
     assert st == 4 and list(acc[:3]) == [-1, -1, -1] and acc[3] >= 0 and acc[4] >= 0
+
+
+def test_verify_hand_worked_examples():
+    """Hand-worked steps of the rule (tests/golden/verify_worked.json) with
+    injected uniforms: accept/reject decisions, the residual and bonus
+    inverse CDF on both sides of a boundary, temperature, L = 0, the greedy
+    drafter and greedy ties."""
+    import json
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "verify_worked.json")
+    cases = json.load(open(path))["cases"]
+    for c in cases:
+        T = c["T"]
+        if "logits" in c:
+            zt = np.array(c["logits"], dtype=np.float64)
+            zd = np.array(c["draft_logits"], dtype=np.float64)
+        else:
+            zt = T * np.log(np.array(c["p"], dtype=np.float64))
+            zd = None if c.get("greedy_drafter") else T * np.log(np.array(c["q"], dtype=np.float64))
+        K = zt.shape[0] - 1
+        ua = np.zeros(K + 1)
+        ur = np.zeros(K + 1)
+        ua[:len(c["u_acc"])] = c["u_acc"]
+        ur[:len(c["u_res"])] = c["u_res"]
+        a, out, _ = oracle.verify_row_u(zt, zd, np.array(c["x"]), c["L"], T, ua, ur)
+        assert a == c["accept"], c["name"]
+        assert out.tolist() == c["tokens"], (c["name"], out.tolist())
