@@ -434,6 +434,50 @@ sv_status sv_vp_draw(const sv_vp_slice *slice, const float *mass_all, int32_t *o
                      void *workspace, size_t workspace_bytes, int32_t *status, void *stream);
 
 /*
+ * sv_verify_host -- schedule and verify a batch whose inputs live in host
+ * memory, moving only the logits the method reads across the host link.
+ *
+ * Verification reads, per row, the target positions 0..L and the draft
+ * positions 0..L-1 that the schedule keeps and nothing past them (umans.ai
+ * page, section "What DSpark adds", item "2. Verify smarter": only the
+ * confident prefix is verified).  This call copies the confidences, tokens
+ * and temperatures in, runs sv_schedule with threshold `load`, copies the
+ * lengths out and waits for them (its one synchronisation of `stream`),
+ * then copies only each row's scheduled runs of both logit arrays (one
+ * cudaMemcpyAsync per contiguous run, adjacent runs merged), runs
+ * sv_verify, and copies out_tokens, out_accept_len and status back.  The
+ * results equal sv_schedule followed by sv_verify on device copies of the
+ * same inputs.
+ *
+ *   target_logits, draft_logits  HOST [B, K+1, V] and [B, K, V] of dtype
+ *                  (draft NULL: greedy drafter); pinned memory lets the copies
+ *                  run asynchronously.
+ *   conf           HOST float32 [B, K], and load: the schedule threshold tau.
+ *                  conf NULL: no schedule and no synchronisation; `lengths`
+ *                  is then a HOST input (e.g. lengths fixed by the caller).
+ *   draft_tokens   HOST int32 [B, K]; temperature: HOST float32 [B].
+ *   out_tokens, out_accept_len   HOST, written once `stream` has drained.
+ *   lengths        HOST int32 [B]: written (by the time the call returns)
+ *                  when conf is given, read when conf is NULL.
+ *   status         HOST int32, nullable: the SV_ROW_* / SV_NOTE_* bits of
+ *                  this call (written once `stream` has drained).
+ *   workspace      DEVICE, >= sv_verify_host_workspace_bytes(), 256-byte
+ *                  aligned: device copies of both logit arrays (only the
+ *                  scheduled runs are written), the small arrays and the
+ *                  sv_verify workspace.
+ *   h2d_bytes      nullable: bytes copied host-to-device by this call.
+ * Returns SV_OK, SV_ERR_ARG, SV_ERR_SHAPE, SV_ERR_DTYPE, SV_ERR_WORKSPACE or
+ * SV_ERR_CUDA.  Argument errors are returned before anything is enqueued.
+ */
+size_t sv_verify_host_workspace_bytes(int B, int K, int V, sv_dtype dtype);
+sv_status sv_verify_host(const void *target_logits, const void *draft_logits, sv_dtype dtype,
+                         int B, int K, int V, const float *conf, float load,
+                         const int32_t *draft_tokens, const float *temperature, uint64_t seed,
+                         int64_t row_base, int32_t *out_tokens, int32_t *out_accept_len,
+                         int32_t *lengths, int32_t *status, void *workspace,
+                         size_t workspace_bytes, size_t *h2d_bytes, void *stream);
+
+/*
  * sv_philox_uniforms -- the uniforms sv_verify draws, for tests:
  * out[k] = u(seed, row[k], pos[k], draw[k]) as defined above.
  * row: device int64 [n] (>= 0); pos, draw: device int32 [n]; out: device

@@ -67,6 +67,10 @@ def lib():
     L.sv_vp_stats.argtypes = [sp, vp, vp, vp, vp, vp]
     L.sv_vp_decide.argtypes = [sp, vp, vp, vp, vp, u64, i64, vp, vp, vp, vp, vp, sz, vp, vp]
     L.sv_vp_draw.argtypes = [sp, vp, vp, vp, sz, vp, vp]
+    L.sv_verify_host_workspace_bytes.argtypes = [i32, i32, i32, i32]
+    L.sv_verify_host_workspace_bytes.restype = sz
+    L.sv_verify_host.argtypes = [vp, vp, i32, i32, i32, i32, vp, ctypes.c_float, vp, vp, u64, i64,
+                                 vp, vp, vp, vp, vp, sz, vp, vp]
     L.sv_philox_uniforms.argtypes = [u64, vp, vp, vp, i32, vp, vp]
     L.sv_philox4x32_10.argtypes = [vp, vp, i32, vp, vp]
     L.sv_profile_begin.argtypes = [i32]
@@ -75,7 +79,8 @@ def lib():
     L.sv_status_string.argtypes = [i32]
     L.sv_status_string.restype = ctypes.c_char_p
     for name in ("sv_schedule", "sv_schedule_admit", "sv_sts_fit", "sv_sts_apply", "sv_verify",
-                 "sv_verify_debug", "sv_verify_noalloc", "sv_vp_stats", "sv_vp_decide",
+                 "sv_verify_debug", "sv_verify_noalloc", "sv_verify_host", "sv_vp_stats",
+                 "sv_vp_decide",
                  "sv_vp_draw",
                  "sv_philox_uniforms",
                  "sv_philox4x32_10", "sv_profile_begin"):
@@ -280,6 +285,52 @@ def sv_vp_draw(slice_: sv_vp_slice, mass_all, out_tokens, workspace, status=None
     _check("sv_vp_draw", lib().sv_vp_draw(
         ctypes.byref(slice_), _ptr(mass_all), _ptr(out_tokens), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream, out_tokens)))
+
+
+def sv_verify_host_workspace_bytes(B: int, K: int, V: int, dtype: int) -> int:
+    return int(lib().sv_verify_host_workspace_bytes(B, K, V, dtype))
+
+
+def _need_host(t: torch.Tensor, dtype, name: str):
+    if t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous {dtype} host tensor")
+
+
+def sv_verify_host(target_logits, draft_logits, conf, load: float, draft_tokens, temperature,
+                   seed: int, out_tokens, out_accept_len, lengths, workspace, status=None,
+                   row_base: int = 0, stream=None) -> int:
+    """Host-resident inputs and outputs (pinned CPU tensors), device
+    workspace; returns the bytes copied host-to-device.  With conf None,
+    `lengths` is an input and no schedule runs.  The outputs are valid once
+    `stream` has drained."""
+    B, K1, V = target_logits.shape
+    K = K1 - 1
+    if target_logits.is_cuda or not target_logits.is_contiguous():
+        raise TypeError("target_logits must be a contiguous host tensor")
+    dt = _dtype(target_logits)
+    if draft_logits is not None:
+        _need_host(draft_logits, target_logits.dtype, "draft_logits")
+        if tuple(draft_logits.shape) != (B, K, V):
+            raise TypeError("draft_logits must be [B, K, V]")
+    if conf is not None:
+        _need_host(conf, torch.float32, "conf")
+    _need_host(draft_tokens, torch.int32, "draft_tokens")
+    _need_host(temperature, torch.float32, "temperature")
+    _need_host(out_tokens, torch.int32, "out_tokens")
+    _need_host(out_accept_len, torch.int32, "out_accept_len")
+    _need_host(lengths, torch.int32, "lengths")
+    if status is not None:
+        _need_host(status, torch.int32, "status")
+    if not workspace.is_cuda:
+        raise TypeError("workspace must be device memory")
+    h2d = ctypes.c_size_t(0)
+    _check("sv_verify_host", lib().sv_verify_host(
+        _ptr(target_logits), _ptr(draft_logits), dt, B, K, V, _ptr(conf), float(load),
+        _ptr(draft_tokens), _ptr(temperature), ctypes.c_uint64(seed & (2**64 - 1)), int(row_base),
+        _ptr(out_tokens), _ptr(out_accept_len), _ptr(lengths), _ptr(status), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), ctypes.byref(h2d),
+        _stream(stream, workspace)))
+    return int(h2d.value)
 
 
 def sv_philox_uniforms(seed: int, row, pos, draw, out, stream=None) -> None:

@@ -15,7 +15,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsv.so")
 SOURCES = [os.path.join(CSRC, f) for f in ("sv_api.cu", "sv_verify.cu", "sv_admit.cu",
-                                           "sv_sts.cu", "sv_vocab.cu")]
+                                           "sv_sts.cu", "sv_vocab.cu", "sv_hostio.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("sv_device.cuh", "sv_host.h")] + \
     [os.path.join(INCLUDE, "sv.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

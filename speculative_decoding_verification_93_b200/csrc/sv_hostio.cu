@@ -1,0 +1,173 @@
+// sv_hostio.cu -- verification of host-resident inputs: only the scheduled
+// logit vectors cross the host link.
+//
+// Per row, verification reads the target positions 0..L and the draft
+// positions 0..L-1 that the confidence schedule keeps, and nothing past
+// them (umans.ai, "DeepSeek V4 Pro DSpark: the model isn't ready, the
+// architecture is", section "What DSpark adds", item "2. Verify smarter":
+// the confident prefix is what gets verified; aiweekly.co alert: the verify
+// length follows prefix survival and load).  So with the logits in host
+// memory the schedule runs first, its lengths come back (the one
+// synchronisation; a caller that already has the lengths passes them
+// instead), and only each row's scheduled runs are copied -- one
+// cudaMemcpyAsync per contiguous run, adjacent runs merged -- before the
+// device verification and the copy of its outputs back to the host.
+#include <cstdint>
+
+#include "sv.h"
+#include "sv_host.h"
+
+namespace sv {
+namespace hostio {
+
+struct Layout {
+    size_t zt, zd, conf, tok, temp, len, otok, oacc, status, ver, ver_bytes, bytes;
+};
+
+static size_t align256(size_t o) { return (o + 255) & ~static_cast<size_t>(255); }
+
+static bool make_layout(int B, int K, int V, sv_dtype dtype, Layout *L) {
+    const size_t ver = sv_verify_workspace_bytes(B, K, V, dtype);
+    if (ver == 0) return false;   // unsupported sizes or dtype
+    const size_t es = dtype == SV_F32 ? 4 : 2;
+    const size_t b = static_cast<size_t>(B), k = static_cast<size_t>(K), v = static_cast<size_t>(V);
+    size_t o = 0;
+    L->zt = o;     o = align256(o + b * (k + 1) * v * es);
+    L->zd = o;     o = align256(o + b * k * v * es);
+    L->conf = o;   o = align256(o + b * k * sizeof(float));
+    L->tok = o;    o = align256(o + b * k * sizeof(int32_t));
+    L->temp = o;   o = align256(o + b * sizeof(float));
+    L->len = o;    o = align256(o + b * sizeof(int32_t));
+    L->otok = o;   o = align256(o + b * (k + 1) * sizeof(int32_t));
+    L->oacc = o;   o = align256(o + b * sizeof(int32_t));
+    L->status = o; o = align256(o + sizeof(int32_t));
+    L->ver = o;    o = align256(o + ver);
+    L->ver_bytes = ver;
+    L->bytes = o;
+    return true;
+}
+
+// Host-to-device copies of contiguous byte runs, merging a run that starts
+// where the pending one ends.
+struct RunCopier {
+    const char *src = nullptr;
+    char *dst = nullptr;
+    size_t n = 0;
+    size_t total = 0;
+    cudaStream_t st;
+    cudaError_t err = cudaSuccess;
+    explicit RunCopier(cudaStream_t s) : st(s) {}
+    void add(const char *s, char *d, size_t bytes) {
+        if (bytes == 0) return;
+        if (n && s == src + n && d == dst + n) { n += bytes; return; }
+        flush();
+        src = s; dst = d; n = bytes;
+    }
+    void flush() {
+        if (n && err == cudaSuccess) err = cudaMemcpyAsync(dst, src, n, cudaMemcpyHostToDevice, st);
+        total += n;
+        n = 0;
+    }
+};
+
+}  // namespace hostio
+}  // namespace sv
+
+extern "C" size_t sv_verify_host_workspace_bytes(int B, int K, int V, sv_dtype dtype) {
+    sv::hostio::Layout L;
+    if (!sv::hostio::make_layout(B, K, V, dtype, &L)) return 0;
+    return L.bytes;
+}
+
+extern "C" sv_status sv_verify_host(const void *target_logits, const void *draft_logits,
+                                    sv_dtype dtype, int B, int K, int V, const float *conf,
+                                    float load, const int32_t *draft_tokens,
+                                    const float *temperature, uint64_t seed, int64_t row_base,
+                                    int32_t *out_tokens, int32_t *out_accept_len,
+                                    int32_t *lengths, int32_t *status, void *workspace,
+                                    size_t workspace_bytes, size_t *h2d_bytes, void *stream) {
+    using sv::hostio::Layout;
+    if (!target_logits || !draft_tokens || !temperature || !out_tokens ||
+        !out_accept_len || !lengths || !workspace)
+        return SV_ERR_ARG;
+    if (dtype != SV_F32 && dtype != SV_BF16) return SV_ERR_DTYPE;
+    Layout L;
+    if (!sv::hostio::make_layout(B, K, V, dtype, &L)) return SV_ERR_SHAPE;
+    if (row_base < 0 || (reinterpret_cast<uintptr_t>(workspace) & 255)) return SV_ERR_ARG;
+    if (workspace_bytes < L.bytes) return SV_ERR_WORKSPACE;
+    const size_t es = dtype == SV_F32 ? 4 : 2;
+    const size_t vb = static_cast<size_t>(V) * es;   // bytes per logit vector
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *w = static_cast<char *>(workspace);
+    float *conf_d = reinterpret_cast<float *>(w + L.conf);
+    int32_t *tok_d = reinterpret_cast<int32_t *>(w + L.tok);
+    float *temp_d = reinterpret_cast<float *>(w + L.temp);
+    int32_t *len_d = reinterpret_cast<int32_t *>(w + L.len);
+    int32_t *otok_d = reinterpret_cast<int32_t *>(w + L.otok);
+    int32_t *oacc_d = reinterpret_cast<int32_t *>(w + L.oacc);
+    int32_t *status_d = reinterpret_cast<int32_t *>(w + L.status);
+    const size_t nb = static_cast<size_t>(B);
+    const size_t nk = static_cast<size_t>(K);
+
+    // 1. Small inputs in; with confidences, schedule and bring the lengths
+    //    back (the one synchronisation), else take the caller's lengths.
+    cudaError_t e =
+        cudaMemcpyAsync(tok_d, draft_tokens, nb * nk * sizeof(int32_t), cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(temp_d, temperature, nb * sizeof(float), cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(status_d, 0, sizeof(int32_t), st);
+    sv_status s = SV_OK;
+    size_t small = nb * nk * sizeof(int32_t) + nb * sizeof(float);
+    if (conf) {
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(conf_d, conf, nb * nk * sizeof(float), cudaMemcpyHostToDevice, st);
+        if (e != cudaSuccess) return sv::note_cuda(e);
+        s = sv_schedule(conf_d, B, K, load, len_d, stream);
+        if (s != SV_OK) return s;
+        e = cudaMemcpyAsync(lengths, len_d, nb * sizeof(int32_t), cudaMemcpyDeviceToHost, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        small += nb * nk * sizeof(float);
+    } else if (e == cudaSuccess) {
+        e = cudaMemcpyAsync(len_d, lengths, nb * sizeof(int32_t), cudaMemcpyHostToDevice, st);
+        small += nb * sizeof(int32_t);
+    }
+    if (e != cudaSuccess) return sv::note_cuda(e);
+
+    // 2. The scheduled runs of every row: target positions 0..L, and draft
+    //    positions 0..L-1 of rows that sample with draft logits.
+    sv::hostio::RunCopier cp(st);
+    const char *zt_h = static_cast<const char *>(target_logits);
+    const char *zd_h = static_cast<const char *>(draft_logits);
+    char *zt_d = w + L.zt;
+    char *zd_d = w + L.zd;
+    for (int b = 0; b < B; ++b) {
+        const int Lb = lengths[b];
+        if (Lb < 0 || Lb > K) continue;   // verification marks the row invalid
+        const size_t off_t = static_cast<size_t>(b) * (nk + 1) * vb;
+        cp.add(zt_h + off_t, zt_d + off_t, static_cast<size_t>(Lb + 1) * vb);
+    }
+    cp.flush();
+    if (zd_h) {
+        for (int b = 0; b < B; ++b) {
+            const int Lb = lengths[b];
+            if (Lb < 1 || Lb > K || !(temperature[b] > 0.f)) continue;
+            const size_t off_d = static_cast<size_t>(b) * nk * vb;
+            cp.add(zd_h + off_d, zd_d + off_d, static_cast<size_t>(Lb) * vb);
+        }
+        cp.flush();
+    }
+    if (cp.err != cudaSuccess) return sv::note_cuda(cp.err);
+    if (h2d_bytes) *h2d_bytes = cp.total + small;
+
+    // 3. Verification on the device, outputs back to the host.
+    s = sv_verify(zt_d, zd_h ? zd_d : nullptr, dtype, B, K, V, tok_d, len_d, temp_d, seed,
+                  row_base, otok_d, oacc_d, w + L.ver, L.ver_bytes, status_d, stream);
+    if (s != SV_OK) return s;
+    e = cudaMemcpyAsync(out_tokens, otok_d, nb * (nk + 1) * sizeof(int32_t),
+                        cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(out_accept_len, oacc_d, nb * sizeof(int32_t), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess && status)
+        e = cudaMemcpyAsync(status, status_d, sizeof(int32_t), cudaMemcpyDeviceToHost, st);
+    return sv::note_cuda(e);
+}

@@ -164,3 +164,27 @@ def test_vocab_parallel_arguments_rejected_on_host():
     assert L.sv_vp_draw(R(ok), v((1 << 22) + 4), p, p, big, None, None) == 1
     assert L.sv_vp_draw(R(ok), None, p, p, big, None, None) == 1
     assert L.sv_vp_draw(R(sl(r=-1)), p, p, p, big, None, None) == 2
+
+
+def test_verify_host_arguments_rejected_on_host():
+    L = sv.lib()
+    v = ctypes.c_void_p
+    n = sv.sv_verify_host_workspace_bytes(4, 4, 1000, sv.SV_BF16)
+    assert n > 4 * 5 * 1000 * 2 + 4 * 4 * 1000 * 2
+    assert sv.sv_verify_host_workspace_bytes(4, 65, 1000, sv.SV_BF16) == 0
+    assert sv.sv_verify_host_workspace_bytes(4, 4, 1000, 9) == 0
+    p = v(1 << 20)
+    ws = v(1 << 24)
+
+    def call(zt=p, conf=p, tok=p, temp=p, ot=p, oa=p, ln=p, w=ws, wsb=1 << 40, dtype=sv.SV_BF16,
+             B=4, K=4, V=1000, row_base=0):
+        return L.sv_verify_host(zt, None, dtype, B, K, V, conf, ctypes.c_float(0.3), tok, temp,
+                                ctypes.c_uint64(0), row_base, ot, oa, ln, None, w, wsb, None,
+                                None)
+    for kw in ("zt", "tok", "temp", "ot", "oa", "ln", "w"):
+        assert call(**{kw: None}) == 1, kw
+    assert call(dtype=4) == 3
+    assert call(K=0) == 2 and call(B=0) == 2 and call(V=(1 << 20) + 1) == 2
+    assert call(row_base=-1) == 1
+    assert call(w=v((1 << 24) + 16)) == 1
+    assert call(wsb=n - 1) == 4
