@@ -396,8 +396,9 @@ def run_ours(args, rank, world, local_rank):
         del hlt, hat, hws
 
     # ---- end-to-end through host buffers: sv_verify_host takes the inputs in
-    # pinned host memory, schedules, copies only the scheduled logit runs to
-    # the device, verifies, and copies the outputs back -------------------------
+    # pinned host memory, schedules on the device, and copies to the device
+    # only the logits the outcome depends on, one position level at a time
+    # (rows leave once decided), then copies the outputs back ----------------
     e2e = None
     if not args.no_e2e:
         host = {n: getattr(batch, n).cpu().pin_memory() for n in
@@ -414,7 +415,7 @@ def run_ours(args, rank, world, local_rank):
             h2d_seen.append(sv.sv_verify_host(
                 host["zt"], host["zd"], host["conf"] if fixed is None else None, batch.tau,
                 host["tokens"], host["temperature"], args.seed + i, h_tok, h_acc, h_len, hws,
-                row_base=row_base))
+                row_base=row_base, levelwise=True))
 
         e2e_step(0)
         torch.cuda.synchronize()
@@ -431,11 +432,12 @@ def run_ours(args, rank, world, local_rank):
         full = sum(host[n].numel() * host[n].element_size() for n in ("zt", "zd"))
         e2e = {"value": positions * world / (ms_e2e / e2e_steps / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": int(max(h2d_seen[1:])), "d2h_bytes_per_step": int(d2h),
-               "steps": e2e_steps, "api": "sv_verify_host",
-               "note": "inputs in pinned host memory; the schedule's lengths come back "
-                       "(one synchronisation) and only the scheduled logit runs cross to the "
-                       f"device ({max(h2d_seen[1:]) / full:.2f} of the {full / 1e9:.2f} GB of "
-                       "logits)"}
+               "steps": e2e_steps, "api": "sv_verify_host (levelwise)",
+               "note": "inputs in pinned host memory; the schedule's lengths come back, then "
+                       "position level l of the rows still undecided is copied and verified "
+                       "(one synchronisation per level), so only the logits the outcome "
+                       f"depends on cross to the device ({max(h2d_seen[1:]) / full:.2f} of the "
+                       f"{full / 1e9:.2f} GB of logits)"}
         del host, hws
 
     # ---- roofline of the main kernel ----------------------------------------

@@ -461,6 +461,15 @@ sv_status sv_vp_draw(const sv_vp_slice *slice, const float *mass_all, int32_t *o
  *                  when conf is given, read when conf is NULL.
  *   status         HOST int32, nullable: the SV_ROW_* / SV_NOTE_* bits of
  *                  this call (written once `stream` has drained).
+ *   levelwise      0: copy every scheduled run at once (one synchronisation).
+ *                  1: copy only what the outcome depends on (target 0..a,
+ *                  draft 0..min(a, L-1), a = accepted length): level l copies
+ *                  position l of the rows still undecided and, from l = 1,
+ *                  verifies with lengths min(L, l); a row is final once it
+ *                  rejects below l or l reaches L.  Same results (the
+ *                  uniforms are keyed by row, position and draw), up to K
+ *                  synchronisations; SV_NOTE_* bits may also come from
+ *                  draws whose rows were still undecided.
  *   workspace      DEVICE, >= sv_verify_host_workspace_bytes(), 256-byte
  *                  aligned: device copies of both logit arrays (only the
  *                  scheduled runs are written), the small arrays and the
@@ -474,7 +483,7 @@ sv_status sv_verify_host(const void *target_logits, const void *draft_logits, sv
                          int B, int K, int V, const float *conf, float load,
                          const int32_t *draft_tokens, const float *temperature, uint64_t seed,
                          int64_t row_base, int32_t *out_tokens, int32_t *out_accept_len,
-                         int32_t *lengths, int32_t *status, void *workspace,
+                         int32_t *lengths, int32_t *status, int levelwise, void *workspace,
                          size_t workspace_bytes, size_t *h2d_bytes, void *stream);
 
 /*

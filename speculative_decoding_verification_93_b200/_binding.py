@@ -70,7 +70,7 @@ def lib():
     L.sv_verify_host_workspace_bytes.argtypes = [i32, i32, i32, i32]
     L.sv_verify_host_workspace_bytes.restype = sz
     L.sv_verify_host.argtypes = [vp, vp, i32, i32, i32, i32, vp, ctypes.c_float, vp, vp, u64, i64,
-                                 vp, vp, vp, vp, vp, sz, vp, vp]
+                                 vp, vp, vp, vp, i32, vp, sz, vp, vp]
     L.sv_philox_uniforms.argtypes = [u64, vp, vp, vp, i32, vp, vp]
     L.sv_philox4x32_10.argtypes = [vp, vp, i32, vp, vp]
     L.sv_profile_begin.argtypes = [i32]
@@ -298,11 +298,12 @@ def _need_host(t: torch.Tensor, dtype, name: str):
 
 def sv_verify_host(target_logits, draft_logits, conf, load: float, draft_tokens, temperature,
                    seed: int, out_tokens, out_accept_len, lengths, workspace, status=None,
-                   row_base: int = 0, stream=None) -> int:
+                   row_base: int = 0, levelwise: bool = False, stream=None) -> int:
     """Host-resident inputs and outputs (pinned CPU tensors), device
     workspace; returns the bytes copied host-to-device.  With conf None,
-    `lengths` is an input and no schedule runs.  The outputs are valid once
-    `stream` has drained."""
+    `lengths` is an input and no schedule runs.  levelwise copies only the
+    logits the outcome depends on, one position level at a time.  The
+    outputs are valid once `stream` has drained."""
     B, K1, V = target_logits.shape
     K = K1 - 1
     if target_logits.is_cuda or not target_logits.is_contiguous():
@@ -327,7 +328,8 @@ def sv_verify_host(target_logits, draft_logits, conf, load: float, draft_tokens,
     _check("sv_verify_host", lib().sv_verify_host(
         _ptr(target_logits), _ptr(draft_logits), dt, B, K, V, _ptr(conf), float(load),
         _ptr(draft_tokens), _ptr(temperature), ctypes.c_uint64(seed & (2**64 - 1)), int(row_base),
-        _ptr(out_tokens), _ptr(out_accept_len), _ptr(lengths), _ptr(status), _ptr(workspace),
+        _ptr(out_tokens), _ptr(out_accept_len), _ptr(lengths), _ptr(status),
+        1 if levelwise else 0, _ptr(workspace),
         workspace.numel() * workspace.element_size(), ctypes.byref(h2d),
         _stream(stream, workspace)))
     return int(h2d.value)

@@ -12,7 +12,17 @@
 // instead), and only each row's scheduled runs are copied -- one
 // cudaMemcpyAsync per contiguous run, adjacent runs merged -- before the
 // device verification and the copy of its outputs back to the host.
+//
+// Level-wise mode copies even less: only the logits the outcome depends on
+// (target 0..a, draft 0..min(a, L-1), a = accepted length).  Level l copies
+// position l of the rows still undecided (target if l <= L, draft if l < L)
+// and, from level 1 on, verifies with lengths min(L, l); a row is final once
+// it rejects below l or l reaches L.  The uniforms are keyed by (row,
+// position, draw), so every decision and draw equals that of one
+// verification with the full lengths, and no kernel reads a position that
+// was not copied.
 #include <cstdint>
+#include <vector>
 
 #include "sv.h"
 #include "sv_host.h"
@@ -84,8 +94,9 @@ extern "C" sv_status sv_verify_host(const void *target_logits, const void *draft
                                     float load, const int32_t *draft_tokens,
                                     const float *temperature, uint64_t seed, int64_t row_base,
                                     int32_t *out_tokens, int32_t *out_accept_len,
-                                    int32_t *lengths, int32_t *status, void *workspace,
-                                    size_t workspace_bytes, size_t *h2d_bytes, void *stream) {
+                                    int32_t *lengths, int32_t *status, int levelwise,
+                                    void *workspace, size_t workspace_bytes, size_t *h2d_bytes,
+                                    void *stream) {
     using sv::hostio::Layout;
     if (!target_logits || !draft_tokens || !temperature || !out_tokens ||
         !out_accept_len || !lengths || !workspace)
@@ -133,13 +144,88 @@ extern "C" sv_status sv_verify_host(const void *target_logits, const void *draft
     }
     if (e != cudaSuccess) return sv::note_cuda(e);
 
-    // 2. The scheduled runs of every row: target positions 0..L, and draft
-    //    positions 0..L-1 of rows that sample with draft logits.
-    sv::hostio::RunCopier cp(st);
     const char *zt_h = static_cast<const char *>(target_logits);
     const char *zd_h = static_cast<const char *>(draft_logits);
     char *zt_d = w + L.zt;
     char *zd_d = w + L.zd;
+    if (levelwise) {
+        // Level l: position l of every undecided row in; from level 1 on,
+        // verify with lengths min(L, l) (finished rows re-run with length 0
+        // on data already present, their outputs ignored), decisions out.
+        const size_t K1 = nk + 1;
+        std::vector<int32_t> lcur(nb), acc(nb), tok(nb * K1);
+        std::vector<char> alive(nb);
+        for (int b = 0; b < B; ++b) {
+            alive[b] = 1;
+            for (size_t i = 0; i < K1; ++i) out_tokens[b * K1 + i] = -1;
+            out_accept_len[b] = -1;
+        }
+        size_t copied = 0;
+        for (int l = 0; l <= K; ++l) {
+            sv::hostio::RunCopier cp(st);
+            int n_alive = 0;
+            for (int b = 0; b < B; ++b) {
+                const int Lb = lengths[b];
+                const bool bad = Lb < 0 || Lb > K;
+                // A row with an invalid length keeps it (it is marked again,
+                // nothing is read); a finished valid row re-runs with length
+                // 0 on its copied position 0.
+                lcur[b] = bad ? Lb : (alive[b] ? (l < Lb ? l : Lb) : 0);
+                if (!alive[b]) continue;
+                ++n_alive;
+                if (bad || l > Lb) continue;
+                const size_t off_t = (static_cast<size_t>(b) * K1 + l) * vb;
+                cp.add(zt_h + off_t, zt_d + off_t, vb);
+            }
+            if (n_alive == 0 && l > 0) break;
+            cp.flush();
+            if (zd_h) {
+                for (int b = 0; b < B; ++b) {
+                    const int Lb = lengths[b];
+                    if (!alive[b] || Lb < 0 || Lb > K || l >= Lb || !(temperature[b] > 0.f))
+                        continue;
+                    const size_t off_d = (static_cast<size_t>(b) * nk + l) * vb;
+                    cp.add(zd_h + off_d, zd_d + off_d, vb);
+                }
+                cp.flush();
+            }
+            if (cp.err != cudaSuccess) return sv::note_cuda(cp.err);
+            copied += cp.total;
+            if (l == 0) continue;   // nothing to test yet; level 1 also settles L = 0
+            e = cudaMemcpyAsync(len_d, lcur.data(), nb * sizeof(int32_t), cudaMemcpyHostToDevice, st);
+            if (e != cudaSuccess) return sv::note_cuda(e);
+            small += nb * sizeof(int32_t);
+            s = sv_verify(zt_d, zd_h ? zd_d : nullptr, dtype, B, K, V, tok_d, len_d, temp_d, seed,
+                          row_base, otok_d, oacc_d, w + L.ver, L.ver_bytes, status_d, stream);
+            if (s != SV_OK) return s;
+            e = cudaMemcpyAsync(acc.data(), oacc_d, nb * sizeof(int32_t), cudaMemcpyDeviceToHost, st);
+            if (e == cudaSuccess)
+                e = cudaMemcpyAsync(tok.data(), otok_d, nb * K1 * sizeof(int32_t),
+                                    cudaMemcpyDeviceToHost, st);
+            if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+            if (e != cudaSuccess) return sv::note_cuda(e);
+            for (int b = 0; b < B; ++b) {
+                if (!alive[b]) continue;
+                const int Lb = lengths[b];
+                const bool bad = Lb < 0 || Lb > K;
+                if (bad || acc[b] < 0 || acc[b] < l || l >= Lb) {   // final: invalid, rejected, or done
+                    alive[b] = 0;
+                    out_accept_len[b] = acc[b];
+                    for (size_t i = 0; i < K1; ++i) out_tokens[b * K1 + i] = tok[b * K1 + i];
+                }
+            }
+        }
+        if (h2d_bytes) *h2d_bytes = copied + small;
+        if (status) {
+            e = cudaMemcpyAsync(status, status_d, sizeof(int32_t), cudaMemcpyDeviceToHost, st);
+            if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        }
+        return sv::note_cuda(e);
+    }
+
+    // 2. The scheduled runs of every row: target positions 0..L, and draft
+    //    positions 0..L-1 of rows that sample with draft logits.
+    sv::hostio::RunCopier cp(st);
     for (int b = 0; b < B; ++b) {
         const int Lb = lengths[b];
         if (Lb < 0 || Lb > K) continue;   // verification marks the row invalid

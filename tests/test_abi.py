@@ -179,7 +179,7 @@ def test_verify_host_arguments_rejected_on_host():
     def call(zt=p, conf=p, tok=p, temp=p, ot=p, oa=p, ln=p, w=ws, wsb=1 << 40, dtype=sv.SV_BF16,
              B=4, K=4, V=1000, row_base=0):
         return L.sv_verify_host(zt, None, dtype, B, K, V, conf, ctypes.c_float(0.3), tok, temp,
-                                ctypes.c_uint64(0), row_base, ot, oa, ln, None, w, wsb, None,
+                                ctypes.c_uint64(0), row_base, ot, oa, ln, None, 1, w, wsb, None,
                                 None)
     for kw in ("zt", "tok", "temp", "ot", "oa", "ln", "w"):
         assert call(**{kw: None}) == 1, kw

@@ -15,7 +15,7 @@ from _parity import gpu_schedule, gpu_verify
 pytestmark = pytest.mark.gpu
 
 
-def _host_run(b, tau, seed, with_draft=True, row_base=0):
+def _host_run(b, tau, seed, with_draft=True, row_base=0, levelwise=False):
     B, K1, V = b.zt.shape
     K = K1 - 1
     dt = sv.SV_BF16 if b.zt.dtype == torch.bfloat16 else sv.SV_F32
@@ -29,7 +29,7 @@ def _host_run(b, tau, seed, with_draft=True, row_base=0):
     n = sv.sv_verify_host_workspace_bytes(B, K, V, dt)
     ws = torch.randint(0, 255, (n,), dtype=torch.uint8, device="cuda")
     h2d = sv.sv_verify_host(zt, zd, conf, tau, tok, temp, seed, ot, oa, ln, ws, status=st,
-                            row_base=row_base)
+                            row_base=row_base, levelwise=levelwise)
     torch.cuda.synchronize()
     return ot.numpy(), oa.numpy(), ln.numpy(), int(st.item()), h2d
 
@@ -52,28 +52,78 @@ def _expected_h2d(b, lengths, with_draft):
     return n + B * K * 8 + B * 4
 
 
+def _expected_h2d_levelwise(b, lengths, accept, with_draft, scheduled=True):
+    """Target 0..a and draft 0..min(a, L-1) of sampled rows, the small
+    arrays, and one length array per verified level."""
+    B, K1, V = b.zt.shape
+    K = K1 - 1
+    es = b.zt.element_size()
+    T = b.temperature.cpu().numpy()
+    n = int(sum((a + 1) * V * es for a in accept))
+    if with_draft:
+        n += int(sum(min(a + 1, L) * V * es for a, L, t in zip(accept, lengths, T) if t > 0))
+    levels = max((a + 1) if a < L else max(L, 1) for a, L in zip(accept, lengths))
+    return n + B * K * 4 + B * 4 + (B * K * 4 if scheduled else 0) + levels * B * 4
+
+
+@pytest.mark.parametrize("levelwise", [False, True])
 @pytest.mark.parametrize("V,dtype,K,B,with_draft", [
     (1000, torch.float32, 4, 32, True), (1001, torch.bfloat16, 6, 48, True),
     (4099, torch.bfloat16, 3, 40, False), (33, torch.float32, 8, 64, True)])
-def test_host_path_equals_device_path(V, dtype, K, B, with_draft):
+def test_host_path_equals_device_path(V, dtype, K, B, with_draft, levelwise):
     b = workloads.random_small(B, K, V, dtype=dtype, seed=V + K, temps=(0.0, 0.6, 1.0))
     for tau, seed in ((0.3, 5), (0.05, 6), (0.9, 7)):
-        ht, ha, hl, hs, h2d = _host_run(b, tau, seed, with_draft, row_base=11)
+        ht, ha, hl, hs, h2d = _host_run(b, tau, seed, with_draft, row_base=11,
+                                        levelwise=levelwise)
         dt_, da, dl, ds = _device_run(b, tau, seed, with_draft, row_base=11)
         assert np.array_equal(hl, dl)
         assert np.array_equal(ha, da) and np.array_equal(ht, dt_)
-        assert hs == ds
-        assert h2d == _expected_h2d(b, hl, with_draft)
+        if levelwise:
+            assert hs & ~sv.SV_NOTE_CDF_FALLBACK == ds & ~sv.SV_NOTE_CDF_FALLBACK
+            assert h2d == _expected_h2d_levelwise(b, hl, ha, with_draft)
+        else:
+            assert hs == ds
+            assert h2d == _expected_h2d(b, hl, with_draft)
 
 
-def test_host_path_full_size_c2():
+@pytest.mark.parametrize("levelwise", [False, True])
+def test_host_path_full_size_c2(levelwise):
     b = workloads.make_batch("c2", device="cuda")
-    ht, ha, hl, hs, h2d = _host_run(b, b.tau, 0)
+    ht, ha, hl, hs, h2d = _host_run(b, b.tau, 0, levelwise=levelwise)
     dt_, da, dl, ds = _device_run(b, b.tau, 0)
     assert np.array_equal(hl, dl) and np.array_equal(ha, da) and np.array_equal(ht, dt_)
-    assert hs == ds == 0
+    assert ds == 0 and hs & ~sv.SV_NOTE_CDF_FALLBACK == 0
     full = (b.zt.numel() + b.zd.numel()) * 2
-    assert h2d == _expected_h2d(b, hl, True) and h2d < 0.6 * full
+    if levelwise:
+        assert h2d == _expected_h2d_levelwise(b, hl, ha, True) and h2d < 0.25 * full
+    else:
+        assert hs == 0
+        assert h2d == _expected_h2d(b, hl, True) and h2d < 0.6 * full
+
+
+def test_levelwise_invalid_rows():
+    """Invalid lengths, temperatures and tokens end as -1 rows with their bits,
+    exactly as on the device path."""
+    b = workloads.random_small(12, 4, 500, dtype=torch.float32, seed=8, temps=(0.0, 1.0))
+    b.lengths = torch.tensor([4, -1, 2, 5, 3, 0, 4, 1, 2, 3, 4, 4], dtype=torch.int32)
+    b.temperature[6] = float("nan")
+    b.tokens[9, 1] = 500
+    B, K1, V = b.zt.shape
+    host = lambda t: t.detach().cpu().contiguous().pin_memory()
+    ln = host(b.lengths)
+    ot = torch.empty((B, K1), dtype=torch.int32).pin_memory()
+    oa = torch.empty((B,), dtype=torch.int32).pin_memory()
+    st = torch.zeros(1, dtype=torch.int32).pin_memory()
+    ws = torch.randint(0, 255, (sv.sv_verify_host_workspace_bytes(B, K1 - 1, V, sv.SV_F32),),
+                       dtype=torch.uint8, device="cuda")
+    sv.sv_verify_host(host(b.zt), host(b.zd), None, 0.0, host(b.tokens), host(b.temperature), 4,
+                      ot, oa, ln, ws, status=st, levelwise=True)
+    torch.cuda.synchronize()
+    g = gpu_verify(b.zt.cuda(), b.zd.cuda(), b.tokens.cuda(), b.lengths.cuda(),
+                   b.temperature.cuda(), 4)
+    assert np.array_equal(oa.numpy(), g["accept"]) and np.array_equal(ot.numpy(), g["tokens"])
+    assert list(oa.numpy()[[1, 3, 6, 9]]) == [-1, -1, -1, -1]
+    assert int(st.item()) & 7 == g["status"] & 7 == 7
 
 
 def test_host_path_with_given_lengths():
