@@ -435,9 +435,10 @@ def run_ours(args, rank, world, local_rank):
                "steps": e2e_steps, "api": "sv_verify_host (levelwise)",
                "note": "inputs in pinned host memory; the schedule's lengths come back, then "
                        "position level l of the rows still undecided is copied and verified "
-                       "(one synchronisation per level), so only the logits the outcome "
-                       f"depends on cross to the device ({max(h2d_seen[1:]) / full:.2f} of the "
-                       f"{full / 1e9:.2f} GB of logits)"}
+                       "(one synchronisation per level), so what crosses to the device is the "
+                       "logits the outcome depends on plus one look-ahead position per "
+                       f"rejecting row ({max(h2d_seen[1:]) / full:.2f} of the {full / 1e9:.2f} GB "
+                       "of logits)"}
         del host, hws
 
     # ---- roofline of the main kernel ----------------------------------------

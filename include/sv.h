@@ -462,11 +462,13 @@ sv_status sv_vp_draw(const sv_vp_slice *slice, const float *mass_all, int32_t *o
  *   status         HOST int32, nullable: the SV_ROW_* / SV_NOTE_* bits of
  *                  this call (written once `stream` has drained).
  *   levelwise      0: copy every scheduled run at once (one synchronisation).
- *                  1: copy only what the outcome depends on (target 0..a,
- *                  draft 0..min(a, L-1), a = accepted length): level l copies
- *                  position l of the rows still undecided and, from l = 1,
- *                  verifies with lengths min(L, l); a row is final once it
- *                  rejects below l or l reaches L.  Same results (the
+ *                  1: level by level: level l copies position l of the rows
+ *                  still undecided and, from l = 1, verifies with lengths
+ *                  min(L, l); a row is final once it rejects below l or l
+ *                  reaches L.  What crosses is what the outcome depends on
+ *                  (target 0..a, draft 0..min(a, L-1), a = accepted length)
+ *                  plus, for a row rejecting at a < L, position a+1, copied
+ *                  before the rejection is known.  Same results (the
  *                  uniforms are keyed by row, position and draw), up to K
  *                  synchronisations; SV_NOTE_* bits may also come from
  *                  draws whose rows were still undecided.

@@ -13,14 +13,16 @@
 // cudaMemcpyAsync per contiguous run, adjacent runs merged -- before the
 // device verification and the copy of its outputs back to the host.
 //
-// Level-wise mode copies even less: only the logits the outcome depends on
-// (target 0..a, draft 0..min(a, L-1), a = accepted length).  Level l copies
-// position l of the rows still undecided (target if l <= L, draft if l < L)
-// and, from level 1 on, verifies with lengths min(L, l); a row is final once
-// it rejects below l or l reaches L.  The uniforms are keyed by (row,
-// position, draw), so every decision and draw equals that of one
-// verification with the full lengths, and no kernel reads a position that
-// was not copied.
+// Level-wise mode copies less: level l copies position l of the rows still
+// undecided (target if l <= L, draft if l < L; one strided 2-D copy per run
+// of consecutive rows) and, from level 1 on, verifies with lengths
+// min(L, l); a row is final once it rejects below l or l reaches L.  What
+// crosses is the logits the outcome depends on (target 0..a, draft
+// 0..min(a, L-1), a = accepted length) plus, for a row that rejects at
+// a < L, position a+1, copied before the rejection is known.  The uniforms
+// are keyed by (row, position, draw), so every decision and draw equals
+// that of one verification with the full lengths, and no kernel reads a
+// position that was not copied.
 #include <cstdint>
 #include <vector>
 
@@ -76,6 +78,35 @@ struct RunCopier {
     void flush() {
         if (n && err == cudaSuccess) err = cudaMemcpyAsync(dst, src, n, cudaMemcpyHostToDevice, st);
         total += n;
+        n = 0;
+    }
+};
+
+// Level-wise copies: position l of a set of rows, one strided 2-D copy per
+// run of consecutive rows (row pitch = one row of the logit array).
+struct LevelCopier {
+    const char *src;
+    char *dst;
+    size_t pitch, width;   // bytes between rows, bytes per vector
+    cudaStream_t st;
+    int b0 = -1, n = 0;
+    size_t total = 0;
+    cudaError_t err = cudaSuccess;
+    LevelCopier(const char *s, char *d, size_t p, size_t w, cudaStream_t q)
+        : src(s), dst(d), pitch(p), width(w), st(q) {}
+    void add(int b) {
+        if (n && b == b0 + n) { ++n; return; }
+        flush();
+        b0 = b;
+        n = 1;
+    }
+    void flush() {
+        if (n && err == cudaSuccess) {
+            const size_t off = static_cast<size_t>(b0) * pitch;
+            err = cudaMemcpy2DAsync(dst + off, pitch, src + off, pitch, width,
+                                    static_cast<size_t>(n), cudaMemcpyHostToDevice, st);
+        }
+        total += static_cast<size_t>(n) * width;
         n = 0;
     }
 };
@@ -162,7 +193,8 @@ extern "C" sv_status sv_verify_host(const void *target_logits, const void *draft
         }
         size_t copied = 0;
         for (int l = 0; l <= K; ++l) {
-            sv::hostio::RunCopier cp(st);
+            const size_t lo = static_cast<size_t>(l) * vb;
+            sv::hostio::LevelCopier ct(zt_h + lo, zt_d + lo, K1 * vb, vb, st);
             int n_alive = 0;
             for (int b = 0; b < B; ++b) {
                 const int Lb = lengths[b];
@@ -174,23 +206,26 @@ extern "C" sv_status sv_verify_host(const void *target_logits, const void *draft
                 if (!alive[b]) continue;
                 ++n_alive;
                 if (bad || l > Lb) continue;
-                const size_t off_t = (static_cast<size_t>(b) * K1 + l) * vb;
-                cp.add(zt_h + off_t, zt_d + off_t, vb);
+                ct.add(b);
             }
             if (n_alive == 0 && l > 0) break;
-            cp.flush();
-            if (zd_h) {
+            ct.flush();
+            size_t level_bytes = ct.total;
+            cudaError_t cerr = ct.err;
+            if (zd_h && l < K) {
+                sv::hostio::LevelCopier cd(zd_h + lo, zd_d + lo, nk * vb, vb, st);
                 for (int b = 0; b < B; ++b) {
                     const int Lb = lengths[b];
                     if (!alive[b] || Lb < 0 || Lb > K || l >= Lb || !(temperature[b] > 0.f))
                         continue;
-                    const size_t off_d = (static_cast<size_t>(b) * nk + l) * vb;
-                    cp.add(zd_h + off_d, zd_d + off_d, vb);
+                    cd.add(b);
                 }
-                cp.flush();
+                cd.flush();
+                level_bytes += cd.total;
+                if (cerr == cudaSuccess) cerr = cd.err;
             }
-            if (cp.err != cudaSuccess) return sv::note_cuda(cp.err);
-            copied += cp.total;
+            if (cerr != cudaSuccess) return sv::note_cuda(cerr);
+            copied += level_bytes;
             if (l == 0) continue;   // nothing to test yet; level 1 also settles L = 0
             e = cudaMemcpyAsync(len_d, lcur.data(), nb * sizeof(int32_t), cudaMemcpyHostToDevice, st);
             if (e != cudaSuccess) return sv::note_cuda(e);

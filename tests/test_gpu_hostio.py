@@ -53,15 +53,17 @@ def _expected_h2d(b, lengths, with_draft):
 
 
 def _expected_h2d_levelwise(b, lengths, accept, with_draft, scheduled=True):
-    """Target 0..a and draft 0..min(a, L-1) of sampled rows, the small
-    arrays, and one length array per verified level."""
+    """Target 0..a and draft 0..min(a, L-1) of sampled rows (what the outcome
+    depends on), plus for a row that rejects at a < L the next position,
+    copied before the rejection is known (target a+1; draft a+1 if a+1 < L);
+    the small arrays; one length array per verified level."""
     B, K1, V = b.zt.shape
     K = K1 - 1
     es = b.zt.element_size()
     T = b.temperature.cpu().numpy()
-    n = int(sum((a + 1) * V * es for a in accept))
+    n = int(sum((a + 2 if a < L else L + 1) * V * es for a, L in zip(accept, lengths)))
     if with_draft:
-        n += int(sum(min(a + 1, L) * V * es for a, L, t in zip(accept, lengths, T) if t > 0))
+        n += int(sum(min(a + 2, L) * V * es for a, L, t in zip(accept, lengths, T) if t > 0))
     levels = max((a + 1) if a < L else max(L, 1) for a, L in zip(accept, lengths))
     return n + B * K * 4 + B * 4 + (B * K * 4 if scheduled else 0) + levels * B * 4
 
@@ -95,7 +97,7 @@ def test_host_path_full_size_c2(levelwise):
     assert ds == 0 and hs & ~sv.SV_NOTE_CDF_FALLBACK == 0
     full = (b.zt.numel() + b.zd.numel()) * 2
     if levelwise:
-        assert h2d == _expected_h2d_levelwise(b, hl, ha, True) and h2d < 0.25 * full
+        assert h2d == _expected_h2d_levelwise(b, hl, ha, True) and h2d < 0.35 * full
     else:
         assert hs == 0
         assert h2d == _expected_h2d(b, hl, True) and h2d < 0.6 * full
