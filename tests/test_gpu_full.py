@@ -7,7 +7,6 @@ independently on each side; rows whose survival product sits within 1e-6 of
 tau are excluded and counted."""
 import numpy as np
 import pytest
-import torch
 
 import oracle
 from speculative_decoding_verification_93_b200 import workloads
