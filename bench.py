@@ -310,6 +310,14 @@ def run_ours(args, rank, world, local_rank):
     clocks = ClockSampler(local_rank)
     if rank == 0:
         clocks.start()
+    # Keep the GPU busy for about half a second of untimed steps while the
+    # sampler (one sample per 200 ms) starts, so its samples see the load the
+    # timed region runs under; every rank runs the same count.
+    n_load = max(1, int(0.5 / 120e-6))
+    for i in range(n_load):
+        step(args.warmup + i, batch.zt, batch.zd, batch.tokens, batch.temperature, batch.conf,
+             ln_buf)
+    torch.cuda.synchronize()
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
