@@ -200,9 +200,10 @@ size_t sv_verify_workspace_bytes(int B, int K, int V, sv_dtype dtype);
  * agrees with are kept, followed by one token of the target's own, and the
  * rest are dropped; the test is rejection sampling, which leaves the emitted
  * tokens distributed exactly as the target's, and a rejected draft gives way
- * to a token of the target's choosing); zhichai.net DSpark topic, section "Why LLMs
- * speak so slowly" (rejection sampling on the target/draft probability
- * ratio; generation restarts from the first error).  In symbols, per row b
+ * to a token of the target's choosing); zhichai.net DSpark topic, section
+ * "Why LLMs speak so slowly" (rejection sampling on the ratio of target to
+ * draft probability; decoding goes on from the first rejected position).
+ * In symbols, per row b
  * with verify length L = lengths[b] and temperature T = temperature[b]:
  *
  *   p_i = softmax(zt[b, i, :] / T),  q_i = softmax(zd[b, i, :] / T);

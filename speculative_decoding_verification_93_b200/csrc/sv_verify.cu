@@ -2,14 +2,14 @@
 //
 // Method (cited as page title + section):
 //  - umans.ai, "DeepSeek V4 Pro DSpark: the model isn't ready, the
-//    architecture is", section "Speculative decoding, briefly": the target
-//    scores the whole draft block in one pass, keeps the prefix it agrees
-//    with plus one token of its own; the acceptance rule is rejection
-//    sampling under which accepted tokens follow the target distribution
-//    exactly, and a rejected token is replaced by one the target would emit.
+//    architecture is", section "Speculative decoding, briefly": one target
+//    pass checks the whole draft block; the drafts it agrees with stay and
+//    one token of its own follows; the test is rejection sampling, which
+//    leaves the emitted tokens distributed exactly as the target's, and a
+//    rejected draft gives way to a token of the target's choosing.
 //  - zhichai.net DSpark topic, section "Why LLMs speak so slowly": the test
-//    is on the target/draft probability ratio; generation restarts from the
-//    first error.
+//    compares the target and draft probabilities by their ratio; decoding
+//    goes on from the first rejected position.
 //  - techvisionai "DeepSeek-V4: Breaking the Efficiency Barrier", Ch. 7
 //    "Deployment with vLLM": greedy drafting (q one-hot at the draft token).
 // In symbols: accept x_i iff u_i < min(1, p_i(x_i)/q_i(x_i)); at the first
@@ -40,9 +40,11 @@
 //      each sampled row's final draw (for p-mass draws the chunk is chosen
 //      from the stream partials) and appends the resample work list.
 //   4. resample_kernel (one CTA per work entry): residual draws sum
-//      max(0, p_j - q_j) over their chunk by 64-unit sub-ranges; the last
-//      chunk CTA of the row (atomic counter, no waiting) picks the sub-range
-//      from the row's table and the token inside it.  p-mass draws locate
+//      max(0, p_j - q_j) over their chunk by 64-unit sub-ranges, and each
+//      chunk CTA also forms its chunk's total in the order the scan will
+//      walk it; the last chunk CTA of the row (atomic counter, no waiting)
+//      picks the chunk from the chunk totals, the sub-range from that
+//      chunk's sub-ranges, and the token inside it.  p-mass draws locate
 //      the token inside the chosen chunk.  Only position j of a rejecting
 //      row is read a second time.
 #include <climits>

@@ -1,5 +1,5 @@
-"""Distribution tests on GPU draws: the emitted tokens follow the target
-distribution (chi-square over 10^6 draws, V <= 8), and the mean accepted
+"""Distribution tests on GPU draws: the emitted tokens are distributed as
+the target's (chi-square over 10^6 draws, V <= 8), and the mean accepted
 length at a large vocabulary matches the closed form
 E[a] = sum_{i=1..L} prod_{j<i} beta_j, beta_j = sum_v min(p_j, q_j)."""
 import math
