@@ -55,10 +55,40 @@ KERNEL_SOURCES = ["speculative_decoding_verification_93_b200/csrc/sv_verify.cu",
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "stream_kernel_c2.md")
 
 
+def code_only(text: str) -> str:
+    """C/C++/CUDA source with comments and whitespace outside string and
+    character literals removed: what the compiler sees, so that editing a
+    comment does not change the hash while any change of code does."""
+    out = []
+    i, n = 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        elif c.isspace():
+            i += 1
+        else:
+            out.append(c)
+            i += 1
+    return "".join(out)
+
+
 def kernel_hash() -> str:
+    """Hash of the main kernel's code (comments and whitespace removed)."""
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        h.update(open(os.path.join(ROOT, f), "rb").read())
+        h.update(code_only(open(os.path.join(ROOT, f)).read()).encode())
+        h.update(b"\0")
     return h.hexdigest()[:16]
 
 
@@ -310,10 +340,11 @@ def run_ours(args, rank, world, local_rank):
     clocks = ClockSampler(local_rank)
     if rank == 0:
         clocks.start()
-    # Keep the GPU busy for about half a second of untimed steps while the
-    # sampler (one sample per 200 ms) starts, so its samples see the load the
-    # timed region runs under; every rank runs the same count.
-    n_load = max(1, int(0.5 / 120e-6))
+    # Keep the GPU busy for --clock-load-s (about half a second) of untimed
+    # steps while the sampler (one sample per 200 ms) starts, so its samples
+    # see the load the timed region runs under; every rank runs the same
+    # count.
+    n_load = max(0, int(args.clock_load_s / 120e-6))
     for i in range(n_load):
         step(args.warmup + i, batch.zt, batch.zd, batch.tokens, batch.temperature, batch.conf,
              ln_buf)
@@ -567,6 +598,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-vocab", action="store_true")
+    ap.add_argument("--clock-load-s", type=float, default=0.5,
+                    help="seconds of untimed steps before the timed region, so the clock "
+                         "sampler sees load (0 under a profiler)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-rows", type=int, default=64)
     args = ap.parse_args()
