@@ -188,3 +188,27 @@ def test_verify_host_arguments_rejected_on_host():
     assert call(row_base=-1) == 1
     assert call(w=v((1 << 24) + 16)) == 1
     assert call(wsb=n - 1) == 4
+
+
+def _declared_arity():
+    """Parameter count of every function declared in include/sv.h."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    out = {}
+    for m in re.finditer(r"\b(sv_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_argtypes_match_header():
+    L = sv.lib()
+    arity = _declared_arity()
+    assert "sv_verify_host" in arity and "sv_vp_decide" in arity
+    checked = 0
+    for name, n in arity.items():
+        fn = getattr(L, name)
+        if fn.argtypes is not None:
+            assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
+            checked += 1
+    assert checked >= 20
