@@ -4,8 +4,9 @@ Each rank holds a contiguous slice of the vocabulary of both models' logits,
 as a serving engine whose output heads are split by vocabulary produces them
 (zhichai.net DSpark topic, "From paper to running service in two weeks";
 techvisionai "DeepSeek-V4: Breaking the Efficiency Barrier", Ch. 7
-"Deployment with vLLM").  One step is three kernels of ``libsv.so`` with
-three collectives between them (``include/sv.h``, sv_vp_*):
+"Deployment with vLLM").  One step is three entry points of ``libsv.so``
+(four kernel launches: sv_vp_decide issues two) with three collectives
+between them (``include/sv.h``, sv_vp_*):
 
     sv_vp_stats -> all-gather (rank order) -> sv_vp_decide
                 -> all-gather (rank order) -> sv_vp_draw -> all-reduce(max)

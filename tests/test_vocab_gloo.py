@@ -200,3 +200,13 @@ def test_gloo_ranks_reproduce_unsplit_vocabulary(tmp_path, world):
     mp.start_processes(_worker, args=(world, _free_port(), path), nprocs=world, join=True,
                        start_method="spawn")
     assert open(path).read() == "ok"
+
+
+def test_exchanges_without_a_process_group():
+    """One rank: the gather copies (or aliases) and the reduction is a no-op."""
+    local = torch.arange(6, dtype=torch.float32).reshape(3, 2)
+    out = torch.zeros(3, 2)
+    assert torch.equal(gather_in_rank_order(local, out), local)
+    assert gather_in_rank_order(local, local) is local
+    tok = torch.tensor([[3, -1], [-1, 5]], dtype=torch.int32)
+    assert torch.equal(reduce_tokens(tok.clone()), tok)
