@@ -448,13 +448,20 @@ def run_ours(args, rank, world, local_rank):
         hws = torch.empty(sv.sv_verify_host_workspace_bytes(B, K, V, dt), dtype=torch.uint8,
                           device=dev)
         e2e_steps = max(1, min(args.steps, args.e2e_steps))
-        h2d_seen = []
+        h2d_seen, d2h_seen = [], []
 
         def e2e_step(i):
             h2d_seen.append(sv.sv_verify_host(
                 host["zt"], host["zd"], host["conf"] if fixed is None else None, batch.tau,
                 host["tokens"], host["temperature"], args.seed + i, h_tok, h_acc, h_len, hws,
                 row_base=row_base, levelwise=True))
+            # Device-to-host bytes: the lengths (when scheduled), then per verified
+            # level the accept lengths and the tokens.  Level-wise outputs are on
+            # the host when the call returns; a row is settled at level a + 1
+            # (rejected) or max(L, 1) (done), and the levels run to the last one.
+            a, L = h_acc.numpy(), h_len.numpy()
+            levels = max(1, int(np.where(a < L, a + 1, np.maximum(L, 1)).max()))
+            d2h_seen.append((B * 4 if fixed is None else 0) + levels * (B * 4 + B * (K + 1) * 4))
 
         e2e_step(0)
         torch.cuda.synchronize()
@@ -467,17 +474,18 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         ms_e2e = e0.elapsed_time(e1)
         ms_e2e = max_over_ranks(ms_e2e, dev)
-        d2h = h_tok.numel() * 4 + h_acc.numel() * 4 + (B * 4 if fixed is None else 0)
+        d2h = sum(d2h_seen[1:]) / len(d2h_seen[1:])
         full = sum(host[n].numel() * host[n].element_size() for n in ("zt", "zd"))
+        h2d_mean = sum(h2d_seen[1:]) / len(h2d_seen[1:])   # varies with each step's acceptances
         e2e = {"value": positions * world / (ms_e2e / e2e_steps / 1e3), "unit": UNIT,
-               "h2d_bytes_per_step": int(max(h2d_seen[1:])), "d2h_bytes_per_step": int(d2h),
+               "h2d_bytes_per_step": int(round(h2d_mean)), "d2h_bytes_per_step": int(round(d2h)),
                "steps": e2e_steps, "api": "sv_verify_host (levelwise)",
                "note": "inputs in pinned host memory; the schedule's lengths come back, then "
                        "position level l of the rows still undecided is copied and verified "
                        "(one synchronisation per level), so what crosses to the device is the "
                        "logits the outcome depends on plus one look-ahead position per "
-                       f"rejecting row ({max(h2d_seen[1:]) / full:.2f} of the {full / 1e9:.2f} GB "
-                       "of logits)"}
+                       f"rejecting row ({h2d_mean / full:.2f} of the {full / 1e9:.2f} GB "
+                       "of logits, mean over the timed steps)"}
         del host, hws
 
     # ---- roofline of the main kernel ----------------------------------------
