@@ -386,6 +386,22 @@ def run_ours(args, rank, world, local_rank):
     sv.sv_profile_begin(0)
     alg_bytes = sum(need) / len(need)
 
+    # ---- the schedule alone (the step above runs it before each verification) --
+    sched = None
+    if rank == 0 and fixed is None:
+        sch_len = torch.empty(B, dtype=torch.int32, device=dev)
+        for _ in range(3):
+            sv.sv_schedule(batch.conf, batch.tau, sch_len)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            sv.sv_schedule(batch.conf, batch.tau, sch_len)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        sched = {"kernel": "sv::schedule_kernel", "us_per_call": round(e0.elapsed_time(e1) /
+                                                                       args.steps * 1e3, 2),
+                 "rows": B, "positions": K, "bound": "launch latency (B threads)"}
+
     # ---- hardware-aware admission on the same confidences (next row of the
     # scheduler): a profiled speed table of the shape steps/s = s0/(1+n/n0) -------
     admit = None
@@ -540,7 +556,8 @@ def run_ours(args, rank, world, local_rank):
                               parallelism=f"dp{world} (row shards, no collective)"),
                "e2e": e2e, "gpu_launches": args.steps * (sv.sv_verify_launches()
                                                          + (1 if fixed is None else 0)),
-               "roofline": roofline, "cpu_baseline": cpu, "clocks": clk, "admission": admit,
+               "roofline": roofline, "cpu_baseline": cpu, "clocks": clk, "schedule": sched,
+               "admission": admit,
                "calibration": calib, "vocab_parallel": vocab,
                "device_status": st, "impl": "ours"}
         print(json.dumps(out), flush=True)
