@@ -210,3 +210,26 @@ def test_exchanges_without_a_process_group():
     assert gather_in_rank_order(local, local) is local
     tok = torch.tensor([[3, -1], [-1, 5]], dtype=torch.int32)
     assert torch.equal(reduce_tokens(tok.clone()), tok)
+
+
+def test_verifier_buffers_and_slice_checks_on_cpu():
+    """Buffer sizing of one rank (no process group) and the slice
+    description's argument checks; no kernel runs."""
+    import speculative_decoding_verification_93_b200 as sv
+    from speculative_decoding_verification_93_b200.vocab_parallel import VocabParallelVerifier
+    v = VocabParallelVerifier(256, 8, 129280, torch.bfloat16, "cpu")
+    assert (v.world, v.rank, v.v0, v.Vs) == (1, 0, 0, 129280)
+    assert v.stats_local.numel() == 256 * 17 * 4 * 16          # four 64 KB chunks per vector
+    assert v.stats_all is v.stats_local and v.mass_all is v.mass_local
+    assert v.workspace.numel() > 256 * 2 * 506 * 4             # two segment tables per row
+    with pytest.raises(TypeError):
+        VocabParallelVerifier(4, 2, 100, torch.float16, "cpu")
+    zt = torch.zeros(2, 3, 50)
+    d = sv.vp_slice(zt, torch.zeros(2, 2, 50), 100, 50, 2, 1)
+    assert (d.B, d.K, d.V, d.v0, d.Vs, d.nshards, d.shard) == (2, 2, 100, 50, 50, 2, 1)
+    with pytest.raises(TypeError):
+        sv.vp_slice(zt, torch.zeros(2, 2, 49), 100, 50, 2, 1)     # draft slice of another width
+    with pytest.raises(TypeError):
+        sv.vp_slice(zt.double(), None, 100, 50, 2, 1)             # unsupported dtype
+    with pytest.raises(ValueError):
+        v.slice_of(torch.zeros(256, 9, 100, dtype=torch.bfloat16), None)
