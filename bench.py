@@ -1,23 +1,27 @@
 """Benchmark: confidence-scheduled speculative verification on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload c2]
+                    [--workload c0|c1|c2|c3|c4] [--tau T]
 
 One step = one pass of the whole hot path over one batch: the schedule
 (prefix survival -> verify lengths) and the verification (softmax statistics,
 accept test, correction/bonus draw), through the library's C ABI.  The
 default workload is the 256-row, 8-draft, 129280-token bf16 batch (per-row
 temperature from {0, 0.6, 1.0}, lengths from the schedule with
-conf ~ Beta(8,2), tau = 0.3).  Inputs are synthetic and seeded.
+conf ~ Beta(8,2), tau = 0.3).  Inputs are synthetic and seeded.  Workloads
+whose inputs are under twice the L2 size are timed step by step with L2
+flushed before each step.
 
 Prints one JSON line (rank 0).  `value` is verified draft positions per
 second over all ranks (sum of the scheduled lengths per step / device time,
-max over ranks); `roofline` is the main verification kernel's algorithmic
-logit bytes per launch over its CUDA-event duration; `e2e` repeats the
-measurement with the inputs in pinned host memory and the host<->device
-copies inside the timed region; `cpu_baseline` is the fp64 CPU oracle on a
-bounded sample of the same workload.  `--impl reference` times the oracle
-alone (rank 0; other ranks exit).
+max over ranks); `roofline` is the main verification kernel's bytes per
+launch -- the logits the outcome depends on -- over its CUDA-event
+duration; `e2e` repeats the measurement with the inputs in pinned host
+memory and the host<->device copies inside the timed region;
+`cpu_baseline` is the fp64 CPU oracle on all host cores and on one core;
+`parity` checks the timed steps' outputs row by row against the oracle.
+`--impl reference` times the oracle alone on the whole batch (rank 0;
+other ranks exit).
 
 Multi-GPU (torchrun): rows are independent, so every rank verifies its own
 batch of B rows (Philox rows offset by rank * B) with no data-path
@@ -29,7 +33,6 @@ import argparse
 import hashlib
 import json
 import os
-import re
 import statistics
 import subprocess
 import sys
@@ -52,7 +55,8 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["speculative_decoding_verification_93_b200/csrc/sv_verify.cu",
                   "speculative_decoding_verification_93_b200/csrc/sv_device.cuh"]
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "stream_kernel_c2.md")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "stream_kernel_traffic.json")
+L2_BYTES = 126 << 20
 
 
 def code_only(text: str) -> str:
@@ -101,18 +105,18 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def committed_traffic():
-    """DRAM bytes per launch of the main kernel from the committed ncu
-    summary, if it was taken on the current kernel source."""
+def committed_traffic(workload: str):
+    """DRAM bytes per launch of the main kernel from the committed ncu figures
+    (a small JSON file keyed by workload), if they were taken on the current
+    kernel code."""
     try:
-        text = open(TRAFFIC_FILE).read()
-    except OSError:
+        d = json.load(open(TRAFFIC_FILE))
+    except (OSError, ValueError):
         return None
-    mh = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
-    mt = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not mh or not mt or mh.group(1) != kernel_hash():
+    if d.get("kernel_source_hash") != kernel_hash():
         return None
-    return float(mt.group(1))
+    w = d.get("workloads", {}).get(workload)
+    return None if w is None else float(w["dram_bytes_per_launch"])
 
 
 class ClockSampler:
@@ -188,42 +192,108 @@ def needed_bytes(accept: np.ndarray, lengths: np.ndarray, temperature: np.ndarra
     return int((esize * V * ((a + 1) + drafts)).sum())
 
 
-def oracle_sample(batch, lengths_np, budget_s: float, seed0: int = 0):
-    """Time the fp64 CPU oracle, as it stands, on whole passes over the batch
-    (one verification seed per pass) until ~budget_s of CPU time is spent."""
+def oracle_leg(batch, gpu_lengths, results, budget_s: float, budget_1core_s: float,
+               parity_budget_s: float, row_base: int = 0):
+    """The CPU-baseline leg: the fp64 oracle, as it stands, on the host cores.
+
+    1. All cores: whole passes over the batch, one per timed step's seed, in
+       order, until ~budget_s of wall time.
+    2. One core: the same rule on row blocks of the first step's seed until
+       ~budget_1core_s.
+    3. Parity of the timed steps: the GPU's outputs at each step's seed
+       (``results``: list of (seed, out_tokens, out_accept)) are checked row
+       by row against the oracle -- each row bit-exact or one of the
+       oracle's tie-window outcomes -- until ~parity_budget_s.
+    The oracle schedules on its own (rows on the schedule window may take
+    either length).  Host copies of the logits are made once, untimed."""
     import oracle
+    from oracle import compare as ocompare
     from speculative_decoding_verification_93_b200.workloads import to_host_logits
     zt = to_host_logits(batch.zt)
     zd = to_host_logits(batch.zd)
     tok = batch.tokens.cpu().numpy()
     tmp = batch.temperature.cpu().numpy()
+    B = tok.shape[0]
+    if batch.lengths is None:
+        L0, Llo, Lhi = ocompare.schedule_span(batch.conf.cpu().numpy(), batch.tau)
+    else:
+        L0 = Llo = Lhi = batch.lengths.cpu().numpy()
+    rid = np.arange(B, dtype=np.int64) + row_base
     nthreads = oracle.default_threads()
+    seeds = [r[0] for r in results]
+
     positions, passes = 0, 0
     t0 = time.perf_counter()
     while True:
-        oracle.verify(zt, zd, tok, lengths_np, tmp, seed0 + passes, nthreads=nthreads)
+        oracle.verify(zt, zd, tok, L0, tmp, seeds[passes % len(seeds)], row_ids=rid,
+                      nthreads=nthreads)
         passes += 1
-        positions += int(lengths_np.sum())
+        positions += int(L0.sum())
         el = time.perf_counter() - t0
         if el >= budget_s or passes >= 1000:
             break
-    return dict(value=positions / el, unit=UNIT, cores=nthreads, kind="oracle",
-                sample=f"{passes} full pass(es) over the {batch.spec.B}-row batch "
-                       f"(seeds {seed0}..{seed0 + passes - 1}), {el:.1f} s wall, "
-                       f"OpenMP over rows")
+    cpu = dict(value=round(positions / el, 1), unit=UNIT, cores=nthreads, kind="oracle",
+               sample=f"{passes} full pass(es) over the {B}-row batch at the timed steps' "
+                      f"seeds, {el:.1f} s wall, OpenMP over rows on {nthreads} threads")
+
+    pos1, rows1 = 0, 0
+    t0 = time.perf_counter()
+    while True:
+        r0 = rows1 % B
+        r1 = min(B, r0 + 8)
+        oracle.verify(zt[r0:r1], zd[r0:r1], tok[r0:r1], L0[r0:r1], tmp[r0:r1],
+                      seeds[(rows1 // B) % len(seeds)], row_ids=rid[r0:r1], nthreads=1)
+        pos1 += int(L0[r0:r1].sum())
+        rows1 += r1 - r0
+        el1 = time.perf_counter() - t0
+        if el1 >= budget_1core_s or rows1 >= 1000 * B:
+            break
+    cpu["single_core"] = {"value": round(pos1 / el1, 1), "unit": UNIT, "cores": 1,
+                          "sample": f"{rows1} rows in blocks of 8 (passes over the batch at "
+                                    f"the timed steps' seeds), {el1:.1f} s"}
+
+    tally = ocompare.Tally()
+    checked = []
+    t0 = time.perf_counter()
+    for seed, g_tok, g_acc in results:
+        tally.add(ocompare.check_rows(lambda idx: (zt[idx], zd[idx]), tok, tmp, seed, L0, Llo,
+                                      Lhi, gpu_lengths, g_tok, g_acc, row_base=row_base,
+                                      block=64, nthreads=nthreads))
+        checked.append(seed)
+        if time.perf_counter() - t0 >= parity_budget_s:
+            break
+    parity = dict(tally.summary(), steps_checked=len(checked),
+                  seeds=f"{checked[0]}..{checked[-1]}",
+                  rule="each row bit-exact against the oracle, or one of the oracle's outcomes "
+                       "for decisions inside the tie windows (|u - min(1, ratio)| < 1e-5; draw "
+                       "target within 1e-5 R of a CDF boundary; |S_i - tau| < 1e-6)")
+    if tally.first_invalid:
+        parity["first_invalid"] = tally.first_invalid
+    return cpu, parity
+
+
+def needs_flush(batch, esize) -> bool:
+    """Inputs smaller than twice the L2 would be partly served from L2 by the
+    next step: those workloads flush L2 before every timed step."""
+    return (batch.zt.numel() + batch.zd.numel()) * esize < 2 * L2_BYTES
 
 
 def workload_config(batch, lengths_np, esize):
     s = batch.spec
     dt = "bf16" if s.dtype == torch.bfloat16 else "fp32"
     inputs = (batch.zt.numel() + batch.zd.numel()) * esize
+    l2 = (f"inputs {inputs / 1e9:.3f} GB < 2 x 126 MB L2: L2 flushed before every timed step "
+          "(a 256 MB buffer written, then another read), each step timed alone with CUDA "
+          "events" if needs_flush(batch, esize) else
+          f"inputs {inputs / 1e9:.2f} GB > 126 MB L2 (no flush; steps back to back)")
     return {"workload": (f"{s.name}: B={s.B} K={s.K} V={s.V} {dt} logits; "
                          f"T per row from {list(s.temps)}; "
                          + (f"lengths from sv_schedule (conf~Beta{s.beta}, tau={batch.tau})"
                             if s.fixed_length is None else f"lengths={s.fixed_length}")),
             "B": s.B, "K": s.K, "V": s.V, "logits": dt,
+            "tau": batch.tau if s.fixed_length is None else None,
             "mean_L": float(lengths_np.mean()),
-            "l2": f"inputs {inputs / 1e9:.2f} GB > 126 MB L2 (no flush)",
+            "l2": l2,
             "data_seed": s.data_seed}
 
 
@@ -307,7 +377,7 @@ def run_ours(args, rank, world, local_rank):
     dist = None
     if world > 1:
         import torch.distributed as dist
-    batch = workloads.make_batch(args.workload, device=dev,
+    batch = workloads.make_batch(args.workload, device=dev, tau=args.tau,
                                  data_seed=workloads.SPECS[args.workload].data_seed + 1000 * rank)
     s = batch.spec
     B, K, V = s.B, s.K, s.V
@@ -348,6 +418,13 @@ def run_ours(args, rank, world, local_rank):
     for i in range(n_load):
         step(args.warmup + i, batch.zt, batch.zd, batch.tokens, batch.temperature, batch.conf,
              ln_buf)
+    flush = needs_flush(batch, esize)
+    if flush:
+        # L2 flush between steps: write one 256 MB buffer, then read another,
+        # so the step starts with none of its inputs in L2 and no dirty lines
+        # left to write back.
+        flush_w = torch.empty(64 << 20, dtype=torch.float32, device=dev)
+        flush_r = torch.ones(64 << 20, dtype=torch.float32, device=dev)
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
@@ -355,15 +432,28 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream(dev)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(args.steps):
-        step(args.warmup + i, batch.zt, batch.zd, batch.tokens, batch.temperature, batch.conf,
-             ln_buf)
-    e1.record(stream)
-    torch.cuda.synchronize()
+    if flush:
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush_w.zero_()
+            flush_r.sum()
+            evs[i][0].record(stream)
+            step(args.warmup + i, batch.zt, batch.zd, batch.tokens, batch.temperature,
+                 batch.conf, ln_buf)
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        ms_total = sum(a.elapsed_time(b) for a, b in evs)
+    else:
+        e0.record(stream)
+        for i in range(args.steps):
+            step(args.warmup + i, batch.zt, batch.zd, batch.tokens, batch.temperature,
+                 batch.conf, ln_buf)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms_total = e0.elapsed_time(e1)
     if dist:
         dist.barrier()
-    ms_total = e0.elapsed_time(e1)
     clk = clocks.stop() if rank == 0 else None
     ms_total = max_over_ranks(ms_total, dev)
     ms_step = ms_total / args.steps
@@ -376,11 +466,17 @@ def run_ours(args, rank, world, local_rank):
     # from overlapping, which costs the step about 10 us) -------------------
     sv.sv_profile_begin(args.steps)
     torch.cuda.synchronize()
-    need = []
+    need, results = [], []
     for i in range(args.steps):
+        if flush:
+            flush_w.zero_()
+            flush_r.sum()
         step(args.warmup + i, batch.zt, batch.zd, batch.tokens, batch.temperature, batch.conf,
              ln_buf)
-        need.append(needed_bytes(out_acc.cpu().numpy(), lengths_np, temp_np, V, esize))
+        acc_np = out_acc.cpu().numpy()
+        need.append(needed_bytes(acc_np, lengths_np, temp_np, V, esize))
+        # same seeds as the timed steps, so these are the timed steps' outputs
+        results.append((args.seed + args.warmup + i, out_tok.cpu().numpy(), acc_np))
     torch.cuda.synchronize()
     kernel_ms = sv.sv_profile_read(args.steps)
     sv.sv_profile_begin(0)
@@ -508,33 +604,39 @@ def run_ours(args, rank, world, local_rank):
     peak, peak_src = measured_hbm_peak()
     kms = [t for t in kernel_ms if t > 0]
     avg_kernel_ms = sum(kms) / len(kms) if kms else float("nan")
-    # achieved: the algorithmic bytes of one launch -- every scheduled logit
-    # once, elt * V * [(L_b + 1) + L_b * (T_b > 0)] per row -- over the
-    # launch's own duration, averaged.  The kernel reads fewer bytes than
-    # that (positions after a row's first rejection are skipped once the
-    # rejection is known); `traffic` and the needed-bytes keys show how many.
-    achieved = (sum(sched_bytes / (t / 1e3) for t in kernel_ms if t > 0) / len(kms) / 1e9
+    # achieved: the bytes the outcome depends on -- target positions 0..a and
+    # draft positions 0..min(a, L-1) of sampled rows, a the accepted length --
+    # each launch's own figure over that launch's duration, averaged.  Those
+    # are the bytes verification must read once; positions after a row's
+    # first rejection never change the output and the kernel skips them.
+    # The bytes of every scheduled logit, read or not, are kept as a
+    # secondary figure.
+    achieved = (sum(nb / (t / 1e3) for nb, t in zip(need, kernel_ms) if t > 0) / len(kms) / 1e9
                 if kms else float("nan"))
-    achieved_needed = (sum(nb / (t / 1e3) for nb, t in zip(need, kernel_ms) if t > 0) / len(kms)
-                       / 1e9 if kms else float("nan"))
-    traffic = committed_traffic()
+    achieved_sched = (sum(sched_bytes / (t / 1e3) for t in kernel_ms if t > 0) / len(kms) / 1e9
+                      if kms else float("nan"))
+    traffic = committed_traffic(args.workload if args.tau is None else
+                                f"{args.workload}_tau{args.tau:g}")
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src ==
                 "measured" else "fallback 6650 GB/s",
                 "kernel": "sv::stream_kernel", "kernel_ms": round(avg_kernel_ms, 5),
-                "algorithmic_bytes_per_launch": int(sched_bytes),
-                "algorithmic_bytes": "every scheduled logit once: elt*V*[(L_b+1) + L_b*(T_b>0)] "
-                                     "per row",
+                "algorithmic_bytes_per_launch": int(alg_bytes),
+                "algorithmic_bytes": "logits the outcome depends on, each read once: target "
+                                     "positions 0..a and draft positions 0..min(a, L-1) of "
+                                     "sampled rows (a = accepted length); mean over the timed "
+                                     "steps",
                 "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
-                "needed_bytes_per_launch": int(alg_bytes),
-                "needed_bytes": "logits the outcome depends on: target positions 0..a and draft "
-                                "positions 0..min(a, L-1) per row (a = accepted length); the "
-                                "kernel skips positions after a row's first rejection once it "
-                                "is known",
-                "achieved_needed": round(achieved_needed, 1),
-                "frac_needed": round(achieved_needed / peak, 4),
-                "step_gbs": round(sched_bytes / (ms_step / 1e3) / 1e9, 1),
+                "scheduled_bytes_per_launch": int(sched_bytes),
+                "scheduled_bytes": "every scheduled logit once, elt*V*[(L_b+1) + L_b*(T_b>0)] "
+                                   "per row; the kernel does not read the positions after a "
+                                   "row's first rejection once it is known",
+                "achieved_if_all_scheduled_read": round(achieved_sched, 1),
+                "frac_if_all_scheduled_read": round(achieved_sched / peak, 4),
+                "traffic_rate_gbs": (round(traffic / (avg_kernel_ms / 1e3) / 1e9, 1)
+                                     if traffic else None),
+                "step_gbs": round(alg_bytes / (ms_step / 1e3) / 1e9, 1),
                 "kernel_timing": "CUDA events around each stream-kernel launch over a second "
                                  "timed pass of the same steps"}
 
@@ -543,9 +645,11 @@ def run_ours(args, rank, world, local_rank):
         vocab = vocab_parallel_probe(batch, ln_buf, V, esize, sched_bytes, args.seed,
                                      min(args.steps, 20), peak)
 
-    cpu = None
+    cpu = parity = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        cpu = oracle_sample(batch, lengths_np, args.cpu_seconds)
+        cpu, parity = oracle_leg(batch, lengths_np, results, args.cpu_seconds,
+                                 args.cpu_1core_seconds, args.parity_seconds,
+                                 row_base=row_base)
 
     if rank == 0:
         out = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
@@ -556,7 +660,8 @@ def run_ours(args, rank, world, local_rank):
                               parallelism=f"dp{world} (row shards, no collective)"),
                "e2e": e2e, "gpu_launches": args.steps * (sv.sv_verify_launches()
                                                          + (1 if fixed is None else 0)),
-               "roofline": roofline, "cpu_baseline": cpu, "clocks": clk, "schedule": sched,
+               "roofline": roofline, "cpu_baseline": cpu, "parity": parity, "clocks": clk,
+               "schedule": sched,
                "admission": admit,
                "calibration": calib, "vocab_parallel": vocab,
                "device_status": st, "impl": "ours"}
@@ -571,7 +676,7 @@ def run_reference(args, rank, world):
     one bounded pass over a row sample of the same workload."""
     if rank != 0:
         return
-    batch = workloads.make_batch(args.workload, device="cpu")
+    batch = workloads.make_batch(args.workload, device="cpu", tau=args.tau)
     s = batch.spec
     import oracle
     from speculative_decoding_verification_93_b200.workloads import to_host_logits
@@ -579,7 +684,7 @@ def run_reference(args, rank, world):
         lengths_np, _, _ = oracle.schedule(batch.conf.numpy(), batch.tau)
     else:
         lengths_np = batch.lengths.numpy()
-    rows = np.arange(min(s.B, args.ref_rows))
+    rows = np.arange(s.B if args.ref_rows <= 0 else min(s.B, args.ref_rows))
     zt = to_host_logits(batch.zt[: len(rows)])
     zd = to_host_logits(batch.zd[: len(rows)])
     tok = batch.tokens[: len(rows)].numpy()
@@ -596,7 +701,8 @@ def run_reference(args, rank, world):
     positions = int(ln.sum())
     value = positions * args.steps / el
     esize = 2 if s.dtype == torch.bfloat16 else 4
-    sample = f"rows 0..{len(rows) - 1} of the {s.B}-row batch per step"
+    sample = (f"the whole {s.B}-row batch per step" if len(rows) == s.B else
+              f"rows 0..{len(rows) - 1} of the {s.B}-row batch per step")
     out = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup,
            "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
@@ -626,8 +732,14 @@ def main():
     ap.add_argument("--clock-load-s", type=float, default=0.5,
                     help="seconds of untimed steps before the timed region, so the clock "
                          "sampler sees load (0 under a profiler)")
+    ap.add_argument("--tau", type=float, default=None,
+                    help="schedule threshold for workloads with scheduled lengths "
+                         "(default: the workload's first)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--ref-rows", type=int, default=64)
+    ap.add_argument("--cpu-1core-seconds", type=float, default=5.0)
+    ap.add_argument("--parity-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-rows", type=int, default=0,
+                    help="rows of the batch the reference arm verifies per step (0: all)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -299,9 +299,10 @@ sv_status sv_verify_debug(const void *target_logits, const void *draft_logits, s
  *   exceeds 16 MiB (16777216 bytes) are rejected with SV_ERR_WORKSPACE
  *   before anything is launched; use sv_verify with a workspace for those.
  *   The library calls no cudaMalloc, cudaFree or other allocating routine.
- *   The first call on a device looks up the array's device address (once
- *   per device, thread-safe); make that first call before any stream
- *   capture.  Every call shares the one array and leaves its contents
+ *   Each call looks up the array's device address on the current device
+ *   (cudaGetSymbolAddress), so the address stays right after the device's
+ *   context is reset; the first call on a device may load the library's
+ *   device code, so make it before any stream capture.  Every call shares the one array and leaves its contents
  *   behind: counters that must start at zero are reset by each call's
  *   first kernel, everything else is written before it is read.  Calls
  *   whose work overlaps on the GPU (other streams, other host threads on the

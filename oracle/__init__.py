@@ -29,6 +29,16 @@ from . import build as _build
 F32, BF16, F64 = 0, 1, 2
 NDIAG = 5
 
+# Tie windows for comparing an fp32 implementation with this fp64 oracle.
+# An accept test with |u - min(1, ratio)| below ACCEPT_WINDOW may go either
+# way.  A final draw may land on any token its target reaches when moved by
+# up to CDF_WINDOW * R (the same bound, read onto the inverse CDF).  A
+# survival product with |S_i - tau| below SCHEDULE_WINDOW may keep or drop
+# position i (fp32 products against fp64).
+ACCEPT_WINDOW = 1e-5
+CDF_WINDOW = 1e-5
+SCHEDULE_WINDOW = 1e-6
+
 _lib = None
 
 
@@ -50,6 +60,12 @@ def lib():
         L.oracle_verify.argtypes = [vp, vp, i32, i64, i32, i32, vp, vp, vp, u64, i64, vp,
                                     vp, vp, vp, i32]
         L.oracle_verify.restype = i32
+        L.oracle_verify_window.argtypes = [vp, vp, i32, i64, i32, i32, vp, vp, vp, u64, i64,
+                                           vp, dbl, dbl, vp, i32]
+        L.oracle_verify_window.restype = i32
+        L.oracle_verify_window_row_u.argtypes = [vp, vp, i32, i32, vp, i32, dbl, vp, vp, dbl,
+                                                 dbl, vp]
+        L.oracle_verify_window_row_u.restype = i32
         L.oracle_stats_batch.argtypes = [vp, i32, i64, i32, vp, vp, vp, vp, i32]
         L.oracle_stats_batch.restype = None
         L.oracle_schedule.argtypes = [vp, i64, i32, dbl, vp, vp]
@@ -151,6 +167,54 @@ def verify(zt, zd, tokens, lengths, temperature, seed, row_base=0, row_ids=None,
                              ctypes.c_uint64(seed & (2**64 - 1)), int(row_base), _p(rid),
                              _p(out), _p(acc), _p(diag), int(nthreads))
     return out, acc, diag, st
+
+
+def verify_window(zt, zd, tokens, lengths, temperature, seed, w_acc=ACCEPT_WINDOW,
+                  w_cdf=CDF_WINDOW, row_base=0, row_ids=None, nthreads=0):
+    """Every outcome the rule allows when each accept test may flip within
+    w_acc of its threshold and each final draw may move within w_cdf * R of
+    its target (see oracle_verify_window in oracle.c).
+
+    Same inputs as :func:`verify`.  Returns (alt [B, K+1, 4] int32 of
+    (a, y, lo, hi) per reachable accepted length a, in increasing a, padded
+    with -1; status bits)."""
+    zt = np.ascontiguousarray(zt)
+    B, K1, V = zt.shape
+    K = K1 - 1
+    dt = _dtype_code(zt)
+    if zd is not None:
+        zd = np.ascontiguousarray(zd)
+        assert zd.shape == (B, K, V) and zd.dtype == zt.dtype
+    tok = np.ascontiguousarray(tokens, dtype=np.int32).reshape(B, K)
+    ln = np.ascontiguousarray(lengths, dtype=np.int32).reshape(B)
+    tp = np.ascontiguousarray(temperature, dtype=np.float32).reshape(B)
+    rid = None if row_ids is None else np.ascontiguousarray(row_ids, dtype=np.int64).reshape(B)
+    alt = np.zeros((B, K + 1, 4), dtype=np.int32)
+    st = lib().oracle_verify_window(_p(zt), _p(zd), dt, B, K, V, _p(tok), _p(ln), _p(tp),
+                                    ctypes.c_uint64(seed & (2**64 - 1)), int(row_base), _p(rid),
+                                    float(w_acc), float(w_cdf), _p(alt), int(nthreads))
+    if st < 0:
+        raise ValueError("oracle_verify_window: bad arguments")
+    return alt, st
+
+
+def verify_window_row_u(zt, zd, x, L, T, u_acc, u_res, w_acc, w_cdf):
+    """One row of :func:`verify_window` with fp64 logits and injected
+    uniforms (zt [K+1, V], zd [K, V] or None).  Returns alt [K+1, 4]."""
+    zt = np.ascontiguousarray(zt, dtype=np.float64)
+    K1, V = zt.shape
+    K = K1 - 1
+    zd_a = None if zd is None else np.ascontiguousarray(zd, dtype=np.float64)
+    x = np.ascontiguousarray(x, dtype=np.int32).reshape(K)
+    ua = np.ascontiguousarray(u_acc, dtype=np.float64).reshape(-1)
+    ur = np.ascontiguousarray(u_res, dtype=np.float64).reshape(-1)
+    assert ua.size >= K + 1 and ur.size >= K + 1
+    alt = np.zeros((K + 1, 4), dtype=np.int32)
+    r = lib().oracle_verify_window_row_u(_p(zt), _p(zd_a), K, V, _p(x), int(L), float(T),
+                                         _p(ua), _p(ur), float(w_acc), float(w_cdf), _p(alt))
+    if r < 0:
+        raise ValueError("oracle_verify_window_row_u: bad arguments")
+    return alt
 
 
 def stats(z, temperature, nthreads=0):

@@ -65,6 +65,9 @@
 
 enum { OR_F32 = 0, OR_BF16 = 1, OR_F64 = 2 };
 
+/* Largest number of drafts per row the window enumeration handles. */
+#define OR_MAX_K 64
+
 /* ---------------------------------------------------------------------------
  * Philox4x32-10 [SC11].  One round: two 32x32->64 multiplications of the
  * even words by the round multipliers; the high halves are XORed with the
@@ -403,6 +406,190 @@ int oracle_verify(const void *zt, const void *zd, int dtype, int64_t B, int K, i
         free(work); free(u_acc); free(u_res);
     }
     return status;
+}
+
+/* ---------------------------------------------------------------------------
+ * Tie windows: every outcome the rule allows when floating point may move
+ * each decision by a small amount.
+ *
+ * The fp32 kernels and this fp64 oracle can legitimately disagree on a
+ * decision that sits within rounding of its threshold.  Two kinds exist:
+ *  - an accept test with |u_i - min(1, ratio_i)| < w_acc, which either side
+ *    may take as accept or reject;
+ *  - a final draw whose target t = u * R lies within w_cdf * R of a CDF
+ *    boundary, where either side may land on a neighbouring token.
+ * Instead of excluding such rows, this function lists every outcome that
+ * decisions inside those windows can reach, so that a result can be checked
+ * to be one of them.
+ *
+ * Per row (T > 0), the tested positions are walked in order exactly as in
+ * verify_row: a position whose test lies inside the accept window can end
+ * the row there (a rejection) or let it go on (an acceptance); a position
+ * outside the window takes its own decision; a clear rejection ends the
+ * walk; reaching L leaves the bonus.  For every reachable accepted length a
+ * the final draw is made as in verify_row (residual max(0, p_a - q_a), the
+ * p_a fallback when that is zero, or p_L for the bonus) at three targets:
+ * u, max(0, u - w_cdf) and u + w_cdf (scaled by R), which give y, lo and hi.
+ * The CDF is monotone in the target, so every token a draw inside the window
+ * can return lies in [lo, hi].  Greedy rows (T == 0) have one outcome, as in
+ * verify_row, with lo = hi = y: their decisions are exact comparisons.
+ *
+ * alt [B, K+1, 4] int32 receives (a, y, lo, hi) per reachable a in
+ * increasing a, then rows of -1.  Invalid rows get -1 everywhere and their
+ * status bits, as in oracle_verify.  With w_acc = w_cdf = 0 the list holds
+ * the single outcome of oracle_verify.
+ * ------------------------------------------------------------------------- */
+#define OR_NALT 4
+
+/* Draw weights of the final token at position j into r[0..V): residual
+ * max(0, p_j - q_j) after a rejection at j < L (p_j when that has no mass),
+ * p_L when every draft survived (j == L).  Returns 1 if the zero-residual
+ * fallback was taken. */
+static int draw_weights(vec_t zt_row, const void *zd_base, int dtype, int V, int j, int L,
+                        const int32_t *x, double T, double *r)
+{
+    vec_t zt = vec_at(zt_row.p, dtype, j, V);
+    double mt, st;
+    softmax_stats(zt, V, T, &mt, &st);
+    if (j == L) {
+        for (int v = 0; v < V; ++v) r[v] = exp((zval(zt, v) - mt) / T) / st;
+        return 0;
+    }
+    double md = 0.0, sd = 1.0;
+    vec_t zd = { NULL, dtype };
+    if (zd_base) {
+        zd = vec_at(zd_base, dtype, j, V);
+        softmax_stats(zd, V, T, &md, &sd);
+    }
+    double R = 0.0;
+    for (int v = 0; v < V; ++v) {
+        double p = exp((zval(zt, v) - mt) / T) / st;
+        double q = zd_base ? exp((zval(zd, v) - md) / T) / sd : (v == x[j] ? 1.0 : 0.0);
+        r[v] = p - q > 0.0 ? p - q : 0.0;
+        R += r[v];
+    }
+    if (R == 0.0) {
+        for (int v = 0; v < V; ++v) r[v] = exp((zval(zt, v) - mt) / T) / st;
+        return 1;
+    }
+    return 0;
+}
+
+static void verify_row_window(vec_t zt_row, const void *zd_base, int dtype, int K, int V,
+                              const int32_t *x, int L, double T, const double *u_acc,
+                              const double *u_res, double w_acc, double w_cdf,
+                              int32_t *alt, double *work)
+{
+    for (int q = 0; q < (K + 1) * OR_NALT; ++q) alt[q] = -1;
+    if (T == 0.0) {
+        int j = L;
+        for (int i = 0; i < L; ++i)
+            if (x[i] != argmax_first(vec_at(zt_row.p, dtype, i, V), V)) { j = i; break; }
+        int y = argmax_first(vec_at(zt_row.p, dtype, j, V), V);
+        alt[0] = j; alt[1] = y; alt[2] = y; alt[3] = y;
+        return;
+    }
+    int n = 0;
+    int ends[OR_MAX_K + 1];
+    int stopped = 0;
+    for (int i = 0; i < L; ++i) {
+        vec_t zt = vec_at(zt_row.p, dtype, i, V);
+        double mt, st;
+        softmax_stats(zt, V, T, &mt, &st);
+        double logp = (zval(zt, x[i]) - mt) / T - log(st);
+        double logq = 0.0;
+        if (zd_base) {
+            vec_t zd = vec_at(zd_base, dtype, i, V);
+            double md, sd;
+            softmax_stats(zd, V, T, &md, &sd);
+            logq = (zval(zd, x[i]) - md) / T - log(sd);
+        }
+        double acc;
+        if (logp == -INFINITY) acc = 0.0;
+        else if (logq == -INFINITY) acc = 1.0;
+        else acc = logp >= logq ? 1.0 : exp(logp - logq);
+        if (fabs(u_acc[i] - acc) < w_acc) {
+            ends[n++] = i;          /* may reject here, or accept and go on */
+            continue;
+        }
+        if (u_acc[i] < acc) continue;
+        ends[n++] = i;              /* clear rejection: the walk ends */
+        stopped = 1;
+        break;
+    }
+    if (!stopped) ends[n++] = L;
+    for (int k = 0; k < n; ++k) {
+        int j = ends[k];
+        draw_weights(zt_row, zd_base, dtype, V, j, L, x, T, work);
+        double mg;
+        int fb;
+        double ulo = u_res[j] - w_cdf;
+        if (ulo < 0.0) ulo = 0.0;
+        alt[k * OR_NALT + 0] = j;
+        alt[k * OR_NALT + 1] = inverse_cdf(work, V, u_res[j], &mg, &fb);
+        alt[k * OR_NALT + 2] = inverse_cdf(work, V, ulo, &mg, &fb);
+        alt[k * OR_NALT + 3] = inverse_cdf(work, V, u_res[j] + w_cdf, &mg, &fb);
+    }
+}
+
+int oracle_verify_window(const void *zt, const void *zd, int dtype, int64_t B, int K, int V,
+                         const int32_t *tokens, const int32_t *lengths,
+                         const float *temperature, uint64_t seed, int64_t row_base,
+                         const int64_t *row_ids, double w_acc, double w_cdf, int32_t *alt,
+                         int nthreads)
+{
+    int status = 0;
+    if (K > OR_MAX_K) return -1;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+#pragma omp parallel reduction(| : status)
+    {
+        double *work = (double *)malloc(sizeof(double) * (size_t)V);
+        double *u_acc = (double *)malloc(sizeof(double) * (size_t)(K + 1));
+        double *u_res = (double *)malloc(sizeof(double) * (size_t)(K + 1));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t b = 0; b < B; ++b) {
+            const int32_t *x = tokens + b * K;
+            int L = lengths[b];
+            float T = temperature[b];
+            int32_t *ab = alt + b * (int64_t)(K + 1) * OR_NALT;
+            int bits = row_errors(K, V, x, L, T);
+            if (bits) {
+                status |= bits;
+                for (int q = 0; q < (K + 1) * OR_NALT; ++q) ab[q] = -1;
+                continue;
+            }
+            uint64_t row = row_ids ? (uint64_t)row_ids[b] : (uint64_t)(row_base + b);
+            for (int i = 0; i <= K; ++i) {
+                u_acc[i] = oracle_uniform(seed, row, (uint32_t)i, 0);
+                u_res[i] = oracle_uniform(seed, row, (uint32_t)i, 1);
+            }
+            vec_t zr = vec_at(zt, dtype, b * (K + 1), V);
+            const void *zdr = zd ? vec_at(zd, dtype, b * K, V).p : NULL;
+            verify_row_window(zr, zdr, dtype, K, V, x, L, (double)T, u_acc, u_res, w_acc,
+                              w_cdf, ab, work);
+        }
+        free(work); free(u_acc); free(u_res);
+    }
+    return status;
+}
+
+/* Single row with fp64 logits and injected uniforms (for the pins). */
+int oracle_verify_window_row_u(const double *zt, const double *zd, int K, int V,
+                               const int32_t *x, int L, double T, const double *u_acc,
+                               const double *u_res, double w_acc, double w_cdf, int32_t *alt)
+{
+    if (K < 0 || K > OR_MAX_K || V <= 0 || L < 0 || L > K || !(T >= 0.0)) return -1;
+    for (int i = 0; i < L; ++i) if (x[i] < 0 || x[i] >= V) return -1;
+    double *work = (double *)malloc(sizeof(double) * (size_t)V);
+    if (!work) return -1;
+    vec_t zr = { zt, OR_F64 };
+    verify_row_window(zr, zd, OR_F64, K, V, x, L, T, u_acc, u_res, w_acc, w_cdf, alt, work);
+    free(work);
+    return 0;
 }
 
 /* Normaliser export: for every vector of a [n, V] array, m and Sigma at the

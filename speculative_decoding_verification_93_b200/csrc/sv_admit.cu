@@ -25,6 +25,7 @@
 // minimum for the first k at which f stops rising.
 #include <cfloat>
 #include <climits>
+#include <atomic>
 #include <cstdint>
 
 #include <cub/block/block_radix_sort.cuh>
@@ -159,15 +160,16 @@ template <int THREADS, int ITEMS>
 static sv_status launch_admit(const float *conf, int B, int K, const float *speed, int n_speed,
                               int32_t *lengths, float *tau_out, cudaStream_t st) {
     constexpr size_t smem = sizeof(typename sv::AdmitSort<THREADS, ITEMS>::Storage);
-    static bool attr_set[64];
+    // Set once per device; threads that race on it set the same value.
+    static std::atomic<bool> attr_set[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return sv::note_cuda(e);
-    if (!attr_set[dev & 63]) {
+    if (!attr_set[dev & 63].load(std::memory_order_acquire)) {
         e = cudaFuncSetAttribute(sv::admit_kernel<THREADS, ITEMS>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (e != cudaSuccess) return sv::note_cuda(e);
-        attr_set[dev & 63] = true;
+        attr_set[dev & 63].store(true, std::memory_order_release);
     }
     return sv::note_cuda(sv::launch_pdl(sv::admit_kernel<THREADS, ITEMS>, dim3(1), dim3(THREADS), smem, st,
                                         conf, B, K, speed, n_speed, lengths, tau_out));
@@ -175,7 +177,8 @@ static sv_status launch_admit(const float *conf, int B, int K, const float *spee
 
 extern "C" sv_status sv_schedule_admit(const float *conf, int B, int K, const float *speed,
                                        int n_speed, int32_t *lengths, float *tau_out,
-                                       void *stream) {
+                                       void *stream) {    sv::NvtxRange nvtx_range("sv_schedule_admit");
+
     if (!conf || !speed || !lengths) return SV_ERR_ARG;
     if (B < 1 || K < 1 || K > SV_MAX_K || static_cast<long long>(B) * K > sv::kAdmitMax ||
         n_speed < 1)

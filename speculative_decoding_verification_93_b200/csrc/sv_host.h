@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "sv.h"
 
@@ -28,6 +29,16 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
+
+// NVTX range over one library call, named after the entry point, so that a
+// profiler timeline shows which call issued which kernels.  Header-only
+// NVTX: without a profiler attached each push and pop returns at once.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 // Optional CUDA events around the main verification kernel (benchmarks).
 void profile_mark_begin(cudaStream_t st);

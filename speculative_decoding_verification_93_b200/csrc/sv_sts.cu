@@ -325,7 +325,8 @@ extern "C" size_t sv_sts_workspace_bytes(int N, int K) {
 
 extern "C" sv_status sv_sts_fit(const float *logits, const int32_t *accept_len, int N, int K,
                                 float tmin, float tmax, float *temperature, float *ece,
-                                void *workspace, size_t workspace_bytes, void *stream) {
+                                void *workspace, size_t workspace_bytes, void *stream) {    sv::NvtxRange nvtx_range("sv_sts_fit");
+
     if (!logits || !accept_len || !temperature || !workspace) return SV_ERR_ARG;
     if (!(tmin > 0.f) || !(tmax > tmin) || !std::isfinite(tmax)) return SV_ERR_ARG;
     sv::StsPlan p;
@@ -373,7 +374,8 @@ extern "C" sv_status sv_sts_fit(const float *logits, const int32_t *accept_len, 
 }
 
 extern "C" sv_status sv_sts_apply(const float *logits, const float *temperature, int N, int K,
-                                  float *conf_out, void *stream) {
+                                  float *conf_out, void *stream) {    sv::NvtxRange nvtx_range("sv_sts_apply");
+
     if (!logits || !temperature || !conf_out) return SV_ERR_ARG;
     if (N < 1 || K < 1 || K > SV_MAX_K) return SV_ERR_SHAPE;
     const long long total = static_cast<long long>(N) * K;

@@ -50,7 +50,7 @@
 #include <climits>
 #include <cstdint>
 #include <cstdio>
-#include <mutex>
+#include <atomic>
 
 #include "sv.h"
 #include "sv_device.cuh"
@@ -1621,12 +1621,16 @@ static bool make_plan(int B, int K, int V, sv_dtype dtype, Plan *p) {
     return true;
 }
 
+// Persistent grid of the stream kernel: resident CTAs per SM x SMs, cached
+// per (dtype, device).  Threads that race on an empty entry compute the
+// same value; the entry is an atomic so each reads a whole one.
 static int stream_grid(int esize, long long max_items) {
-    static int cache[2][64];
+    static std::atomic<int> cache[2][64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return -1;
-    int &slot = cache[esize == 4 ? 1 : 0][dev & 63];
-    if (slot == 0) {
+    std::atomic<int> &slot = cache[esize == 4 ? 1 : 0][dev & 63];
+    int n = slot.load(std::memory_order_relaxed);
+    if (n == 0) {
         int sms = 0, per = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return -1;
@@ -1637,9 +1641,10 @@ static int stream_grid(int esize, long long max_items) {
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fn, kBlock, kRingBytes) !=
             cudaSuccess)
             return -1;
-        slot = sms * (per > 0 ? per : 1);
+        n = sms * (per > 0 ? per : 1);
+        slot.store(n, std::memory_order_relaxed);
     }
-    return static_cast<int>(max_items < slot ? max_items : slot);
+    return static_cast<int>(max_items < n ? max_items : n);
 }
 
 static sv_status verify_impl(const void *zt, const void *zd, sv_dtype dtype, int B, int K, int V,
@@ -1722,7 +1727,8 @@ extern "C" sv_status sv_verify(const void *target_logits, const void *draft_logi
                                const int32_t *lengths, const float *temperature, uint64_t seed,
                                int64_t row_base, int32_t *out_tokens, int32_t *out_accept_len,
                                void *workspace, size_t workspace_bytes, int32_t *status,
-                               void *stream) {
+                               void *stream) {    sv::NvtxRange nvtx_range("sv_verify");
+
     return sv::verify_impl(target_logits, draft_logits, dtype, B, K, V, draft_tokens, lengths,
                            temperature, seed, row_base, out_tokens, out_accept_len, workspace,
                            workspace_bytes, status, nullptr, stream);
@@ -1734,7 +1740,8 @@ extern "C" sv_status sv_verify_debug(const void *target_logits, const void *draf
                                      const float *temperature, uint64_t seed, int64_t row_base,
                                      int32_t *out_tokens, int32_t *out_accept_len,
                                      void *workspace, size_t workspace_bytes, int32_t *status,
-                                     float *stats_out, void *stream) {
+                                     float *stats_out, void *stream) {    sv::NvtxRange nvtx_range("sv_verify_debug");
+
     if (!stats_out) return SV_ERR_ARG;
     return sv::verify_impl(target_logits, draft_logits, dtype, B, K, V, draft_tokens, lengths,
                            temperature, seed, row_base, out_tokens, out_accept_len, workspace,
@@ -1754,25 +1761,18 @@ namespace sv {
 constexpr size_t kStaticScratchBytes = size_t(16) << 20;   // 16 MiB per device
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
-static std::mutex g_static_scratch_mu;
-static void *g_static_scratch_addr[64];
-
 // Device address of g_static_scratch on the current device.  In host code
 // the symbol names only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
+// with the device current.  It is looked up on every call (a cheap table
+// lookup in the runtime), so that it stays right when the device's context
+// is torn down and created again (cudaDeviceReset reloads the module and
+// may move the array).  The first lookup on a device may load the module.
 static sv_status static_scratch_address(void **out) {
-    int dev = 0;
-    const cudaError_t e0 = cudaGetDevice(&dev);
-    if (e0 != cudaSuccess) return note_cuda(e0);
-    if (dev < 0 || dev >= 64) return SV_ERR_ARG;
-    std::lock_guard<std::mutex> lock(g_static_scratch_mu);
-    if (g_static_scratch_addr[dev] == nullptr) {
-        void *p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
-        if (e != cudaSuccess || p == nullptr) return note_cuda(e != cudaSuccess ? e : cudaErrorUnknown);
-        g_static_scratch_addr[dev] = p;
-    }
-    *out = g_static_scratch_addr[dev];
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return note_cuda(e);
+    if (p == nullptr) return note_cuda(cudaErrorUnknown);
+    *out = p;
     return SV_OK;
 }
 
@@ -1783,7 +1783,8 @@ extern "C" sv_status sv_verify_noalloc(const void *target_logits, const void *dr
                                        const int32_t *draft_tokens, const int32_t *lengths,
                                        const float *temperature, uint64_t seed, int64_t row_base,
                                        int32_t *out_tokens, int32_t *out_accept_len,
-                                       int32_t *status, void *stream) {
+                                       int32_t *status, void *stream) {    sv::NvtxRange nvtx_range("sv_verify_noalloc");
+
     if (!target_logits || !draft_tokens || !lengths || !temperature || !out_tokens ||
         !out_accept_len)
         return SV_ERR_ARG;

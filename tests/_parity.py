@@ -1,13 +1,14 @@
 """Helpers for GPU-vs-oracle parity: run both sides on the same seeded
-inputs and compare element by element.
+inputs and compare row by row.
 
-Tie windows (decisions that floating point may legitimately flip between the
-fp32 kernels and the fp64 oracle) are taken from the oracle's own
-diagnostics, never from the GPU: a row is excluded when one of its tested
-positions has |u - min(1, ratio)| < 1e-5, when its final draw lies within
-1e-5 * R of a CDF boundary, or when a survival product lies within 1e-6 of
-tau.  Excluded rows are counted and returned; everything else must match bit
-for bit.
+Every row is checked; none is excluded.  A row must either equal the
+oracle's own result bit for bit, or be one of the outcomes the oracle lists
+for decisions that lie inside the tie windows (``oracle.verify_window``):
+an accept test with |u - min(1, ratio)| < 1e-5 may go either way, a final
+draw may land on any token its target reaches within 1e-5 * R, and a
+survival product within 1e-6 of tau may keep or drop its position.  The
+outcome sets come from the oracle alone; the GPU result is only checked for
+membership (``oracle.compare``).
 """
 from __future__ import annotations
 
@@ -15,12 +16,13 @@ import numpy as np
 import torch
 
 import oracle
+from oracle import compare as ocompare
 import speculative_decoding_verification_93_b200 as sv
 from speculative_decoding_verification_93_b200.workloads import to_host_logits
 
-ACCEPT_TIE = 1e-5
-CDF_TIE = 1e-5
-SCHEDULE_TIE = 1e-6
+ACCEPT_TIE = oracle.ACCEPT_WINDOW
+CDF_TIE = oracle.CDF_WINDOW
+SCHEDULE_TIE = oracle.SCHEDULE_WINDOW
 
 
 def gpu_verify(zt, zd, tokens, lengths, temperature, seed, row_base=0, debug=False,
@@ -75,32 +77,61 @@ def oracle_verify(zt, zd, tokens, lengths_np, temperature, seed, rows=None, row_
         tmp = temperature.cpu().numpy()
         ln = np.asarray(lengths_np)
         rid = None
+    nt = oracle.default_threads()
     out, acc, diag, st = oracle.verify(zt_h, zd_h, tok, ln, tmp, seed, row_base=row_base,
-                                       row_ids=rid, nthreads=oracle.default_threads())
-    return dict(tokens=out, accept=acc, diag=diag, status=st)
+                                       row_ids=rid, nthreads=nt)
+    alt, _ = oracle.verify_window(zt_h, zd_h, tok, ln, tmp, seed, row_base=row_base,
+                                  row_ids=rid, nthreads=nt)
+    return dict(tokens=out, accept=acc, diag=diag, status=st, alt=alt, x=tok, lengths=ln)
 
 
-def compare(g, o, rows=None, extra_excluded=None):
-    """Element-by-element comparison; returns counts.  Raises on a mismatch
-    outside the tie windows."""
+def compare(g, o, rows=None):
+    """Row-by-row check of a GPU result against the oracle result ``o`` (from
+    :func:`oracle_verify`, same lengths on both sides).  Raises unless every
+    row is bit-exact or one of the oracle's tie-window outcomes.  Returns the
+    counts: rows, bit_exact, window_valid (rows that differ from the oracle's
+    own result but lie inside a window), ties (rows with any window)."""
     gt = g["tokens"] if rows is None else g["tokens"][rows]
     ga = g["accept"] if rows is None else g["accept"][rows]
-    diag = o["diag"]
-    tie = np.zeros(len(ga), dtype=bool)
-    with np.errstate(invalid="ignore"):
-        tie |= diag[:, 0] < ACCEPT_TIE
-        tie |= diag[:, 1] < CDF_TIE
-    if extra_excluded is not None:
-        tie |= extra_excluded
-    same = (ga == o["accept"]) & np.all(gt == o["tokens"], axis=1)
-    bad = ~same & ~tie
-    if bad.any():
-        r = int(np.flatnonzero(bad)[0])
-        raise AssertionError(
-            f"{int(bad.sum())} rows differ outside the tie windows; first row {r}: "
-            f"gpu a={ga[r]} tokens={gt[r].tolist()} oracle a={o['accept'][r]} "
-            f"tokens={o['tokens'][r].tolist()} diag={diag[r].tolist()}")
-    return dict(rows=len(ga), ties=int(tie.sum()), tie_mismatches=int((~same & tie).sum()))
+    alt = o["alt"]
+    n = len(ga)
+    alts = [[tuple(r) for r in alt[q] if r[0] >= 0] for q in range(n)]
+    L = np.asarray(o["lengths"])
+    t = ocompare.classify(np.arange(n) if rows is None else np.asarray(rows), o["x"],
+                          o["tokens"], o["accept"], alt, alts, L, L, L, L, gt, ga)
+    if t.invalid:
+        raise AssertionError(f"{t.invalid} rows are neither bit-exact nor inside a tie window; "
+                             f"first: {t.first_invalid}")
+    ties = sum(1 for q in range(n) if len(alts[q]) > 1 or any(r[2] != r[3] for r in alts[q]))
+    return dict(rows=n, bit_exact=t.bit_exact, window_valid=t.window_valid, ties=ties,
+                tie_mismatches=t.window_valid)
+
+
+def check_batch(batch, ln_gpu, g, seed, rows=None, row_base=0):
+    """Complete check of a GPU verification of ``batch`` whose lengths came
+    from ``sv_schedule`` (or are fixed): the oracle schedules on its own (rows
+    whose survival product sits within the schedule window may take either
+    length), then every row in ``rows`` (default all) must be bit-exact or a
+    tie-window outcome.  Logits are copied to the host in row blocks."""
+    tok = batch.tokens.cpu().numpy()
+    tmp = batch.temperature.cpu().numpy()
+    if batch.lengths is None:
+        L0, lo, hi = ocompare.schedule_span(batch.conf.cpu().numpy(), batch.tau)
+    else:
+        L0 = batch.lengths.cpu().numpy()
+        lo = hi = L0
+
+    def fetch(idx):
+        ix = torch.as_tensor(idx, device=batch.zt.device, dtype=torch.long)
+        zd = None if batch.zd is None else to_host_logits(batch.zd.index_select(0, ix))
+        return to_host_logits(batch.zt.index_select(0, ix)), zd
+
+    t = ocompare.check_rows(fetch, tok, tmp, seed, L0, lo, hi, ln_gpu.cpu().numpy(),
+                            g["tokens"], g["accept"], rows=rows, row_base=row_base)
+    if t.invalid:
+        raise AssertionError(f"{t.invalid} rows are neither bit-exact nor inside a tie window; "
+                             f"first: {t.first_invalid}")
+    return t.summary()
 
 
 def check_structure(g, tokens_np, lengths_np):

@@ -40,3 +40,29 @@ def test_code_only_ignores_comments_and_layout_but_not_code():
     assert bench.code_only(src.replace("// one", "// uno")) == bench.code_only(src)
     assert bench.code_only(src.replace("a = 1", "a = 2")) != bench.code_only(src)
     assert bench.code_only("char c = '\\'';  // x") == "charc='\\'';"
+
+
+def test_committed_traffic_needs_the_current_kernel_hash(tmp_path, monkeypatch):
+    p = tmp_path / "t.json"
+    p.write_text('{"kernel_source_hash": "%s", "workloads": {"c2": '
+                 '{"dram_bytes_per_launch": 123}}}' % bench.kernel_hash())
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(p))
+    assert bench.committed_traffic("c2") == 123.0
+    assert bench.committed_traffic("c3") is None
+    p.write_text('{"kernel_source_hash": "0000", "workloads": {"c2": '
+                 '{"dram_bytes_per_launch": 123}}}')
+    assert bench.committed_traffic("c2") is None
+
+
+def test_l2_flush_only_for_inputs_near_the_l2_size():
+    from types import SimpleNamespace
+    import torch
+    small = SimpleNamespace(zt=torch.empty(4, 5, 1000), zd=torch.empty(4, 4, 1000))
+    big = SimpleNamespace(zt=torch.empty(1, 1, 1), zd=torch.empty(1, 1, 1))
+    big.zt = SimpleNamespace(numel=lambda: 64 * 5 * 129280)
+    big.zd = SimpleNamespace(numel=lambda: 64 * 4 * 129280)
+    assert bench.needs_flush(small, 4)            # c0: 0.14 MB
+    assert bench.needs_flush(big, 2)              # c1: 149 MB < 252 MB
+    big.zt = SimpleNamespace(numel=lambda: 256 * 9 * 129280)
+    big.zd = SimpleNamespace(numel=lambda: 256 * 8 * 129280)
+    assert not bench.needs_flush(big, 2)          # c2: 1.1 GB
