@@ -182,6 +182,24 @@ sv_status sv_sts_apply(const float *logits, const float *temperature, int N, int
                        float *conf_out, void *stream);
 
 /*
+ * Test exports for the bounded wait of sv_sts_fit's grid barrier (no
+ * counterpart on the pages: they exist so that the failure path of a wait
+ * can be exercised without hanging or faulting a GPU).
+ *
+ * sv_debug_sts_wait_limit -- wall-time limit, in ns, of one barrier wait of
+ *   the calibration kernel on the current device; 0 restores the default
+ *   (1 s).  With a limit near zero the fit gives up at its first barrier:
+ *   sv_sts_fit still returns SV_OK, the temperatures come out NaN and ECE is
+ *   left unwritten.  Affects later launches only; not thread-safe against
+ *   fits in flight.  Returns SV_OK or SV_ERR_CUDA.
+ * sv_debug_sts_timeouts -- the number of barrier waits on the current device
+ *   that ran out since the previous call (then cleared); -1 on a CUDA error.
+ *   Synchronous (it copies from device memory).
+ */
+sv_status sv_debug_sts_wait_limit(uint64_t limit_ns);
+int sv_debug_sts_timeouts(void);
+
+/*
  * sv_verify_workspace_bytes -- device scratch that sv_verify needs for
  * (B, K, V, dtype): work counters, per-row state (length, first rejection
  * found so far, per-position completion counts), the position-major work

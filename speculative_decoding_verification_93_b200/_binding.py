@@ -51,6 +51,10 @@ def lib():
     L.sv_sts_fit.argtypes = [vp, vp, i32, i32, ctypes.c_float, ctypes.c_float, vp, vp, vp, sz,
                              vp]
     L.sv_sts_apply.argtypes = [vp, vp, i32, i32, vp, vp]
+    L.sv_debug_sts_wait_limit.argtypes = [u64]
+    L.sv_debug_sts_wait_limit.restype = i32
+    L.sv_debug_sts_timeouts.argtypes = []
+    L.sv_debug_sts_timeouts.restype = i32
     L.sv_verify_workspace_bytes.argtypes = [i32, i32, i32, i32]
     L.sv_verify_workspace_bytes.restype = sz
     L.sv_verify.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, u64, i64, vp, vp, vp, sz, vp,
@@ -193,6 +197,20 @@ def sv_sts_apply(logits: torch.Tensor, temperature: torch.Tensor, conf_out: torc
     N, K = logits.shape
     _check("sv_sts_apply", lib().sv_sts_apply(_ptr(logits), _ptr(temperature), N, K,
                                               _ptr(conf_out), _stream(stream, logits)))
+
+
+def sv_debug_sts_wait_limit(limit_ns: int) -> None:
+    """Test export: wall-time limit of the calibration barrier's wait on the
+    current device (0 restores the 1 s default)."""
+    _check("sv_debug_sts_wait_limit", lib().sv_debug_sts_wait_limit(int(limit_ns)))
+
+
+def sv_debug_sts_timeouts() -> int:
+    """Test export: barrier waits that ran out since the previous call."""
+    n = lib().sv_debug_sts_timeouts()
+    if n < 0:
+        raise SVError("sv_debug_sts_timeouts", 5)
+    return n
 
 
 def sv_verify_workspace_bytes(B: int, K: int, V: int, dtype: int) -> int:

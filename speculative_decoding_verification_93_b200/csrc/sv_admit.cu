@@ -177,8 +177,8 @@ static sv_status launch_admit(const float *conf, int B, int K, const float *spee
 
 extern "C" sv_status sv_schedule_admit(const float *conf, int B, int K, const float *speed,
                                        int n_speed, int32_t *lengths, float *tau_out,
-                                       void *stream) {    sv::NvtxRange nvtx_range("sv_schedule_admit");
-
+                                       void *stream) {
+    sv::NvtxRange nvtx_range("sv_schedule_admit");
     if (!conf || !speed || !lengths) return SV_ERR_ARG;
     if (B < 1 || K < 1 || K > SV_MAX_K || static_cast<long long>(B) * K > sv::kAdmitMax ||
         n_speed < 1)

@@ -97,8 +97,8 @@ static void profile_release() {
 }  // namespace sv
 
 extern "C" sv_status sv_schedule(const float *conf, int B, int K, float load, int32_t *lengths,
-                                 void *stream) {    sv::NvtxRange nvtx_range("sv_schedule");
-
+                                 void *stream) {
+    sv::NvtxRange nvtx_range("sv_schedule");
     if (!conf || !lengths) return SV_ERR_ARG;
     if (B < 1 || K < 1 || K > SV_MAX_K) return SV_ERR_SHAPE;
     const int threads = 256;

@@ -127,8 +127,8 @@ extern "C" sv_status sv_verify_host(const void *target_logits, const void *draft
                                     int32_t *out_tokens, int32_t *out_accept_len,
                                     int32_t *lengths, int32_t *status, int levelwise,
                                     void *workspace, size_t workspace_bytes, size_t *h2d_bytes,
-                                    void *stream) {    sv::NvtxRange nvtx_range("sv_verify_host");
-
+                                    void *stream) {
+    sv::NvtxRange nvtx_range("sv_verify_host");
     using sv::hostio::Layout;
     if (!target_logits || !draft_tokens || !temperature || !out_tokens ||
         !out_accept_len || !lengths || !workspace)

@@ -91,9 +91,16 @@ __device__ __forceinline__ int ld_acquire_i32(const int *p) {
     return v;
 }
 
+// Wall-time bound of a grid-barrier wait (1 s; no legitimate wait comes
+// close) and the number of waits that ran out.  Both are set and read only
+// through the test exports at the end of this file.
+__device__ unsigned long long g_sts_wait_limit_ns = 1000000000ull;
+__device__ unsigned int g_sts_timeouts;
+
 // Grid barrier (sense by generation).  Every CTA of the cooperative launch
 // is resident, so a wait ends as soon as the last CTA arrives; the wait is
-// still bounded in wall time.  Returns false (in every thread) on timeout.
+// still bounded in wall time.  Returns false (in every thread) on timeout
+// and counts the timeout.
 __device__ bool grid_barrier(int *bar, int nblocks) {
     __shared__ int ok;
     __syncthreads();
@@ -107,8 +114,13 @@ __device__ bool grid_barrier(int *bar, int nblocks) {
             atomicAdd(&bar[1], 1);
         } else {
             const uint64_t t0 = global_ns();
+            const uint64_t limit = g_sts_wait_limit_ns;
             while (ld_acquire_i32(&bar[1]) == gen) {
-                if (global_ns() - t0 > 1000000000ull) { good = 0; break; }
+                if (global_ns() - t0 > limit) {
+                    good = 0;
+                    atomicAdd(&g_sts_timeouts, 1u);
+                    break;
+                }
                 __nanosleep(64);
             }
         }
@@ -325,8 +337,8 @@ extern "C" size_t sv_sts_workspace_bytes(int N, int K) {
 
 extern "C" sv_status sv_sts_fit(const float *logits, const int32_t *accept_len, int N, int K,
                                 float tmin, float tmax, float *temperature, float *ece,
-                                void *workspace, size_t workspace_bytes, void *stream) {    sv::NvtxRange nvtx_range("sv_sts_fit");
-
+                                void *workspace, size_t workspace_bytes, void *stream) {
+    sv::NvtxRange nvtx_range("sv_sts_fit");
     if (!logits || !accept_len || !temperature || !workspace) return SV_ERR_ARG;
     if (!(tmin > 0.f) || !(tmax > tmin) || !std::isfinite(tmax)) return SV_ERR_ARG;
     sv::StsPlan p;
@@ -374,8 +386,8 @@ extern "C" sv_status sv_sts_fit(const float *logits, const int32_t *accept_len, 
 }
 
 extern "C" sv_status sv_sts_apply(const float *logits, const float *temperature, int N, int K,
-                                  float *conf_out, void *stream) {    sv::NvtxRange nvtx_range("sv_sts_apply");
-
+                                  float *conf_out, void *stream) {
+    sv::NvtxRange nvtx_range("sv_sts_apply");
     if (!logits || !temperature || !conf_out) return SV_ERR_ARG;
     if (N < 1 || K < 1 || K > SV_MAX_K) return SV_ERR_SHAPE;
     const long long total = static_cast<long long>(N) * K;
@@ -383,4 +395,22 @@ extern "C" sv_status sv_sts_apply(const float *logits, const float *temperature,
     return sv::note_cuda(sv::launch_pdl(sv::sts_apply_kernel, dim3(blocks), dim3(256), 0,
                                         static_cast<cudaStream_t>(stream), logits, temperature,
                                         total, K, conf_out));
+}
+
+// Test exports for the bounded wait of the calibration's grid barrier: set
+// the wall-time limit on the current device (0 restores the 1 s default),
+// and read-and-clear the count of waits that ran out.  A limit near zero
+// makes every CTA but the last to arrive give up at the first barrier, so
+// the fit returns with T = NaN instead of waiting: the failure path runs
+// without a fault or a hang.
+extern "C" sv_status sv_debug_sts_wait_limit(uint64_t limit_ns) {
+    const unsigned long long v = limit_ns ? limit_ns : 1000000000ull;
+    return sv::note_cuda(cudaMemcpyToSymbol(sv::g_sts_wait_limit_ns, &v, sizeof(v)));
+}
+
+extern "C" int sv_debug_sts_timeouts(void) {
+    unsigned int n = 0, z = 0;
+    if (cudaMemcpyFromSymbol(&n, sv::g_sts_timeouts, sizeof(n)) != cudaSuccess) return -1;
+    if (cudaMemcpyToSymbol(sv::g_sts_timeouts, &z, sizeof(z)) != cudaSuccess) return -1;
+    return static_cast<int>(n);
 }

@@ -821,8 +821,8 @@ extern "C" size_t sv_vp_workspace_bytes(const sv_vp_slice *s) {
 
 extern "C" sv_status sv_vp_stats(const sv_vp_slice *s, const int32_t *draft_tokens,
                                  const int32_t *lengths, const float *temperature,
-                                 void *stats_local, void *stream) {    sv::NvtxRange nvtx_range("sv_vp_stats");
-
+                                 void *stats_local, void *stream) {
+    sv::NvtxRange nvtx_range("sv_vp_stats");
     Plan p;
     const sv_status st0 = sv::vp::check_slice(s, &p);
     if (st0 != SV_OK) return st0;
@@ -849,8 +849,8 @@ extern "C" sv_status sv_vp_decide(const sv_vp_slice *s, const void *stats_all,
                                   const float *temperature, uint64_t seed, int64_t row_base,
                                   int32_t *out_tokens, int32_t *out_accept_len, float *mass_local,
                                   float *norm_out, void *workspace, size_t workspace_bytes,
-                                  int32_t *status, void *stream) {    sv::NvtxRange nvtx_range("sv_vp_decide");
-
+                                  int32_t *status, void *stream) {
+    sv::NvtxRange nvtx_range("sv_vp_decide");
     Plan p;
     const sv_status st0 = sv::vp::check_slice(s, &p);
     if (st0 != SV_OK) return st0;
@@ -891,8 +891,8 @@ extern "C" sv_status sv_vp_decide(const sv_vp_slice *s, const void *stats_all,
 
 extern "C" sv_status sv_vp_draw(const sv_vp_slice *s, const float *mass_all, int32_t *out_tokens,
                                 void *workspace, size_t workspace_bytes, int32_t *status,
-                                void *stream) {    sv::NvtxRange nvtx_range("sv_vp_draw");
-
+                                void *stream) {
+    sv::NvtxRange nvtx_range("sv_vp_draw");
     Plan p;
     const sv_status st0 = sv::vp::check_slice(s, &p);
     if (st0 != SV_OK) return st0;

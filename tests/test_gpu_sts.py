@@ -71,3 +71,31 @@ def test_sts_apply():
     torch.cuda.synchronize()
     want = 1.0 / (1.0 + np.exp(-(l.astype(np.float64) / T.astype(np.float64))))
     np.testing.assert_allclose(out.cpu().numpy(), want, rtol=2e-6, atol=1e-7)
+
+
+def test_barrier_wait_that_runs_out_returns_nan():
+    """The grid barrier's wait is bounded in wall time.  With the bound set
+    near zero (a test export), the CTAs that arrive early give up at once:
+    the call returns, the temperatures come out NaN, the ECE output is not
+    written, and the expired waits are counted.  Nothing hangs or faults,
+    and with the bound restored the same fit matches the oracle again."""
+    l, a = sts_heldout(8192, 4, seed=13)      # 4 chunks x 4 positions: 16 CTAs
+    sv.sv_debug_sts_timeouts()                # clear the count
+    outcomes = []
+    try:
+        sv.sv_debug_sts_wait_limit(1)
+        for _ in range(3):
+            T, ece = gpu_fit(l, a)
+            outcomes.append((sv.sv_debug_sts_timeouts(), T, ece))
+    finally:
+        sv.sv_debug_sts_wait_limit(0)         # back to the 1 s default
+    timed_out = [o for o in outcomes if o[0] > 0]
+    assert timed_out, [o[0] for o in outcomes]
+    for n, T, ece in timed_out:
+        assert np.all(np.isnan(T)), T
+        assert list(ece) == [-1.0, -1.0]      # left as the caller filled it
+    for n, T, ece in outcomes:
+        if n == 0:                            # a fit whose barriers all met in time
+            assert np.all(np.isfinite(T))
+    check(l, a)
+    assert sv.sv_debug_sts_timeouts() == 0
