@@ -39,17 +39,14 @@
 //      merges the normalisers of positions 0..j, writes greedy rows, sets up
 //      each sampled row's final draw (for p-mass draws the chunk is chosen
 //      from the stream partials) and appends the resample work list.
-//   4. resample_sum_kernel (persistent, four CTAs per SM): for every row
-//      with a residual draw, the residual mass max(0, p_j - q_j) of each
-//      64-unit sub-range of position j, into the row's sub-range table.
-//      Items of 16 sub-ranges are dealt out in a fixed stride; each warp
-//      issues all of its loads for two sub-ranges before the math.  Only
-//      position j of a rejecting row is read a second time.
-//   5. resample_pick_kernel (one CTA per row): residual draws form the
-//      chunk totals from the table in the order the scan walks them, pick
-//      the chunk, the sub-range and the token inside it; p-mass draws
-//      locate the token inside the chunk the accept kernel chose.  Writes
-//      the row's outputs.
+//   4. resample_kernel (persistent, three CTAs per SM): first the p-mass
+//      draws (bonus, greedy drafter), each located inside the chunk the
+//      accept kernel chose; then, for every row with a residual draw, the
+//      residual mass max(0, p_j - q_j) of each 64-unit sub-range of
+//      position j, in items of 16 sub-ranges dealt out in a fixed stride.
+//      The CTA that completes a row's last item (atomic count, no waiting)
+//      picks the chunk, the sub-range and the token.  Only position j of a
+//      rejecting row is read a second time.
 #include <climits>
 #include <cstdint>
 #include <cstdio>
@@ -85,7 +82,8 @@ struct VerifyArgs {
     int32_t *out_accept;       // [B]
     int32_t *status;           // nullable
     float *dbg;                // nullable [B, S, 2]
-    int *ctr;                  // [0] next item, [1] total items, [2] rows with a residual draw
+    int *ctr;                  // [0] next item, [1] total items, [2] residual draws, [3] p-mass draws
+    int *rcnt;                 // [B]  residual items of the row finished
     int *leff;                 // [B]  verify length of a valid row, -1 for an invalid one
     int *row_j;                // [B]  first rejection found so far (starts at L)
     int *pcnt;                 // [B, K+1] item partials published per (row, position)
@@ -95,7 +93,7 @@ struct VerifyArgs {
     float *rtbl;               // [B, nsub] residual mass per sub-range
     int nsub;                  // sub-ranges per row
     int nitem;                 // residual-sum items per row (kSumItemSubs sub-ranges each)
-    int *work;                 // [B] rows with a residual draw (ctr[2] of them)
+    int *work;                 // [2B] rows with a residual draw (ctr[2]), then p-mass draws (ctr[3])
     struct DrawRecord *rec;    // [B] accept result and draw set-up
 };
 
@@ -170,6 +168,7 @@ __global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(VerifyArgs a
         }
         a.leff[b] = Lb;
         a.row_j[b] = Lb;
+        a.rcnt[b] = 0;
         for (int i = 0; i < K1; ++i) a.pcnt[static_cast<long long>(b) * K1 + i] = 0;
         if (b < kPrologueSmemRows)
             s_row[b] = Lb < 0 ? -1 : (Lb | ((draft && a.temp[b] > 0.f) ? (1 << 30) : 0));
@@ -213,6 +212,7 @@ __global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(VerifyArgs a
         a.ctr[0] = 0;
         a.ctr[1] = acc;
         a.ctr[2] = 0;
+        a.ctr[3] = 0;
     }
 }
 
@@ -365,14 +365,23 @@ template <int ESIZE>
 __device__ void producer(const VerifyArgs &a, StreamSmem &sm, uint4 *ring, int total) {
     uint32_t it = 0;
     bool ok = true;
-    // The next claim is taken as the current item starts, so that the
-    // counter's round trip overlaps the item.  The row's status is read when
-    // the item's turn comes and again before each later stage: a rejection
-    // only ever lowers it, so a stale value costs redundant bytes, never a
-    // wrong result.
-    int w = atomicAdd(&a.ctr[0], 1);
+    // Claims run two items ahead.  While item k is classified, item k+1 is
+    // already decoded with its row's first-rejection marker requested, and
+    // the claim of item k+2 is in flight, so a run of skipped items costs
+    // about one decode each instead of a claim, a decode and a marker read
+    // in series.  The marker only ever goes down, so a stale value costs
+    // redundant bytes, never a wrong result; a streamed item reads it again
+    // before every stage (the read is issued before the wait for the slot).
+    int w0 = atomicAdd(&a.ctr[0], 1);
+    int w1 = atomicAdd(&a.ctr[0], 1);
+    ItemRef c0 = {0, 0, 0, 0};
+    int rj0 = 0;
+    if (w0 < total) {
+        c0 = decode_item(a, w0);
+        rj0 = ld_relaxed(&a.row_j[c0.b]);
+    }
     while (ok) {
-        if (w >= total) {
+        if (w0 >= total) {
             const int st = it % kStages;
             const uint32_t ph = (it / kStages) & 1u;
             if (!mbar_wait(&sm.empty[st], ph ^ 1u, kWaitLimitNs)) { ok = false; break; }
@@ -381,13 +390,17 @@ __device__ void producer(const VerifyArgs &a, StreamSmem &sm, uint4 *ring, int t
             ++it;
             break;
         }
-        const ItemRef cur = decode_item(a, w);
-        const int rj = ld_relaxed(&a.row_j[cur.b]);
-        const int wnext = atomicAdd(&a.ctr[0], 1);
+        const int w2 = (w1 < total) ? atomicAdd(&a.ctr[0], 1) : total;
+        ItemRef c1 = {0, 0, 0, 0};
+        int rj1 = 0;
+        if (w1 < total) {
+            c1 = decode_item(a, w1);
+            rj1 = ld_relaxed(&a.row_j[c1.b]);
+        }
         // A row that has already rejected an earlier position never needs
         // this one: skip it without reading a byte.
-        if (rj >= cur.i) {
-            const int b = cur.b, i = cur.i, slot = cur.slot, chunk = cur.chunk;
+        if (rj0 >= c0.i) {
+            const int b = c0.b, i = c0.i, slot = c0.slot, chunk = c0.chunk;
             const float T = __ldg(&a.temp[b]);
             const float k = (T > 0.f) ? kLog2e / T : 0.f;
             const VecGeom g = vec_geom<ESIZE>(vec_ptr<ESIZE>(a, b, slot), a.V);
@@ -398,13 +411,14 @@ __device__ void producer(const VerifyArgs &a, StreamSmem &sm, uint4 *ring, int t
                 // Abandon the rest of the item once the row has rejected an
                 // earlier position: the consumers reset at the next item's
                 // first stage, and no partial of this item is ever read.
-                if (p > 0 && ld_relaxed(&a.row_j[b]) < i) break;
+                const int fresh = ld_relaxed(&a.row_j[b]);
                 const int st = it % kStages;
                 const uint32_t ph = (it / kStages) & 1u;
                 if (!mbar_wait(&sm.empty[st], ph ^ 1u, kWaitLimitNs) || vload(sm.abort)) {
                     ok = false;
                     break;
                 }
+                if (fresh < i) break;
                 const int pu0 = u0 + p * kStageUnits;
                 const int pn = max(0, min(u1 - pu0, kStageUnits));
                 StageDesc &d = sm.desc[st];
@@ -423,7 +437,7 @@ __device__ void producer(const VerifyArgs &a, StreamSmem &sm, uint4 *ring, int t
                 ++it;
             }
         }
-        w = wnext;
+        w0 = w1; c0 = c1; rj0 = rj1; w1 = w2;
     }
     if (!ok) {
         // Unwind: report, then wait (bounded) for the copies still in flight
@@ -1334,25 +1348,25 @@ __global__ void __launch_bounds__(kDrawThreads) accept_kernel(VerifyArgs a) {
         r.cd = resid ? log2f(ds.s[K + 1 + j]) : 0.f;
         r.note = note;
         *rec = r;
-        // Residual draws need the sub-range table: list the row for the sum
-        // kernel.  p-mass draws go straight to the pick kernel.
+        // List the row for the resample kernel: residual draws need the
+        // sub-range table first, p-mass draws only the chosen chunk.
         if (resid) a.work[atomicAdd(&a.ctr[2], 1)] = b;
+        else a.work[a.B + atomicAdd(&a.ctr[3], 1)] = b;
     }
 }
 
 // ---------------------------------------------------------------------------
-// 4. Residual sums: a persistent grid over (residual row, item) pairs, where
-//    an item is kSumItemSubs consecutive sub-ranges of position j of the row.
-//    Warp w of a CTA takes sub-ranges 2w and 2w+1 of the item: every lane
-//    issues its four target and four draft 16-byte loads before any math,
-//    so each SM keeps its four CTAs' loads in flight while other warps
+// Residual sums by items of kSumItemSubs consecutive sub-ranges of position
+//    j of a row.  Warp w of a CTA takes sub-ranges 2w and 2w+1 of the item:
+//    every lane issues its four target and four draft 16-byte loads before
+//    any math, so an SM keeps its CTAs' loads in flight while other warps
 //    compute.  The sums are formed exactly as the draw's scan expects them
 //    (per lane: unit q, then unit q + 32; the head joins sub-range 0 and the
-//    tail the last one; then a fixed shuffle tree).  Nothing waits on
-//    another CTA and no counter is kept: the pick kernel reads the table.
+//    tail the last one; then a fixed shuffle tree).
 // ---------------------------------------------------------------------------
 constexpr int kSumThreads = 256;
 constexpr int kSumItemSubs = 2 * (kSumThreads / 32);   // sub-ranges per item
+static_assert(kSumThreads == kDrawThreads, "finish_row runs on the resample CTA");
 
 // Residual sums of sub-ranges s0 and s0 + 1 (one warp) into tbl.
 template <int ESIZE>
@@ -1431,45 +1445,17 @@ __device__ __forceinline__ DrawCtx draw_ctx(const VerifyArgs &a, int b, const Dr
     return c;
 }
 
+// Final draw of row b and its outputs, by the whole CTA.  Residual draws:
+// warp w forms the totals of chunks w, w + 8, ... from the sub-range table
+// (in the order the scan walks them); warp 0 then picks the chunk, the
+// sub-range inside it, and the token inside that.  p-mass draws (bonus,
+// greedy drafter): the chunk was chosen by the accept kernel; the CTA
+// splits it into warp segments, scans them and walks the elements.
 template <int ESIZE>
-__global__ void __launch_bounds__(kSumThreads, 4) resample_sum_kernel(VerifyArgs a) {
-    const int warp = threadIdx.x >> 5;
-    griddep_wait();
-    griddep_launch_dependents();   // the pick CTAs wait for this grid anyway
-    const int nres = __ldcg(&a.ctr[2]);
-    const int per_row = a.nitem;
-    const int total = nres * per_row;   // < INT_MAX / 2 (checked by the plan)
-    for (int w = blockIdx.x; w < total; w += gridDim.x) {
-        const int e = w / per_row;
-        const int item = w - e * per_row;
-        const int b = __ldcg(&a.work[e]);
-        const DrawRecord r = a.rec[b];   // written by the accept kernel
-        const DrawCtx c = draw_ctx<ESIZE>(a, b, r);
-        const int nsub = max(1, (c.gt.n16 + kSubUnits - 1) / kSubUnits);
-        const int s0 = item * kSumItemSubs + 2 * warp;
-        if (s0 < nsub)
-            subrange_pair<ESIZE>(c, s0, nsub, a.rtbl + static_cast<long long>(b) * a.nsub);
-    }
-}
-
-// ---------------------------------------------------------------------------
-// 5. Pick kernel: one CTA per row.  Residual draws: warp w forms the totals
-//    of chunks w, w + 8, ... from the sub-range table (in the order the scan
-//    walks them); warp 0 then picks the chunk, the sub-range inside it, and
-//    the token inside that.  p-mass draws (bonus, greedy drafter): the chunk
-//    was chosen by the accept kernel; the CTA splits it into warp segments,
-//    scans them and walks the elements.  Writes the row's outputs.
-// ---------------------------------------------------------------------------
-template <int ESIZE>
-__global__ void __launch_bounds__(kDrawThreads) resample_pick_kernel(VerifyArgs a) {
-    __shared__ DrawSmem ds;
-    __shared__ float s_ct[kMaxChunks];
+__device__ __forceinline__ void finish_row(const VerifyArgs &a, int b, const DrawRecord &r, DrawSmem &ds,
+                           float *s_ct) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int b = blockIdx.x;
     const int K = a.K, C = a.C;
-    griddep_wait();
-    const DrawRecord r = a.rec[b];   // written by the accept kernel
-    if (r.mode == kDrawDone) return;
     const bool resid = r.mode == kDrawResidual;
     const int j = r.j;
     DrawCtx c = draw_ctx<ESIZE>(a, b, r);
@@ -1571,6 +1557,64 @@ __global__ void __launch_bounds__(kDrawThreads) resample_pick_kernel(VerifyArgs 
         a.out_tokens[static_cast<long long>(b) * (K + 1) + t] = v;
     }
     if (tid == 0) a.out_accept[b] = j;
+    __syncthreads();   // shared state is reused by the CTA's next item
+}
+
+// ---------------------------------------------------------------------------
+// 4. Resample kernel: one persistent grid (three CTAs per SM) over the draws
+//    the accept kernel listed.  Items are dealt out in a fixed stride:
+//    first one item per p-mass draw (bonus, greedy drafter: the CTA locates
+//    the token inside the chosen chunk), then, for every residual draw, its
+//    items of kSumItemSubs sub-ranges of position j (warp w sums sub-ranges
+//    2w and 2w + 1, every load issued before the math).  The CTA that
+//    completes a row's last residual item (atomic count; nothing waits)
+//    picks the row's token at once.  Only position j of a rejecting row is
+//    read a second time.
+// ---------------------------------------------------------------------------
+template <int ESIZE>
+__global__ void __launch_bounds__(kSumThreads, 3) resample_kernel(VerifyArgs a) {
+    __shared__ DrawSmem ds;
+    __shared__ float s_ct[kMaxChunks];
+    __shared__ int s_last;
+    const int warp = threadIdx.x >> 5;
+    griddep_wait();
+    const int nres = __ldcg(&a.ctr[2]);
+    const int npm = __ldcg(&a.ctr[3]);
+    const int per_row = a.nitem;
+    const int total = npm + nres * per_row;   // < INT_MAX / 2 (checked by the plan)
+    for (int w = blockIdx.x; w < total; w += gridDim.x) {
+        int b;
+        bool finish = true;
+        if (w < npm) {
+            b = __ldcg(&a.work[a.B + w]);
+        } else {
+            const int e = (w - npm) / per_row;
+            const int item = (w - npm) - e * per_row;
+            b = __ldcg(&a.work[e]);
+            {
+                const DrawRecord r = a.rec[b];   // written by the accept kernel
+                const DrawCtx c = draw_ctx<ESIZE>(a, b, r);
+                const int nsub = max(1, (c.gt.n16 + kSubUnits - 1) / kSubUnits);
+                const int s0 = item * kSumItemSubs + 2 * warp;
+                if (s0 < nsub)
+                    subrange_pair<ESIZE>(c, s0, nsub,
+                                         a.rtbl + static_cast<long long>(b) * a.nsub);
+            }
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                __threadfence();
+                const int done = atomicAdd(&a.rcnt[b], 1) + 1;
+                s_last = done == per_row;
+                if (s_last) __threadfence();
+            }
+            __syncthreads();
+            finish = s_last != 0;
+        }
+        if (finish) {
+            const DrawRecord r = a.rec[b];
+            finish_row<ESIZE>(a, b, r, ds, s_ct);
+        }
+    }
 }
 
 template <int ESIZE> static const void *stream_kernel_ptr() {
@@ -1584,8 +1628,8 @@ struct Plan {
     int C, U, S;
     int nsub;
     int nitem;
-    size_t off_leff, off_rowj, off_pcnt, off_lvloff, off_lvlrow, off_part, off_rtbl, off_work,
-        off_rec, bytes;
+    size_t off_rcnt, off_leff, off_rowj, off_pcnt, off_lvloff, off_lvlrow, off_part, off_rtbl,
+        off_work, off_rec, bytes;
 };
 
 static bool make_plan(int B, int K, int V, sv_dtype dtype, Plan *p) {
@@ -1606,6 +1650,7 @@ static bool make_plan(int B, int K, int V, sv_dtype dtype, Plan *p) {
     const size_t iB = sizeof(int) * static_cast<size_t>(B);
     auto align16 = [](size_t o) { return (o + 15) & ~static_cast<size_t>(15); };
     size_t off = 16;
+    p->off_rcnt = off;   off = align16(off + iB);
     p->off_leff = off;   off = align16(off + iB);
     p->off_rowj = off;   off = align16(off + iB);
     p->off_pcnt = off;   off = align16(off + iB * (K + 1));
@@ -1616,8 +1661,8 @@ static bool make_plan(int B, int K, int V, sv_dtype dtype, Plan *p) {
     if (p->nsub < 1) p->nsub = 1;
     p->off_rtbl = off;   off = align16(off + sizeof(float) * static_cast<size_t>(B) * p->nsub);
     p->nitem = (p->nsub + kSumItemSubs - 1) / kSumItemSubs;
-    if (static_cast<long long>(B) * p->nitem >= INT_MAX / 2) return false;
-    p->off_work = off;   off = align16(off + iB);
+    if (static_cast<long long>(B) * (p->nitem + 1) >= INT_MAX / 2) return false;
+    p->off_work = off;   off = align16(off + 2 * iB);
     p->off_rec = off;    off = align16(off + sizeof(DrawRecord) * static_cast<size_t>(B));
     p->bytes = off;
     return true;
@@ -1649,9 +1694,9 @@ static int stream_grid(int esize, long long max_items) {
     return static_cast<int>(max_items < n ? max_items : n);
 }
 
-// Persistent grid of the residual-sum kernel: resident CTAs per SM x SMs
+// Persistent grid of the resample kernel: resident CTAs per SM x SMs
 // (cached per dtype and device), at most one CTA per item.
-static int resample_sum_grid(int esize, long long max_items) {
+static int resample_grid(int esize, long long max_items) {
     static std::atomic<int> cache[2][64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return -1;
@@ -1661,8 +1706,8 @@ static int resample_sum_grid(int esize, long long max_items) {
         int sms = 0, per = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return -1;
-        const void *fn = esize == 4 ? reinterpret_cast<const void *>(&resample_sum_kernel<4>)
-                                    : reinterpret_cast<const void *>(&resample_sum_kernel<2>);
+        const void *fn = esize == 4 ? reinterpret_cast<const void *>(&resample_kernel<4>)
+                                    : reinterpret_cast<const void *>(&resample_kernel<2>);
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fn, kSumThreads, 0) !=
             cudaSuccess)
             return -1;
@@ -1699,6 +1744,7 @@ static sv_status verify_impl(const void *zt, const void *zd, sv_dtype dtype, int
     a.out_tokens = out_tokens; a.out_accept = out_accept; a.status = status; a.dbg = dbg;
     char *w = static_cast<char *>(ws);
     a.ctr = reinterpret_cast<int *>(w);
+    a.rcnt = reinterpret_cast<int *>(w + p.off_rcnt);
     a.leff = reinterpret_cast<int *>(w + p.off_leff);
     a.row_j = reinterpret_cast<int *>(w + p.off_rowj);
     a.pcnt = reinterpret_cast<int *>(w + p.off_pcnt);
@@ -1725,20 +1771,16 @@ static sv_status verify_impl(const void *zt, const void *zd, sv_dtype dtype, int
                   : launch_pdl(stream_kernel<2>, dim3(grid), dim3(kBlock), kRingBytes, st, a);
     if (e != cudaSuccess) return note_cuda(e);
     profile_mark_end(st);
-    const int sum_grid = resample_sum_grid(es, static_cast<long long>(B) * p.nitem);
-    if (sum_grid <= 0) return note_cuda(cudaGetLastError());
+    const int rs_grid = resample_grid(es, static_cast<long long>(B) * (p.nitem + 1));
+    if (rs_grid <= 0) return note_cuda(cudaGetLastError());
     if (es == 4) {
         e = launch_pdl(accept_kernel<4>, dim3(B), dim3(kDrawThreads), 0, st, a);
         if (e == cudaSuccess)
-            e = launch_pdl(resample_sum_kernel<4>, dim3(sum_grid), dim3(kSumThreads), 0, st, a);
-        if (e == cudaSuccess)
-            e = launch_pdl(resample_pick_kernel<4>, dim3(B), dim3(kDrawThreads), 0, st, a);
+            e = launch_pdl(resample_kernel<4>, dim3(rs_grid), dim3(kSumThreads), 0, st, a);
     } else {
         e = launch_pdl(accept_kernel<2>, dim3(B), dim3(kDrawThreads), 0, st, a);
         if (e == cudaSuccess)
-            e = launch_pdl(resample_sum_kernel<2>, dim3(sum_grid), dim3(kSumThreads), 0, st, a);
-        if (e == cudaSuccess)
-            e = launch_pdl(resample_pick_kernel<2>, dim3(B), dim3(kDrawThreads), 0, st, a);
+            e = launch_pdl(resample_kernel<2>, dim3(rs_grid), dim3(kSumThreads), 0, st, a);
     }
     if (e != cudaSuccess) return note_cuda(e);
     return note_cuda(cudaGetLastError());
@@ -1778,7 +1820,7 @@ extern "C" sv_status sv_verify_debug(const void *target_logits, const void *draf
                            workspace_bytes, status, stats_out, stream);
 }
 
-extern "C" int sv_verify_launches(void) { return 5; }
+extern "C" int sv_verify_launches(void) { return 4; }
 
 // ---------------------------------------------------------------------------
 // Allocation-free variant: the scratch lives in a fixed device array that
