@@ -490,12 +490,16 @@ sv_status sv_vp_draw(const sv_vp_slice *slice, const float *mass_all, int32_t *o
  *                  plus, for a row rejecting at a < L, position a+1, copied
  *                  before the rejection is known.  Same results (the
  *                  uniforms are keyed by row, position and draw), up to K
- *                  synchronisations; SV_NOTE_* bits may also come from
- *                  draws whose rows were still undecided.
+ *                  synchronisations per half; SV_NOTE_* bits may also come
+ *                  from draws whose rows were still undecided.  The rows
+ *                  run in two halves on `stream` and on a second stream the
+ *                  library creates once per device (kept until exit), so
+ *                  one half's copies overlap the other half's verification;
+ *                  each level's lengths are computed on the device.
  *   workspace      DEVICE, >= sv_verify_host_workspace_bytes(), 256-byte
  *                  aligned: device copies of both logit arrays (only the
  *                  scheduled runs are written), the small arrays and the
- *                  sv_verify workspace.
+ *                  sv_verify workspaces (one per half in level-wise mode).
  *   h2d_bytes      nullable: bytes copied host-to-device by this call.
  * Returns SV_OK, SV_ERR_ARG, SV_ERR_SHAPE, SV_ERR_DTYPE, SV_ERR_WORKSPACE or
  * SV_ERR_CUDA.  Argument errors are returned before anything is enqueued.

@@ -24,6 +24,7 @@
 // that of one verification with the full lengths, and no kernel reads a
 // position that was not copied.
 #include <cstdint>
+#include <mutex>
 #include <vector>
 
 #include "sv.h"
@@ -33,7 +34,9 @@ namespace sv {
 namespace hostio {
 
 struct Layout {
-    size_t zt, zd, conf, tok, temp, len, otok, oacc, status, ver, ver_bytes, bytes;
+    size_t zt, zd, conf, tok, temp, len, lcur, otok, oacc, status, ver, ver_bytes, ver1,
+        ver1_bytes, bytes;
+    int half;   // rows of the first group in level-wise mode
 };
 
 static size_t align256(size_t o) { return (o + 255) & ~static_cast<size_t>(255); }
@@ -50,11 +53,18 @@ static bool make_layout(int B, int K, int V, sv_dtype dtype, Layout *L) {
     L->tok = o;    o = align256(o + b * k * sizeof(int32_t));
     L->temp = o;   o = align256(o + b * sizeof(float));
     L->len = o;    o = align256(o + b * sizeof(int32_t));
+    L->lcur = o;   o = align256(o + b * sizeof(int32_t));
     L->otok = o;   o = align256(o + b * (k + 1) * sizeof(int32_t));
     L->oacc = o;   o = align256(o + b * sizeof(int32_t));
     L->status = o; o = align256(o + sizeof(int32_t));
     L->ver = o;    o = align256(o + ver);
     L->ver_bytes = ver;
+    // Level-wise mode runs the rows in two halves on two streams; the second
+    // half needs its own sv_verify workspace (the first uses `ver`).
+    L->half = B >= 2 ? B / 2 : B;
+    const size_t ver1 = B - L->half > 0 ? sv_verify_workspace_bytes(B - L->half, K, V, dtype) : 0;
+    L->ver1 = o;   o = align256(o + ver1);
+    L->ver1_bytes = ver1;
     L->bytes = o;
     return true;
 }
@@ -110,6 +120,53 @@ struct LevelCopier {
         n = 0;
     }
 };
+
+// Lengths of level l (l >= 1) of level-wise mode, from each row's
+// scheduled length L and its accepted length at level l - 1: a row that
+// accepted every position tested so far (a == l - 1 < L) verifies min(L, l);
+// every other valid row is final and re-runs with length 0 on its copied
+// position 0; an invalid length is passed on so the row is marked again.
+__global__ void level_lengths_kernel(const int32_t *__restrict__ L,
+                                     const int32_t *__restrict__ acc_prev, int n, int K, int l,
+                                     int32_t *__restrict__ lcur) {
+    for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < n; b += gridDim.x * blockDim.x) {
+        const int Lb = L[b];
+        int v;
+        if (Lb < 0 || Lb > K) v = Lb;
+        else if (l == 1) v = Lb < 1 ? Lb : 1;
+        else v = (acc_prev[b] == l - 1 && l - 1 < Lb) ? (Lb < l ? Lb : l) : 0;
+        lcur[b] = v;
+    }
+}
+
+// A second stream (and an event to order it after the caller's stream) per
+// device, created on first use and kept for the life of the process: the
+// level-wise mode copies one half of the rows while the other half verifies.
+struct Aux {
+    cudaStream_t st = nullptr;
+    cudaEvent_t ev = nullptr;
+};
+static std::mutex g_aux_mu;
+static Aux g_aux[64];
+
+static sv_status aux_stream(Aux *out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return note_cuda(e);
+    if (dev < 0 || dev >= 64) return SV_ERR_ARG;
+    std::lock_guard<std::mutex> lock(g_aux_mu);
+    Aux &a = g_aux[dev];
+    if (!a.st) {
+        e = cudaStreamCreateWithFlags(&a.st, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&a.ev, cudaEventDisableTiming);
+        if (e != cudaSuccess) {
+            a.st = nullptr;
+            return note_cuda(e);
+        }
+    }
+    *out = a;
+    return SV_OK;
+}
 
 }  // namespace hostio
 }  // namespace sv
@@ -184,8 +241,33 @@ extern "C" sv_status sv_verify_host(const void *target_logits, const void *draft
         // Level l: position l of every undecided row in; from level 1 on,
         // verify with lengths min(L, l) (finished rows re-run with length 0
         // on data already present, their outputs ignored), decisions out.
+        // The rows run in two halves, each on its own stream, ping-pong:
+        // while the host waits for one half's decisions, the other half's
+        // copies keep the host link busy.  The lengths of each level are
+        // computed on the device from the previous level's accept lengths.
         const size_t K1 = nk + 1;
-        std::vector<int32_t> lcur(nb), acc(nb), tok(nb * K1);
+        sv::hostio::Aux aux;
+        const int h = L.half;
+        const bool two = B - h > 0;
+        if (two) {
+            s = sv::hostio::aux_stream(&aux);
+            if (s != SV_OK) return s;
+            // the second stream starts after the small inputs and the schedule
+            e = cudaEventRecord(aux.ev, st);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(aux.st, aux.ev, 0);
+            if (e != cudaSuccess) return sv::note_cuda(e);
+        }
+        struct Group {
+            int b0, n;
+            cudaStream_t st;
+            char *ver;
+            size_t ver_bytes;
+            bool active;
+        };
+        Group grp[2] = {{0, h, st, w + L.ver, L.ver_bytes, true},
+                        {h, B - h, two ? aux.st : st, w + L.ver1, L.ver1_bytes, two}};
+        int32_t *lcur_d = reinterpret_cast<int32_t *>(w + L.lcur);
+        std::vector<int32_t> acc(nb), tok(nb * K1);
         std::vector<char> alive(nb);
         for (int b = 0; b < B; ++b) {
             alive[b] = 1;
@@ -193,63 +275,103 @@ extern "C" sv_status sv_verify_host(const void *target_logits, const void *draft
             out_accept_len[b] = -1;
         }
         size_t copied = 0;
-        for (int l = 0; l <= K; ++l) {
+        // Copies of level l for the live rows of group g (target position l
+        // if l <= L, draft position l if l < L and the row samples).
+        auto copy_level = [&](const Group &g, int l) -> cudaError_t {
             const size_t lo = static_cast<size_t>(l) * vb;
-            sv::hostio::LevelCopier ct(zt_h + lo, zt_d + lo, K1 * vb, vb, st);
-            int n_alive = 0;
-            for (int b = 0; b < B; ++b) {
+            sv::hostio::LevelCopier ct(zt_h + lo, zt_d + lo, K1 * vb, vb, g.st);
+            for (int b = g.b0; b < g.b0 + g.n; ++b) {
                 const int Lb = lengths[b];
-                const bool bad = Lb < 0 || Lb > K;
-                // A row with an invalid length keeps it (it is marked again,
-                // nothing is read); a finished valid row re-runs with length
-                // 0 on its copied position 0.
-                lcur[b] = bad ? Lb : (alive[b] ? (l < Lb ? l : Lb) : 0);
-                if (!alive[b]) continue;
-                ++n_alive;
-                if (bad || l > Lb) continue;
+                if (!alive[b] || Lb < 0 || Lb > K || l > Lb) continue;
                 ct.add(b);
             }
-            if (n_alive == 0 && l > 0) break;
             ct.flush();
-            size_t level_bytes = ct.total;
-            cudaError_t cerr = ct.err;
+            copied += ct.total;
+            if (ct.err != cudaSuccess) return ct.err;
             if (zd_h && l < K) {
-                sv::hostio::LevelCopier cd(zd_h + lo, zd_d + lo, nk * vb, vb, st);
-                for (int b = 0; b < B; ++b) {
+                sv::hostio::LevelCopier cd(zd_h + lo, zd_d + lo, nk * vb, vb, g.st);
+                for (int b = g.b0; b < g.b0 + g.n; ++b) {
                     const int Lb = lengths[b];
                     if (!alive[b] || Lb < 0 || Lb > K || l >= Lb || !(temperature[b] > 0.f))
                         continue;
                     cd.add(b);
                 }
                 cd.flush();
-                level_bytes += cd.total;
-                if (cerr == cudaSuccess) cerr = cd.err;
+                copied += cd.total;
+                if (cd.err != cudaSuccess) return cd.err;
             }
-            if (cerr != cudaSuccess) return sv::note_cuda(cerr);
-            copied += level_bytes;
-            if (l == 0) continue;   // nothing to test yet; level 1 also settles L = 0
-            e = cudaMemcpyAsync(len_d, lcur.data(), nb * sizeof(int32_t), cudaMemcpyHostToDevice, st);
-            if (e != cudaSuccess) return sv::note_cuda(e);
-            small += nb * sizeof(int32_t);
-            s = sv_verify(zt_d, zd_h ? zd_d : nullptr, dtype, B, K, V, tok_d, len_d, temp_d, seed,
-                          row_base, otok_d, oacc_d, w + L.ver, L.ver_bytes, status_d, stream);
-            if (s != SV_OK) return s;
-            e = cudaMemcpyAsync(acc.data(), oacc_d, nb * sizeof(int32_t), cudaMemcpyDeviceToHost, st);
-            if (e == cudaSuccess)
-                e = cudaMemcpyAsync(tok.data(), otok_d, nb * K1 * sizeof(int32_t),
-                                    cudaMemcpyDeviceToHost, st);
-            if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-            if (e != cudaSuccess) return sv::note_cuda(e);
-            for (int b = 0; b < B; ++b) {
+            return cudaSuccess;
+        };
+        // Lengths of level l and the verification of group g's rows.
+        auto verify_level = [&](const Group &g, int l) -> sv_status {
+            const int threads = 256;
+            const int blocks = (g.n + threads - 1) / threads;
+            sv::hostio::level_lengths_kernel<<<blocks, threads, 0, g.st>>>(
+                len_d + g.b0, oacc_d + g.b0, g.n, K, l, lcur_d + g.b0);
+            cudaError_t le = cudaGetLastError();
+            if (le != cudaSuccess) return sv::note_cuda(le);
+            return sv_verify(zt_d + static_cast<size_t>(g.b0) * K1 * vb,
+                             zd_h ? zd_d + static_cast<size_t>(g.b0) * nk * vb : nullptr, dtype,
+                             g.n, K, V, tok_d + static_cast<size_t>(g.b0) * nk, lcur_d + g.b0,
+                             temp_d + g.b0, seed, row_base + g.b0,
+                             otok_d + static_cast<size_t>(g.b0) * K1, oacc_d + g.b0, g.ver,
+                             g.ver_bytes, status_d, g.st);
+        };
+        // Decisions of level l of group g back (the copy into pageable host
+        // memory returns once the group's stream has reached it); rows that
+        // rejected below l, reached their length, or are invalid are final.
+        auto read_level = [&](Group &g, int l) -> cudaError_t {
+            cudaError_t re = cudaMemcpyAsync(acc.data() + g.b0, oacc_d + g.b0,
+                                             static_cast<size_t>(g.n) * sizeof(int32_t),
+                                             cudaMemcpyDeviceToHost, g.st);
+            if (re == cudaSuccess)
+                re = cudaMemcpyAsync(tok.data() + static_cast<size_t>(g.b0) * K1,
+                                     otok_d + static_cast<size_t>(g.b0) * K1,
+                                     static_cast<size_t>(g.n) * K1 * sizeof(int32_t),
+                                     cudaMemcpyDeviceToHost, g.st);
+            if (re == cudaSuccess) re = cudaStreamSynchronize(g.st);
+            if (re != cudaSuccess) return re;
+            int n_alive = 0;
+            for (int b = g.b0; b < g.b0 + g.n; ++b) {
                 if (!alive[b]) continue;
                 const int Lb = lengths[b];
                 const bool bad = Lb < 0 || Lb > K;
-                if (bad || acc[b] < 0 || acc[b] < l || l >= Lb) {   // final: invalid, rejected, or done
+                if (bad || acc[b] < 0 || acc[b] < l || l >= Lb) {
                     alive[b] = 0;
                     out_accept_len[b] = acc[b];
                     for (size_t i = 0; i < K1; ++i) out_tokens[b * K1 + i] = tok[b * K1 + i];
+                } else {
+                    ++n_alive;
                 }
             }
+            g.active = n_alive > 0;
+            return cudaSuccess;
+        };
+        for (Group &g : grp) {
+            if (!g.active) continue;
+            e = copy_level(g, 0);
+            if (e != cudaSuccess) return sv::note_cuda(e);
+        }
+        int last = 0;
+        for (int l = 1; l <= K && (grp[0].active || grp[1].active); ++l) {
+            for (Group &g : grp) {
+                if (!g.active) continue;
+                if (l >= 2) {
+                    e = read_level(g, l - 1);
+                    if (e != cudaSuccess) return sv::note_cuda(e);
+                    if (!g.active) continue;
+                }
+                e = copy_level(g, l);
+                if (e != cudaSuccess) return sv::note_cuda(e);
+                s = verify_level(g, l);
+                if (s != SV_OK) return s;
+            }
+            last = l;
+        }
+        for (Group &g : grp) {
+            if (!g.active || last == 0) continue;
+            e = read_level(g, last);
+            if (e != cudaSuccess) return sv::note_cuda(e);
         }
         if (h2d_bytes) *h2d_bytes = copied + small;
         if (status) {

@@ -56,7 +56,7 @@ def _expected_h2d_levelwise(b, lengths, accept, with_draft, scheduled=True):
     """Target 0..a and draft 0..min(a, L-1) of sampled rows (what the outcome
     depends on), plus for a row that rejects at a < L the next position,
     copied before the rejection is known (target a+1; draft a+1 if a+1 < L);
-    the small arrays; one length array per verified level."""
+    the small arrays.  The lengths of each level are computed on the device."""
     B, K1, V = b.zt.shape
     K = K1 - 1
     es = b.zt.element_size()
@@ -64,8 +64,7 @@ def _expected_h2d_levelwise(b, lengths, accept, with_draft, scheduled=True):
     n = int(sum((a + 2 if a < L else L + 1) * V * es for a, L in zip(accept, lengths)))
     if with_draft:
         n += int(sum(min(a + 2, L) * V * es for a, L, t in zip(accept, lengths, T) if t > 0))
-    levels = max((a + 1) if a < L else max(L, 1) for a, L in zip(accept, lengths))
-    return n + B * K * 4 + B * 4 + (B * K * 4 if scheduled else 0) + levels * B * 4
+    return n + B * K * 4 + B * 4 + (B * K * 4 if scheduled else 0)
 
 
 @pytest.mark.parametrize("levelwise", [False, True])
