@@ -348,6 +348,19 @@ __device__ __forceinline__ void griddep_launch_dependents() {
 }  // namespace sv
 
 namespace sv {
+// atomicAdd with acquire-release semantics at GPU scope: the caller's earlier
+// writes are visible to whoever observes the new value, and the caller's
+// later reads see every write released before earlier increments of the
+// same counter.
+__device__ __forceinline__ int atom_add_acq_rel(int *p, int v) {
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;"
+                 : "=r"(old)
+                 : "l"(p), "r"(v)
+                 : "memory");
+    return old;
+}
+
 // Relaxed load of a flag that other CTAs update (a stale value only makes
 // the caller do redundant work).
 __device__ __forceinline__ int ld_relaxed(const int *p) {

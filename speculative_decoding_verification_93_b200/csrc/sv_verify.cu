@@ -39,14 +39,14 @@
 //      merges the normalisers of positions 0..j, writes greedy rows, sets up
 //      each sampled row's final draw (for p-mass draws the chunk is chosen
 //      from the stream partials) and appends the resample work list.
-//   4. resample_kernel (persistent, three CTAs per SM): first the p-mass
-//      draws (bonus, greedy drafter), each located inside the chunk the
-//      accept kernel chose; then, for every row with a residual draw, the
-//      residual mass max(0, p_j - q_j) of each 64-unit sub-range of
-//      position j, in items of 16 sub-ranges dealt out in a fixed stride.
-//      The CTA that completes a row's last item (atomic count, no waiting)
-//      picks the chunk, the sub-range and the token.  Only position j of a
-//      rejecting row is read a second time.
+//   4. resample_kernel (one CTA per work entry): residual draws sum
+//      max(0, p_j - q_j) over their chunk by 64-unit sub-ranges, and each
+//      chunk CTA also forms its chunk's total in the order the scan will
+//      walk it; the last chunk CTA of the row (atomic counter, no waiting)
+//      picks the chunk from the chunk totals, the sub-range from that
+//      chunk's sub-ranges, and the token inside it.  p-mass draws locate
+//      the token inside the chosen chunk.  Only position j of a rejecting
+//      row is read a second time.
 #include <climits>
 #include <cstdint>
 #include <cstdio>
@@ -82,8 +82,8 @@ struct VerifyArgs {
     int32_t *out_accept;       // [B]
     int32_t *status;           // nullable
     float *dbg;                // nullable [B, S, 2]
-    int *ctr;                  // [0] next item, [1] total items, [2] residual draws, [3] p-mass draws
-    int *rcnt;                 // [B]  residual items of the row finished
+    int *ctr;                  // [0] next item, [1] total items, [2] resample work entries
+    int *rcnt;                 // [B]  chunks of the residual draw done
     int *leff;                 // [B]  verify length of a valid row, -1 for an invalid one
     int *row_j;                // [B]  first rejection found so far (starts at L)
     int *pcnt;                 // [B, K+1] item partials published per (row, position)
@@ -91,9 +91,9 @@ struct VerifyArgs {
     int *lvl_row;              // [K+1, B+1] per-level exclusive prefix of row item counts
     float4 *part;              // [B, S, C]: (m, s, argmax bits, 0)
     float *rtbl;               // [B, nsub] residual mass per sub-range
+    float *ctot;               // [B, C] residual mass per chunk (its sub-ranges, in scan order)
     int nsub;                  // sub-ranges per row
-    int nitem;                 // residual-sum items per row (kSumItemSubs sub-ranges each)
-    int *work;                 // [2B] rows with a residual draw (ctr[2]), then p-mass draws (ctr[3])
+    int *work;                 // [B * C] (row * C + chunk) of the resample CTAs with work
     struct DrawRecord *rec;    // [B] accept result and draw set-up
 };
 
@@ -212,7 +212,6 @@ __global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(VerifyArgs a
         a.ctr[0] = 0;
         a.ctr[1] = acc;
         a.ctr[2] = 0;
-        a.ctr[3] = 0;
     }
 }
 
@@ -271,7 +270,8 @@ struct StreamSmem {
 // oracle: accept x_i iff u(seed, row, i, 0) < min(1, p_i(x_i) / q_i(x_i)),
 // greedy rows iff x_i is the target argmax.  A rejection lowers row_j[b].
 template <int ESIZE>
-__device__ void decide_position(const VerifyArgs &a, int b, int i) {
+__device__ void decide_position(const VerifyArgs &a, int b, int i, int x, float zt_x,
+                                float zd_x) {
     const int lane = threadIdx.x & 31;
     const int K = a.K, S = a.S, C = a.C;
     const float T = __ldg(&a.temp[b]);
@@ -310,18 +310,13 @@ __device__ void decide_position(const VerifyArgs &a, int b, int i) {
         }
     }
     if (lane == 0) {
-        const int x = a.tokens[static_cast<long long>(b) * K + i];
         bool acc;
         if (greedy) {
             acc = (x == (at == INT_MAX ? 0 : at));
         } else {
-            const float zt_x = ld_elem<ESIZE>(vec_ptr<ESIZE>(a, b, i), x);
             const float lp = fmaf(zt_x - mt, k, -log2f(st));
             float lq = 0.f;
-            if (has_draft) {
-                const float zd_x = ld_elem<ESIZE>(vec_ptr<ESIZE>(a, b, K + 1 + i), x);
-                lq = fmaf(zd_x - md, k, -log2f(sd));
-            }
+            if (has_draft) lq = fmaf(zd_x - md, k, -log2f(sd));
             const uint64_t row = static_cast<uint64_t>(a.row_base) + static_cast<uint64_t>(b);
             const float u = uniform24(a.seed, row, static_cast<uint32_t>(i), 0u);
             if (lp == kNegInf) acc = false;
@@ -611,21 +606,36 @@ __device__ void publisher(const VerifyArgs &a, StreamSmem &sm) {
                 lse_merge(rm, rs, m2, s2, im.k);
             }
         }
-        int complete = 0;
+        int complete = 0, x = 0;
+        float zt_x = 0.f, zd_x = 0.f;
         if (lane == 0) {
+            const int Lb = __ldg(&a.leff[im.b]);
+            const bool tested = im.level < Lb;   // positions 0..L-1 take an accept test
+            const bool draft_here = (a.zd != nullptr) && !greedy && tested;
+            const int need = a.C * (draft_here ? 2 : 1);
+            // The draft token is requested before the count's round trip, and
+            // both models' logits at it right after, so that the item that
+            // completes the position can test it at once.
+            if (tested) x = __ldg(&a.tokens[static_cast<long long>(im.b) * a.K + im.level]);
             a.part[(static_cast<long long>(im.b) * a.S + im.slot) * a.C + im.chunk] =
                 make_float4(rm, greedy ? 0.f : rs, __int_as_float(greedy ? ri : 0), 0.f);
-            __threadfence();
-            const int Lb = __ldg(&a.leff[im.b]);
-            const bool draft_here = (a.zd != nullptr) && !greedy && im.level < Lb;
-            const int need = a.C * (draft_here ? 2 : 1);
+            // Release: this partial is visible before the count; acquire: the
+            // completing item sees every partial counted before it.
             const int done =
-                atomicAdd(&a.pcnt[static_cast<long long>(im.b) * (a.K + 1) + im.level], 1) + 1;
-            complete = (done == need) && (im.level < Lb);
-            if (complete) __threadfence();
+                atom_add_acq_rel(&a.pcnt[static_cast<long long>(im.b) * (a.K + 1) + im.level], 1) + 1;
+            if (tested && !greedy) {
+                zt_x = ld_elem<ESIZE>(vec_ptr<ESIZE>(a, im.b, im.level), x);
+                if (draft_here) zd_x = ld_elem<ESIZE>(vec_ptr<ESIZE>(a, im.b, a.K + 1 + im.level), x);
+            }
+            complete = (done == need) && tested;
         }
         complete = __shfl_sync(0xffffffffu, complete, 0);
-        if (complete) decide_position<ESIZE>(a, im.b, im.level);
+        if (complete) {
+            x = __shfl_sync(0xffffffffu, x, 0);
+            zt_x = __shfl_sync(0xffffffffu, zt_x, 0);
+            zd_x = __shfl_sync(0xffffffffu, zd_x, 0);
+            decide_position<ESIZE>(a, im.b, im.level, x, zt_x, zd_x);
+        }
     }
 }
 
@@ -1049,6 +1059,8 @@ __device__ __forceinline__ void chunk_masses(const VerifyArgs &a, int b, int j, 
 // ---------------------------------------------------------------------------
 constexpr int kSubUnits = 64;   // units per sub-range; chunk sizes are multiples of it
 constexpr int kRunUnits = 3;    // local units per lane in a located sub-range (66 / 32)
+constexpr int kResidParts = 1;  // resample CTAs per chunk of a residual draw
+static_assert(kResidParts == 1, "each chunk CTA forms its chunk's residual total");
 
 // Draw weight of `count` (< one unit) elements from element `first`,
 // loaded directly (vector head or tail).
@@ -1065,6 +1077,74 @@ __device__ __forceinline__ float partial_sum(const DrawCtx &c, int first, int co
 #pragma unroll
     for (int e = 0; e < kPer; ++e) t += elem_weight<ESIZE, MODE>(c, u, e);
     return t;
+}
+
+// Residual weight of every sub-range of part `part` of chunk `ch` into tbl.
+// Warp w takes the 256-unit blocks w, w + 8, ... of the part with eight units per lane in
+// flight; unit base + lane + 32 q lies in sub-range base / 64 + q / 2.  The
+// head joins sub-range 0 and the tail the last one.  Each sum has a fixed
+// order.
+template <int ESIZE>
+__device__ void residual_subranges(const DrawCtx &c, int ch, int part, int U, float *tbl) {
+    constexpr int kPer = 16 / ESIZE;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int PU = (U / kResidParts + kSubUnits - 1) / kSubUnits * kSubUnits;   // units per part
+    const int u0 = ch * U + part * PU;
+    const int u1 = max(u0, min(min(u0 + PU, (ch + 1) * U), c.gt.n16));
+    const int slast = c.gt.n16 > 0 ? (c.gt.n16 - 1) / kSubUnits : 0;
+    const uint32_t pw = neg_inf_word<ESIZE>();
+    const uint4 pad = make_uint4(pw, pw, pw, pw);
+    int nblk = (u1 - u0 + 255) / 256;
+    if (c.gt.n16 == 0 && ch == 0 && part == 0) nblk = 1;   // head and tail only
+    for (int blk = warp; blk < nblk; blk += kDrawWarps) {
+        const int base = u0 + blk * 256;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        if (c.aligned) {
+            uint4 t[8], d[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int u = base + lane + 32 * q;
+                const long long off = static_cast<long long>(u) * 16;
+                t[q] = u < u1 ? ld_reuse(c.gt.body + off) : pad;
+                d[q] = u < u1 ? ld_reuse(c.gd.body + off) : pad;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[q >> 1] += body_sum<ESIZE, kDrawResidual>(c, t[q], d[q]);
+        } else {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int u = base + lane + 32 * q;
+                if (u < u1) {
+                    UnitData ud;
+                    ud.t = ld_reuse(c.gt.body + static_cast<long long>(u) * 16);
+                    ud.d = make_uint4(0u, 0u, 0u, 0u);
+                    ud.count = kPer;
+                    ud.first = c.gt.head + u * kPer;
+#pragma unroll
+                    for (int e = 0; e < kPer; ++e)
+                        acc[q >> 1] += elem_weight<ESIZE, kDrawResidual>(c, ud, e);
+                }
+            }
+        }
+        const int s0 = base / kSubUnits;
+        if (lane == 0) {
+            if (s0 == 0 && c.gt.head > 0) acc[0] += partial_sum<ESIZE, kDrawResidual>(c, 0, c.gt.head);
+            if (c.gt.tail > 0 && slast >= s0 && slast < s0 + 4)
+                acc[slast - s0] += partial_sum<ESIZE, kDrawResidual>(
+                    c, c.gt.head + c.gt.n16 * kPer, c.gt.tail);
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], o);
+        if (lane == 0) {
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int s = s0 + r;
+                if (s * kSubUnits < u1 || (c.gt.n16 == 0 && s == 0)) tbl[s] = acc[r];
+            }
+        }
+    }
 }
 
 // Sum of n table entries by one warp: rounds of 32 entries in order, a
@@ -1348,117 +1428,57 @@ __global__ void __launch_bounds__(kDrawThreads) accept_kernel(VerifyArgs a) {
         r.cd = resid ? log2f(ds.s[K + 1 + j]) : 0.f;
         r.note = note;
         *rec = r;
-        // List the row for the resample kernel: residual draws need the
-        // sub-range table first, p-mass draws only the chosen chunk.
-        if (resid) a.work[atomicAdd(&a.ctr[2], 1)] = b;
-        else a.work[a.B + atomicAdd(&a.ctr[3], 1)] = b;
+        // Resample work: every chunk of a residual draw, the selected chunk
+        // of a p-mass draw.
+        if (resid) {
+            const int base = atomicAdd(&a.ctr[2], C * kResidParts);
+            for (int q = 0; q < C * kResidParts; ++q) a.work[base + q] = b * C * kResidParts + q;
+        } else {
+            a.work[atomicAdd(&a.ctr[2], 1)] = (b * C + (ds.gsel < 0 ? 0 : ds.gsel)) * kResidParts;
+        }
     }
 }
 
 // ---------------------------------------------------------------------------
-// Residual sums by items of kSumItemSubs consecutive sub-ranges of position
-//    j of a row.  Warp w of a CTA takes sub-ranges 2w and 2w+1 of the item:
-//    every lane issues its four target and four draft 16-byte loads before
-//    any math, so an SM keeps its CTAs' loads in flight while other warps
-//    compute.  The sums are formed exactly as the draw's scan expects them
-//    (per lane: unit q, then unit q + 32; the head joins sub-range 0 and the
-//    tail the last one; then a fixed shuffle tree).
+// 4. Resample kernel: one CTA per (row, chunk).  p-mass draws: the CTA of
+//    the selected chunk locates the token inside it.  Residual draws: every
+//    chunk CTA sums max(0, p_j - q_j) over its chunk by segments; the last
+//    one (atomic counter, no waiting) selects the chunk and the segment from
+//    those sums and locates the token.
 // ---------------------------------------------------------------------------
-constexpr int kSumThreads = 256;
-constexpr int kSumItemSubs = 2 * (kSumThreads / 32);   // sub-ranges per item
-static_assert(kSumThreads == kDrawThreads, "finish_row runs on the resample CTA");
-
-// Residual sums of sub-ranges s0 and s0 + 1 (one warp) into tbl.
 template <int ESIZE>
-__device__ __forceinline__ void subrange_pair(const DrawCtx &c, int s0, int nsub, float *tbl) {
-    constexpr int kPer = 16 / ESIZE;
-    const int lane = threadIdx.x & 31;
-    const int n16 = c.gt.n16;
-    const int slast = n16 > 0 ? (n16 - 1) / kSubUnits : 0;
-    float acc[2] = {0.f, 0.f};
-    if (c.aligned) {
-        const uint32_t pw = neg_inf_word<ESIZE>();
-        const uint4 pad = make_uint4(pw, pw, pw, pw);
-        uint4 t[4], d[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int u = s0 * kSubUnits + lane + 32 * q;
-            const long long off = static_cast<long long>(u) * 16;
-            t[q] = u < n16 ? ld_stream(c.gt.body + off) : pad;
-            d[q] = u < n16 ? ld_stream(c.gd.body + off) : pad;
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[q >> 1] += body_sum<ESIZE, kDrawResidual>(c, t[q], d[q]);
-    } else {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int u = s0 * kSubUnits + lane + 32 * q;
-            if (u < n16) {
-                UnitData ud;
-                ud.t = ld_stream(c.gt.body + static_cast<long long>(u) * 16);
-                ud.d = make_uint4(0u, 0u, 0u, 0u);
-                ud.count = kPer;
-                ud.first = c.gt.head + u * kPer;
-#pragma unroll
-                for (int e = 0; e < kPer; ++e)
-                    acc[q >> 1] += elem_weight<ESIZE, kDrawResidual>(c, ud, e);
-            }
-        }
-    }
-    if (lane == 0) {
-        if (s0 == 0 && c.gt.head > 0) acc[0] += partial_sum<ESIZE, kDrawResidual>(c, 0, c.gt.head);
-        if (c.gt.tail > 0 && (slast == s0 || slast == s0 + 1)) {
-            const float tw = partial_sum<ESIZE, kDrawResidual>(c, c.gt.head + n16 * kPer,
-                                                               c.gt.tail);
-            if (slast == s0) acc[0] += tw; else acc[1] += tw;
-        }
-    }
-#pragma unroll
-    for (int r = 0; r < 2; ++r)
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], o);
-    if (lane == 0) {
-        if (s0 < nsub) tbl[s0] = acc[0];
-        if (s0 + 1 < nsub) tbl[s0 + 1] = acc[1];
-    }
-}
+__global__ void __launch_bounds__(kDrawThreads, 3) resample_kernel(VerifyArgs a) {
+    __shared__ DrawSmem ds;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    griddep_wait();
+    // CTA w takes work entry w; the entries of every row with a draw were
+    // appended by the accept kernel, so all the work sits in the first CTAs.
+    if (static_cast<int>(blockIdx.x) >= __ldcg(&a.ctr[2])) return;
+    const int entry = __ldcg(&a.work[blockIdx.x]);
+    const int part = entry % kResidParts;
+    const int b = entry / kResidParts / a.C;
+    const int chunk = entry / kResidParts - b * a.C;
+    const int K = a.K, C = a.C;
+    const DrawRecord r = a.rec[b];   // written by the previous launch
+    if (r.mode == kDrawDone) return;
+    const bool resid = r.mode == kDrawResidual;
+    const int j = r.j;
 
-// Draw context of row b's final draw at position r.j from its record.
-template <int ESIZE>
-__device__ __forceinline__ DrawCtx draw_ctx(const VerifyArgs &a, int b, const DrawRecord &r) {
     DrawCtx c;
     c.k = r.k;
     c.mode = r.mode;
-    c.gt = vec_geom<ESIZE>(vec_ptr<ESIZE>(a, b, r.j), a.V);
+    c.gt = vec_geom<ESIZE>(vec_ptr<ESIZE>(a, b, j), a.V);
     c.mt = r.mt;
     c.ct = r.ct;
     c.xj = r.xj;
-    if (r.mode == kDrawResidual) {
-        c.gd = vec_geom<ESIZE>(vec_ptr<ESIZE>(a, b, a.K + 1 + r.j), a.V);
+    if (resid) {
+        c.gd = vec_geom<ESIZE>(vec_ptr<ESIZE>(a, b, K + 1 + j), a.V);
         c.md = r.md;
         c.cd = r.cd;
     } else {
         c.gd = c.gt; c.md = 0.f; c.cd = 0.f;
     }
     c.aligned = (c.gd.head == c.gt.head);
-    c.ubody0 = 0; c.nbody = 0; c.has_head = false; c.has_tail = false;
-    return c;
-}
-
-// Final draw of row b and its outputs, by the whole CTA.  Residual draws:
-// warp w forms the totals of chunks w, w + 8, ... from the sub-range table
-// (in the order the scan walks them); warp 0 then picks the chunk, the
-// sub-range inside it, and the token inside that.  p-mass draws (bonus,
-// greedy drafter): the chunk was chosen by the accept kernel; the CTA
-// splits it into warp segments, scans them and walks the elements.
-template <int ESIZE>
-__device__ __forceinline__ void finish_row(const VerifyArgs &a, int b, const DrawRecord &r, DrawSmem &ds,
-                           float *s_ct) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int K = a.K, C = a.C;
-    const bool resid = r.mode == kDrawResidual;
-    const int j = r.j;
-    DrawCtx c = draw_ctx<ESIZE>(a, b, r);
     auto set_chunk = [&](int cc) {
         c.ubody0 = cc * a.U;
         c.nbody = max(0, min(c.ubody0 + a.U, c.gt.n16) - c.ubody0);
@@ -1471,20 +1491,37 @@ __device__ __forceinline__ void finish_row(const VerifyArgs &a, int b, const Dra
     int y = -1;
     bool fb = false;
     if (resid) {
-        const float *tb = a.rtbl + static_cast<long long>(b) * a.nsub;
-        for (int cc = warp; cc < C; cc += kDrawWarps) {
+        // Residual weight of this chunk by sub-ranges; the last chunk CTA of
+        // the row (atomic counter, no waiting) picks the sub-range from the
+        // row's table and the token inside it.
+        set_chunk(chunk);
+        float *tb = a.rtbl + static_cast<long long>(b) * a.nsub;
+        float *ct = a.ctot + static_cast<long long>(b) * C;
+        residual_subranges<ESIZE>(c, chunk, part, a.U, tb);
+        __syncthreads();
+        if (warp == 0) {
+            // This chunk's total, formed as the last CTA's scan will walk it.
             int s0, s1;
-            chunk_subranges(c.gt, cc, a.U, &s0, &s1);
+            chunk_subranges(c.gt, chunk, a.U, &s0, &s1);
             const float tot = table_total(tb + s0, s1 - s0);
-            if (lane == 0) s_ct[cc] = tot;
+            if (lane == 0) ct[chunk] = tot;
+        }
+        if (tid == 0) {
+            __threadfence();
+            const int done = atomicAdd(&a.rcnt[b], 1) + 1;
+            __threadfence();
+            ds.last = (done == C * kResidParts);
         }
         __syncthreads();
+        if (!ds.last) return;
         if (warp == 0) {
             // Chunk totals in order, then the sub-ranges of the chosen chunk.
             bool zero = false, fbw = false;
             const int nsub = max(1, (c.gt.n16 + kSubUnits - 1) / kSubUnits);
+            const float w0 = lane < C ? __ldcg(ct + lane) : 0.f;
+            const float w1 = lane + 32 < C ? __ldcg(ct + lane + 32) : 0.f;
             float R = 0.f;
-            for (int q = 0; q < C; ++q) R += s_ct[q];
+            for (int q = 0; q < C; ++q) R += __shfl_sync(0xffffffffu, q < 32 ? w0 : w1, q & 31);
             int sel = -1;
             float dsel = 0.f;
             if (!(R > 0.f)) {
@@ -1494,7 +1531,7 @@ __device__ __forceinline__ void finish_row(const VerifyArgs &a, int b, const Dra
                 float cum = 0.f, tc = 0.f;
                 int cs = -1, clast = 0;
                 for (int q = 0; q < C; ++q) {
-                    const float w = s_ct[q];
+                    const float w = __shfl_sync(0xffffffffu, q < 32 ? w0 : w1, q & 31);
                     if (w > 0.f) clast = q;
                     if (cs < 0 && cum + w > t) { cs = q; tc = t - cum; }
                     if (cs < 0) cum += w;
@@ -1557,64 +1594,6 @@ __device__ __forceinline__ void finish_row(const VerifyArgs &a, int b, const Dra
         a.out_tokens[static_cast<long long>(b) * (K + 1) + t] = v;
     }
     if (tid == 0) a.out_accept[b] = j;
-    __syncthreads();   // shared state is reused by the CTA's next item
-}
-
-// ---------------------------------------------------------------------------
-// 4. Resample kernel: one persistent grid (three CTAs per SM) over the draws
-//    the accept kernel listed.  Items are dealt out in a fixed stride:
-//    first one item per p-mass draw (bonus, greedy drafter: the CTA locates
-//    the token inside the chosen chunk), then, for every residual draw, its
-//    items of kSumItemSubs sub-ranges of position j (warp w sums sub-ranges
-//    2w and 2w + 1, every load issued before the math).  The CTA that
-//    completes a row's last residual item (atomic count; nothing waits)
-//    picks the row's token at once.  Only position j of a rejecting row is
-//    read a second time.
-// ---------------------------------------------------------------------------
-template <int ESIZE>
-__global__ void __launch_bounds__(kSumThreads, 3) resample_kernel(VerifyArgs a) {
-    __shared__ DrawSmem ds;
-    __shared__ float s_ct[kMaxChunks];
-    __shared__ int s_last;
-    const int warp = threadIdx.x >> 5;
-    griddep_wait();
-    const int nres = __ldcg(&a.ctr[2]);
-    const int npm = __ldcg(&a.ctr[3]);
-    const int per_row = a.nitem;
-    const int total = npm + nres * per_row;   // < INT_MAX / 2 (checked by the plan)
-    for (int w = blockIdx.x; w < total; w += gridDim.x) {
-        int b;
-        bool finish = true;
-        if (w < npm) {
-            b = __ldcg(&a.work[a.B + w]);
-        } else {
-            const int e = (w - npm) / per_row;
-            const int item = (w - npm) - e * per_row;
-            b = __ldcg(&a.work[e]);
-            {
-                const DrawRecord r = a.rec[b];   // written by the accept kernel
-                const DrawCtx c = draw_ctx<ESIZE>(a, b, r);
-                const int nsub = max(1, (c.gt.n16 + kSubUnits - 1) / kSubUnits);
-                const int s0 = item * kSumItemSubs + 2 * warp;
-                if (s0 < nsub)
-                    subrange_pair<ESIZE>(c, s0, nsub,
-                                         a.rtbl + static_cast<long long>(b) * a.nsub);
-            }
-            __syncthreads();
-            if (threadIdx.x == 0) {
-                __threadfence();
-                const int done = atomicAdd(&a.rcnt[b], 1) + 1;
-                s_last = done == per_row;
-                if (s_last) __threadfence();
-            }
-            __syncthreads();
-            finish = s_last != 0;
-        }
-        if (finish) {
-            const DrawRecord r = a.rec[b];
-            finish_row<ESIZE>(a, b, r, ds, s_ct);
-        }
-    }
 }
 
 template <int ESIZE> static const void *stream_kernel_ptr() {
@@ -1627,9 +1606,9 @@ template <int ESIZE> static const void *stream_kernel_ptr() {
 struct Plan {
     int C, U, S;
     int nsub;
-    int nitem;
-    size_t off_rcnt, off_leff, off_rowj, off_pcnt, off_lvloff, off_lvlrow, off_part, off_rtbl,
-        off_work, off_rec, bytes;
+    size_t off_rcnt, off_leff, off_rowj, off_pcnt, off_lvloff, off_lvlrow, off_part, off_rtbl, off_ctot,
+        off_work,
+        off_rec, bytes;
 };
 
 static bool make_plan(int B, int K, int V, sv_dtype dtype, Plan *p) {
@@ -1660,9 +1639,8 @@ static bool make_plan(int B, int K, int V, sv_dtype dtype, Plan *p) {
     p->nsub = static_cast<int>((n16 + kSubUnits - 1) / kSubUnits);
     if (p->nsub < 1) p->nsub = 1;
     p->off_rtbl = off;   off = align16(off + sizeof(float) * static_cast<size_t>(B) * p->nsub);
-    p->nitem = (p->nsub + kSumItemSubs - 1) / kSumItemSubs;
-    if (static_cast<long long>(B) * (p->nitem + 1) >= INT_MAX / 2) return false;
-    p->off_work = off;   off = align16(off + 2 * iB);
+    p->off_ctot = off;   off = align16(off + sizeof(float) * static_cast<size_t>(B) * C);
+    p->off_work = off;   off = align16(off + sizeof(int) * static_cast<size_t>(B) * C * kResidParts);
     p->off_rec = off;    off = align16(off + sizeof(DrawRecord) * static_cast<size_t>(B));
     p->bytes = off;
     return true;
@@ -1691,30 +1669,6 @@ static int stream_grid(int esize, long long max_items) {
         n = sms * (per > 0 ? per : 1);
         slot.store(n, std::memory_order_relaxed);
     }
-    return static_cast<int>(max_items < n ? max_items : n);
-}
-
-// Persistent grid of the resample kernel: resident CTAs per SM x SMs
-// (cached per dtype and device), at most one CTA per item.
-static int resample_grid(int esize, long long max_items) {
-    static std::atomic<int> cache[2][64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
-    std::atomic<int> &slot = cache[esize == 4 ? 1 : 0][dev & 63];
-    int n = slot.load(std::memory_order_relaxed);
-    if (n == 0) {
-        int sms = 0, per = 0;
-        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return -1;
-        const void *fn = esize == 4 ? reinterpret_cast<const void *>(&resample_kernel<4>)
-                                    : reinterpret_cast<const void *>(&resample_kernel<2>);
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fn, kSumThreads, 0) !=
-            cudaSuccess)
-            return -1;
-        n = sms * (per > 0 ? per : 1);
-        slot.store(n, std::memory_order_relaxed);
-    }
-    if (max_items < 1) max_items = 1;
     return static_cast<int>(max_items < n ? max_items : n);
 }
 
@@ -1752,8 +1706,8 @@ static sv_status verify_impl(const void *zt, const void *zd, sv_dtype dtype, int
     a.lvl_row = reinterpret_cast<int *>(w + p.off_lvlrow);
     a.part = reinterpret_cast<float4 *>(w + p.off_part);
     a.rtbl = reinterpret_cast<float *>(w + p.off_rtbl);
+    a.ctot = reinterpret_cast<float *>(w + p.off_ctot);
     a.nsub = p.nsub;
-    a.nitem = p.nitem;
     a.work = reinterpret_cast<int *>(w + p.off_work);
     a.rec = reinterpret_cast<DrawRecord *>(w + p.off_rec);
 
@@ -1771,16 +1725,15 @@ static sv_status verify_impl(const void *zt, const void *zd, sv_dtype dtype, int
                   : launch_pdl(stream_kernel<2>, dim3(grid), dim3(kBlock), kRingBytes, st, a);
     if (e != cudaSuccess) return note_cuda(e);
     profile_mark_end(st);
-    const int rs_grid = resample_grid(es, static_cast<long long>(B) * (p.nitem + 1));
-    if (rs_grid <= 0) return note_cuda(cudaGetLastError());
+    const unsigned draw_grid = static_cast<unsigned>(B) * static_cast<unsigned>(p.C) * kResidParts;
     if (es == 4) {
         e = launch_pdl(accept_kernel<4>, dim3(B), dim3(kDrawThreads), 0, st, a);
         if (e == cudaSuccess)
-            e = launch_pdl(resample_kernel<4>, dim3(rs_grid), dim3(kSumThreads), 0, st, a);
+            e = launch_pdl(resample_kernel<4>, dim3(draw_grid), dim3(kDrawThreads), 0, st, a);
     } else {
         e = launch_pdl(accept_kernel<2>, dim3(B), dim3(kDrawThreads), 0, st, a);
         if (e == cudaSuccess)
-            e = launch_pdl(resample_kernel<2>, dim3(rs_grid), dim3(kSumThreads), 0, st, a);
+            e = launch_pdl(resample_kernel<2>, dim3(draw_grid), dim3(kDrawThreads), 0, st, a);
     }
     if (e != cudaSuccess) return note_cuda(e);
     return note_cuda(cudaGetLastError());

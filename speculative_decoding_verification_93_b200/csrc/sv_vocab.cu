@@ -44,6 +44,7 @@ constexpr int kStatsThreads = 256;
 constexpr int kStatsWarps = kStatsThreads / 32;
 constexpr int kBatch = 8;                      // 16-byte units per thread per load batch
 constexpr int kChunkBytes = 64 * 1024;         // target bytes per stats chunk
+constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s: no legitimate copy comes close
 constexpr int kMaxChunks = 64;
 constexpr int kDecideThreads = 256;
 constexpr int kDecideWarps = kDecideThreads / 32;
@@ -100,11 +101,24 @@ __device__ __forceinline__ const char *dft_vec(const Args &a, int b, int i) {
 }
 
 // ---------------------------------------------------------------------------
-// 1. Slice statistics.
+// 1. Slice statistics.  One CTA per (row, slot, chunk): the chunk's body is
+//    brought into shared memory by one bulk copy per piece of up to 32 KB
+//    (cp.async.bulk, mbarrier completion, no multicast), so a CTA holds no
+//    load registers and six CTAs fit on an SM: their copies stay in flight
+//    while other CTAs reduce.  Each thread reduces its units of the piece in
+//    two batches of four (packed bf16x2 max tree, one exp2 per element).
 // ---------------------------------------------------------------------------
+constexpr int kPieceUnits = 2048;                       // 16-byte units per bulk copy (32 KB)
+constexpr int kPieceBytes = kPieceUnits * 16;
+constexpr int kUnitsPerThread = kPieceUnits / kStatsThreads;   // 8
+static_assert(kUnitsPerThread == 8, "two batches of four units per thread");
+
 template <int ESIZE>
-__global__ void __launch_bounds__(kStatsThreads, 4) vp_stats_kernel(Args a) {
+__global__ void __launch_bounds__(kStatsThreads, 6) vp_stats_kernel(Args a) {
     constexpr int kPer = 16 / ESIZE;
+    extern __shared__ __align__(128) uint4 piece[];
+    __shared__ uint64_t full;
+    __shared__ float4 wp[kStatsWarps];
     griddep_wait();
     griddep_launch_dependents();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -132,6 +146,11 @@ __global__ void __launch_bounds__(kStatsThreads, 4) vp_stats_kernel(Args a) {
     const int u0 = min(c * U, g.n16), u1 = min(u0 + U, g.n16);
     const uint32_t pw = neg_inf_word<ESIZE>();
     const uint4 pad = make_uint4(pw, pw, pw, pw);
+    if (tid == 0) {
+        mbar_init(&full, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
 
     float m = kNegInf, s = 0.f;
     int idx = INT_MAX;
@@ -145,20 +164,49 @@ __global__ void __launch_bounds__(kStatsThreads, 4) vp_stats_kernel(Args a) {
             lse_update<ESIZE, 1>(h1, k, m, s);
         }
     }
-    for (int ub = u0; ub < u1; ub += kBatch * kStatsThreads) {
-        uint4 v[kBatch];
-#pragma unroll
-        for (int q = 0; q < kBatch; ++q) {
-            const int u = ub + q * kStatsThreads + tid;
-            v[q] = u < u1 ? ld_stream(g.body + static_cast<long long>(u) * 16) : pad;
+    bool ok = true;
+    uint32_t phase = 0;
+    for (int pb = u0; pb < u1 && ok; pb += kPieceUnits, phase ^= 1u) {
+        const int n = min(kPieceUnits, u1 - pb);
+        if (tid == 0) {
+            mbar_arrive_expect_tx(&full, static_cast<uint32_t>(n) * 16u);
+            bulk_g2s(piece, g.body + static_cast<long long>(pb) * 16, static_cast<uint32_t>(n) * 16u,
+                     &full);
         }
-        if (greedy) {
+        ok = mbar_wait(&full, phase, kWaitLimitNs);
+        if (ok) {
 #pragma unroll
-            for (int q = 0; q < kBatch; ++q)
-                consider_unit<ESIZE>(v[q], g.head + (ub + q * kStatsThreads + tid) * kPer, m, idx);
-        } else {
-            lse_update<ESIZE, kBatch>(v, k, m, s);
+            for (int h = 0; h < 2; ++h) {
+                uint4 v[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int u = (4 * h + q) * kStatsThreads + tid;
+                    v[q] = u < n ? piece[u] : pad;
+                }
+                if (greedy) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        consider_unit<ESIZE>(v[q], g.head + (pb + (4 * h + q) * kStatsThreads + tid) * kPer,
+                                             m, idx);
+                } else {
+                    lse_update<ESIZE, 4>(v, k, m, s);
+                }
+            }
         }
+        __syncthreads();   // the piece is consumed before the next copy overwrites it
+    }
+    if (!ok) {
+        // A copy that did not complete in time: wait (bounded) for it once
+        // more so that nothing lands after the block exits, and leave a NaN
+        // record, which the decide step turns into NaN normalisers.
+        if (tid == 0) {
+            mbar_wait(&full, phase, kWaitLimitNs / 4);
+            const float nan = __int_as_float(0x7fc00000);
+            a.stats_local[(static_cast<long long>(b) * a.S + slot) * a.C + c] =
+                make_float4(nan, nan, nan, 0.f);
+        }
+        __syncthreads();
+        return;
     }
     // Tail elements (last chunk, thread 1) follow every body element.
     if (c == a.C - 1 && tid == 1 && g.tail > 0) {
@@ -182,7 +230,6 @@ __global__ void __launch_bounds__(kStatsThreads, 4) vp_stats_kernel(Args a) {
             lse_merge(m, s, m2, s2, k);
         }
     }
-    __shared__ float4 wp[kStatsWarps];
     if (lane == 0) wp[warp] = make_float4(m, s, 0.f, __int_as_float(idx));
     __syncthreads();
     if (tid != 0) return;
@@ -836,9 +883,9 @@ extern "C" sv_status sv_vp_stats(const sv_vp_slice *s, const int32_t *draft_toke
     sv::profile_mark_begin(st);
     const cudaError_t e =
         p.es == 4 ? sv::launch_pdl(sv::vp::vp_stats_kernel<4>, dim3(grid),
-                                   dim3(sv::vp::kStatsThreads), 0, st, a)
+                                   dim3(sv::vp::kStatsThreads), sv::vp::kPieceBytes, st, a)
                   : sv::launch_pdl(sv::vp::vp_stats_kernel<2>, dim3(grid),
-                                   dim3(sv::vp::kStatsThreads), 0, st, a);
+                                   dim3(sv::vp::kStatsThreads), sv::vp::kPieceBytes, st, a);
     if (e != cudaSuccess) return sv::note_cuda(e);
     sv::profile_mark_end(st);
     return sv::note_cuda(cudaGetLastError());
