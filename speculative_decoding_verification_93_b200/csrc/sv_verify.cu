@@ -241,9 +241,6 @@ __device__ __forceinline__ void vstore(int &x, int v) {
 }
 
 constexpr int kItemSlots = 8;   // > kStages: consumer warps are never more than kStages items apart
-constexpr int kRowCache = 1024; // rows whose rejection marker each CTA keeps in shared memory
-constexpr int kClaimAhead = 4;  // claims in flight per producer
-constexpr uint32_t kIdleHintNs = 2000;   // publisher wait between marker refreshes
 
 struct ItemMeta {
     int b;        // row; -1 = no more items
@@ -266,12 +263,6 @@ struct StreamSmem {
     uint64_t ifull[kItemSlots];
     uint64_t ifree[kItemSlots];
     int abort;
-    // Copy of the first-rejection marker of rows 0..kRowCache-1: the
-    // publisher refreshes it from global memory whenever it is idle and
-    // lowers it at once for its own decisions; the producer classifies
-    // items from it without a round trip.  Markers only go down, so a
-    // stale entry costs redundant bytes, never a wrong result.
-    int rowj[kRowCache];
 };
 
 // Accept test of position i of row b, once every chunk partial of that
@@ -279,8 +270,8 @@ struct StreamSmem {
 // oracle: accept x_i iff u(seed, row, i, 0) < min(1, p_i(x_i) / q_i(x_i)),
 // greedy rows iff x_i is the target argmax.  A rejection lowers row_j[b].
 template <int ESIZE>
-__device__ void decide_position(const VerifyArgs &a, int *rowj_cache, int b, int i, int x,
-                                float zt_x, float zd_x) {
+__device__ void decide_position(const VerifyArgs &a, int b, int i, int x, float zt_x,
+                                float zd_x) {
     const int lane = threadIdx.x & 31;
     const int K = a.K, S = a.S, C = a.C;
     const float T = __ldg(&a.temp[b]);
@@ -332,10 +323,7 @@ __device__ void decide_position(const VerifyArgs &a, int *rowj_cache, int b, int
             else if (lq == kNegInf) acc = true;
             else acc = (lp >= lq) || (u < exp2f(lp - lq));
         }
-        if (!acc) {
-            atomicMin(&a.row_j[b], i);
-            if (b < kRowCache) atomicMin(&rowj_cache[b], i);
-        }
+        if (!acc) atomicMin(&a.row_j[b], i);
     }
 }
 
@@ -372,20 +360,23 @@ template <int ESIZE>
 __device__ void producer(const VerifyArgs &a, StreamSmem &sm, uint4 *ring, int total) {
     uint32_t it = 0;
     bool ok = true;
-    // Claims run kClaimAhead items ahead, so that each claim's round trip
-    // overlaps the items before it.  Items are classified from the shared
-    // copy of the rows' first-rejection markers when their turn comes, and
-    // a streamed item is checked again before every later stage: a skipped
-    // item costs a decode and no round trip.
-    auto marker = [&](int b) {
-        return b < kRowCache ? vload(sm.rowj[b]) : ld_relaxed(&a.row_j[b]);
-    };
-    int q[kClaimAhead];
-#pragma unroll
-    for (int k = 0; k < kClaimAhead; ++k) q[k] = atomicAdd(&a.ctr[0], 1);
+    // Claims run two items ahead.  While item k is classified, item k+1 is
+    // already decoded with its row's first-rejection marker requested, and
+    // the claim of item k+2 is in flight, so a run of skipped items costs
+    // about one decode each instead of a claim, a decode and a marker read
+    // in series.  The marker only ever goes down, so a stale value costs
+    // redundant bytes, never a wrong result; a streamed item reads it again
+    // before every stage (the read is issued before the wait for the slot).
+    int w0 = atomicAdd(&a.ctr[0], 1);
+    int w1 = atomicAdd(&a.ctr[0], 1);
+    ItemRef c0 = {0, 0, 0, 0};
+    int rj0 = 0;
+    if (w0 < total) {
+        c0 = decode_item(a, w0);
+        rj0 = ld_relaxed(&a.row_j[c0.b]);
+    }
     while (ok) {
-        const int w = q[0];
-        if (w >= total) {
+        if (w0 >= total) {
             const int st = it % kStages;
             const uint32_t ph = (it / kStages) & 1u;
             if (!mbar_wait(&sm.empty[st], ph ^ 1u, kWaitLimitNs)) { ok = false; break; }
@@ -394,15 +385,17 @@ __device__ void producer(const VerifyArgs &a, StreamSmem &sm, uint4 *ring, int t
             ++it;
             break;
         }
-        const int qn = (q[kClaimAhead - 1] < total) ? atomicAdd(&a.ctr[0], 1) : total;
-#pragma unroll
-        for (int k = 0; k + 1 < kClaimAhead; ++k) q[k] = q[k + 1];
-        q[kClaimAhead - 1] = qn;
-        const ItemRef cur = decode_item(a, w);
+        const int w2 = (w1 < total) ? atomicAdd(&a.ctr[0], 1) : total;
+        ItemRef c1 = {0, 0, 0, 0};
+        int rj1 = 0;
+        if (w1 < total) {
+            c1 = decode_item(a, w1);
+            rj1 = ld_relaxed(&a.row_j[c1.b]);
+        }
         // A row that has already rejected an earlier position never needs
         // this one: skip it without reading a byte.
-        if (marker(cur.b) >= cur.i) {
-            const int b = cur.b, i = cur.i, slot = cur.slot, chunk = cur.chunk;
+        if (rj0 >= c0.i) {
+            const int b = c0.b, i = c0.i, slot = c0.slot, chunk = c0.chunk;
             const float T = __ldg(&a.temp[b]);
             const float k = (T > 0.f) ? kLog2e / T : 0.f;
             const VecGeom g = vec_geom<ESIZE>(vec_ptr<ESIZE>(a, b, slot), a.V);
@@ -413,13 +406,14 @@ __device__ void producer(const VerifyArgs &a, StreamSmem &sm, uint4 *ring, int t
                 // Abandon the rest of the item once the row has rejected an
                 // earlier position: the consumers reset at the next item's
                 // first stage, and no partial of this item is ever read.
+                const int fresh = ld_relaxed(&a.row_j[b]);
                 const int st = it % kStages;
                 const uint32_t ph = (it / kStages) & 1u;
                 if (!mbar_wait(&sm.empty[st], ph ^ 1u, kWaitLimitNs) || vload(sm.abort)) {
                     ok = false;
                     break;
                 }
-                if (p > 0 && marker(b) < i) break;
+                if (fresh < i) break;
                 const int pu0 = u0 + p * kStageUnits;
                 const int pn = max(0, min(u1 - pu0, kStageUnits));
                 StageDesc &d = sm.desc[st];
@@ -438,6 +432,7 @@ __device__ void producer(const VerifyArgs &a, StreamSmem &sm, uint4 *ring, int t
                 ++it;
             }
         }
+        w0 = w1; c0 = c1; rj0 = rj1; w1 = w2;
     }
     if (!ok) {
         // Unwind: report, then wait (bounded) for the copies still in flight
@@ -582,34 +577,10 @@ __device__ void consumers(const VerifyArgs &a, StreamSmem &sm, const uint4 *ring
 template <int ESIZE>
 __device__ void publisher(const VerifyArgs &a, StreamSmem &sm) {
     const int lane = threadIdx.x & 31;
-    const int ncache = min(a.B, kRowCache);
     uint32_t iseq = 0;
     while (true) {
         const uint32_t slot_i = iseq % kItemSlots, use = iseq / kItemSlots;
-        // Wait for the next item; while idle, refresh the marker copy (one
-        // round of loads per refresh, eight rows per lane in flight).
-        bool got = __all_sync(0xffffffffu, mbar_try_wait_hint(&sm.ifull[slot_i], use & 1u,
-                                                              kIdleHintNs));
-        const uint64_t t0 = got ? 0 : global_ns();
-        while (!got && !vload(sm.abort)) {
-            for (int r0 = 0; r0 < ncache; r0 += 32 * 8) {
-                int v[8];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const int r = r0 + q * 32 + lane;
-                    v[q] = r < ncache ? ld_relaxed(&a.row_j[r]) : INT_MAX;
-                }
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const int r = r0 + q * 32 + lane;
-                    if (r < ncache) atomicMin(&sm.rowj[r], v[q]);
-                }
-            }
-            if (global_ns() - t0 > kWaitLimitNs) break;
-            got = __all_sync(0xffffffffu, mbar_try_wait_hint(&sm.ifull[slot_i], use & 1u,
-                                                             kIdleHintNs));
-        }
-        if (!got || vload(sm.abort)) {
+        if (!mbar_wait(&sm.ifull[slot_i], use & 1u, kWaitLimitNs) || vload(sm.abort)) {
             vstore(sm.abort, 1);
             if (a.status && lane == 0) atomicOr(a.status, SV_NOTE_TIMEOUT);
             break;
@@ -663,7 +634,7 @@ __device__ void publisher(const VerifyArgs &a, StreamSmem &sm) {
             x = __shfl_sync(0xffffffffu, x, 0);
             zt_x = __shfl_sync(0xffffffffu, zt_x, 0);
             zd_x = __shfl_sync(0xffffffffu, zd_x, 0);
-            decide_position<ESIZE>(a, sm.rowj, im.b, im.level, x, zt_x, zd_x);
+            decide_position<ESIZE>(a, im.b, im.level, x, zt_x, zd_x);
         }
     }
 }
@@ -690,8 +661,6 @@ __global__ void __launch_bounds__(kBlock, 3) stream_kernel(VerifyArgs a) {
     }
     __syncthreads();
     griddep_wait();
-    for (int b = tid; b < min(a.B, kRowCache); b += kBlock) sm.rowj[b] = __ldcg(&a.row_j[b]);
-    __syncthreads();
     const int total = __ldcg(&a.ctr[1]);
     if (tid >= kConsumers + 32) {
         publisher<ESIZE>(a, sm);
