@@ -42,7 +42,6 @@ namespace vp {
 
 constexpr int kStatsThreads = 256;
 constexpr int kStatsWarps = kStatsThreads / 32;
-constexpr int kBatch = 8;                      // 16-byte units per thread per load batch
 constexpr int kChunkBytes = 64 * 1024;         // target bytes per stats chunk
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s: no legitimate copy comes close
 constexpr int kMaxChunks = 64;
