@@ -204,8 +204,8 @@ int sv_debug_sts_timeouts(void);
  * (B, K, V, dtype): work counters, per-row state (length, first rejection
  * found so far, per-position completion counts), the position-major work
  * list, the per-chunk softmax partials, the residual draw table and the
- * resample work list: about B * V * elt / 256 + B * (2K+1) * V * elt / 4096
- * bytes (0.58 MB at B = 256, K = 8, V = 129280 bf16).  Returns 0 for
+ * resample work list: about B * V * elt / 256 + B * (2K+1) * V * elt / 8192
+ * bytes (0.44 MB at B = 256, K = 8, V = 129280 bf16).  Returns 0 for
  * unsupported sizes.
  */
 size_t sv_verify_workspace_bytes(int B, int K, int V, sv_dtype dtype);

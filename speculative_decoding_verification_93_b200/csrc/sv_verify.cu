@@ -64,7 +64,7 @@ constexpr int kBlock = kConsumers + 64;           // + one producer and one publ
 constexpr int kStages = 4;                        // shared-memory ring depth
 constexpr int kStageUnits = 1024;                 // 16-byte units per stage (16 KB)
 constexpr int kRingBytes = kStages * kStageUnits * 16;
-constexpr int kMaxUnitsPerItem = 4 * kStageUnits; // an item spans up to 4 stages
+constexpr int kMaxUnitsPerItem = 8 * kStageUnits; // an item spans up to 8 stages (128 KB)
 constexpr int kMaxSlots = 2 * SV_MAX_K + 1;
 constexpr int kMaxChunks = 64;                    // V <= SV_MAX_V keeps C within this
 constexpr int kPrologueThreads = 1024;
@@ -360,23 +360,14 @@ template <int ESIZE>
 __device__ void producer(const VerifyArgs &a, StreamSmem &sm, uint4 *ring, int total) {
     uint32_t it = 0;
     bool ok = true;
-    // Claims run two items ahead.  While item k is classified, item k+1 is
-    // already decoded with its row's first-rejection marker requested, and
-    // the claim of item k+2 is in flight, so a run of skipped items costs
-    // about one decode each instead of a claim, a decode and a marker read
-    // in series.  The marker only ever goes down, so a stale value costs
-    // redundant bytes, never a wrong result; a streamed item reads it again
-    // before every stage (the read is issued before the wait for the slot).
-    int w0 = atomicAdd(&a.ctr[0], 1);
-    int w1 = atomicAdd(&a.ctr[0], 1);
-    ItemRef c0 = {0, 0, 0, 0};
-    int rj0 = 0;
-    if (w0 < total) {
-        c0 = decode_item(a, w0);
-        rj0 = ld_relaxed(&a.row_j[c0.b]);
-    }
+    // The next claim is taken as the current item starts, so that the
+    // counter's round trip overlaps the item.  The row's status is read when
+    // the item's turn comes and again before each later stage: a rejection
+    // only ever lowers it, so a stale value costs redundant bytes, never a
+    // wrong result.
+    int w = atomicAdd(&a.ctr[0], 1);
     while (ok) {
-        if (w0 >= total) {
+        if (w >= total) {
             const int st = it % kStages;
             const uint32_t ph = (it / kStages) & 1u;
             if (!mbar_wait(&sm.empty[st], ph ^ 1u, kWaitLimitNs)) { ok = false; break; }
@@ -385,17 +376,13 @@ __device__ void producer(const VerifyArgs &a, StreamSmem &sm, uint4 *ring, int t
             ++it;
             break;
         }
-        const int w2 = (w1 < total) ? atomicAdd(&a.ctr[0], 1) : total;
-        ItemRef c1 = {0, 0, 0, 0};
-        int rj1 = 0;
-        if (w1 < total) {
-            c1 = decode_item(a, w1);
-            rj1 = ld_relaxed(&a.row_j[c1.b]);
-        }
+        const ItemRef cur = decode_item(a, w);
+        const int rj = ld_relaxed(&a.row_j[cur.b]);
+        const int wnext = atomicAdd(&a.ctr[0], 1);
         // A row that has already rejected an earlier position never needs
         // this one: skip it without reading a byte.
-        if (rj0 >= c0.i) {
-            const int b = c0.b, i = c0.i, slot = c0.slot, chunk = c0.chunk;
+        if (rj >= cur.i) {
+            const int b = cur.b, i = cur.i, slot = cur.slot, chunk = cur.chunk;
             const float T = __ldg(&a.temp[b]);
             const float k = (T > 0.f) ? kLog2e / T : 0.f;
             const VecGeom g = vec_geom<ESIZE>(vec_ptr<ESIZE>(a, b, slot), a.V);
@@ -406,14 +393,13 @@ __device__ void producer(const VerifyArgs &a, StreamSmem &sm, uint4 *ring, int t
                 // Abandon the rest of the item once the row has rejected an
                 // earlier position: the consumers reset at the next item's
                 // first stage, and no partial of this item is ever read.
-                const int fresh = ld_relaxed(&a.row_j[b]);
+                if (p > 0 && ld_relaxed(&a.row_j[b]) < i) break;
                 const int st = it % kStages;
                 const uint32_t ph = (it / kStages) & 1u;
                 if (!mbar_wait(&sm.empty[st], ph ^ 1u, kWaitLimitNs) || vload(sm.abort)) {
                     ok = false;
                     break;
                 }
-                if (fresh < i) break;
                 const int pu0 = u0 + p * kStageUnits;
                 const int pn = max(0, min(u1 - pu0, kStageUnits));
                 StageDesc &d = sm.desc[st];
@@ -432,7 +418,7 @@ __device__ void producer(const VerifyArgs &a, StreamSmem &sm, uint4 *ring, int t
                 ++it;
             }
         }
-        w0 = w1; c0 = c1; rj0 = rj1; w1 = w2;
+        w = wnext;
     }
     if (!ok) {
         // Unwind: report, then wait (bounded) for the copies still in flight
@@ -801,7 +787,12 @@ __device__ __forceinline__ float unit_sum(const DrawCtx &c, const UnitData &u) {
     return t;
 }
 
-constexpr int kRunMax = 4;      // units per thread in the located segment
+// Units per thread in the located segment of a chunk: a chunk of at most
+// kMaxUnitsPerItem body units plus head and tail, split into kDrawWarps
+// segments, each spread over the kDrawThreads threads of the CTA.
+constexpr int kRunMax =
+    (((kMaxUnitsPerItem + 2 + kDrawWarps - 1) / kDrawWarps) + kDrawThreads - 1) / kDrawThreads;
+static_assert(kRunMax == 5, "128 KB items: five units per thread in the located segment");
 
 // Segment g of the chunk (for warp g of the draw CTA): local units
 // [g * SU, min((g+1) * SU, NU)), SU = ceil(NU / kDrawWarps).

@@ -41,6 +41,9 @@ SMALL = [
     (1000, torch.bfloat16, 4, 32), (1001, torch.bfloat16, 6, 32), (1003, torch.float32, 2, 24),
     (4099, torch.float32, 3, 16), (8193, torch.bfloat16, 7, 16), (20011, torch.float32, 3, 12),
     (40000, torch.bfloat16, 4, 12), (65543, torch.bfloat16, 2, 8),
+    # chunks of exactly 8192 16-byte units (the largest item): the p-mass
+    # draw spreads a chunk segment over five units per thread
+    (131072, torch.bfloat16, 2, 16), (65536, torch.float32, 2, 16),
 ]
 
 
@@ -98,7 +101,7 @@ def test_normalisers_match_oracle(V, dtype):
 
 
 @pytest.mark.parametrize("V,dtype", [(7, torch.float32), (1000, torch.bfloat16),
-                                     (129280, torch.bfloat16)])
+                                     (129280, torch.bfloat16), (131072, torch.bfloat16)])
 def test_greedy_drafter_matches_oracle(V, dtype):
     b = _cuda(workloads.random_small(24, 5, V, dtype=dtype, seed=11, temps=(0.0, 0.7, 1.0)))
     for seed in (1, 2):
