@@ -286,11 +286,11 @@ def workload_config(batch, lengths_np, esize):
           "(a 256 MB buffer written, then another read), each step timed alone with CUDA "
           "events" if needs_flush(batch, esize) else
           f"inputs {inputs / 1e9:.2f} GB > 126 MB L2 (no flush; steps back to back)")
-    return {"workload": (f"{s.name}: B={s.B} K={s.K} V={s.V} {dt} logits; "
+    return {"workload": (f"{s.name}: B={int(batch.zt.shape[0])} K={s.K} V={s.V} {dt} logits; "
                          f"T per row from {list(s.temps)}; "
                          + (f"lengths from sv_schedule (conf~Beta{s.beta}, tau={batch.tau})"
                             if s.fixed_length is None else f"lengths={s.fixed_length}")),
-            "B": s.B, "K": s.K, "V": s.V, "logits": dt,
+            "B": int(batch.zt.shape[0]), "K": s.K, "V": s.V, "logits": dt,
             "tau": batch.tau if s.fixed_length is None else None,
             "mean_L": float(lengths_np.mean()),
             "l2": l2,
@@ -378,9 +378,10 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         import torch.distributed as dist
     batch = workloads.make_batch(args.workload, device=dev, tau=args.tau,
+                                 B=args.rows if args.rows > 0 else None,
                                  data_seed=workloads.SPECS[args.workload].data_seed + 1000 * rank)
     s = batch.spec
-    B, K, V = s.B, s.K, s.V
+    B, K, V = int(batch.zt.shape[0]), s.K, s.V
     esize = 2 if s.dtype == torch.bfloat16 else 4
     dt = sv.SV_BF16 if esize == 2 else sv.SV_F32
     ws = torch.empty(sv.sv_verify_workspace_bytes(B, K, V, dt), dtype=torch.uint8, device=dev)
@@ -735,6 +736,9 @@ def main():
     ap.add_argument("--tau", type=float, default=None,
                     help="schedule threshold for workloads with scheduled lengths "
                          "(default: the workload's first)")
+    ap.add_argument("--rows", type=int, default=0,
+                    help="rows of the batch (0: the workload's own B); smaller batches of the "
+                         "same workload for profiler captures")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--cpu-1core-seconds", type=float, default=5.0)
     ap.add_argument("--parity-seconds", type=float, default=15.0)
