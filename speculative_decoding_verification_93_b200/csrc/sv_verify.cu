@@ -169,10 +169,11 @@ __global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(VerifyArgs a
         a.leff[b] = Lb;
         a.row_j[b] = Lb;
         a.rcnt[b] = 0;
-        for (int i = 0; i < K1; ++i) a.pcnt[static_cast<long long>(b) * K1 + i] = 0;
         if (b < kPrologueSmemRows)
             s_row[b] = Lb < 0 ? -1 : (Lb | ((draft && a.temp[b] > 0.f) ? (1 << 30) : 0));
     }
+    // Completion counts of every (row, position), zeroed with coalesced stores.
+    for (long long q = tid; q < static_cast<long long>(a.B) * K1; q += kPrologueThreads) a.pcnt[q] = 0;
     __syncthreads();
     // Levels: warp w scans levels w, w + 32, ... over the rows.
     for (int i = warp; i < K1; i += kPrologueThreads / 32) {
@@ -1051,7 +1052,6 @@ __device__ __forceinline__ void chunk_masses(const VerifyArgs &a, int b, int j, 
 constexpr int kSubUnits = 64;   // units per sub-range; chunk sizes are multiples of it
 constexpr int kRunUnits = 3;    // local units per lane in a located sub-range (66 / 32)
 constexpr int kResidParts = 1;  // resample CTAs per chunk of a residual draw
-static_assert(kResidParts == 1, "each chunk CTA forms its chunk's residual total");
 
 // Draw weight of `count` (< one unit) elements from element `first`,
 // loaded directly (vector head or tail).
@@ -1490,7 +1490,7 @@ __global__ void __launch_bounds__(kDrawThreads, 3) resample_kernel(VerifyArgs a)
         float *ct = a.ctot + static_cast<long long>(b) * C;
         residual_subranges<ESIZE>(c, chunk, part, a.U, tb);
         __syncthreads();
-        if (warp == 0) {
+        if (kResidParts == 1 && warp == 0) {
             // This chunk's total, formed as the last CTA's scan will walk it.
             int s0, s1;
             chunk_subranges(c.gt, chunk, a.U, &s0, &s1);
@@ -1505,6 +1505,18 @@ __global__ void __launch_bounds__(kDrawThreads, 3) resample_kernel(VerifyArgs a)
         }
         __syncthreads();
         if (!ds.last) return;
+        if (kResidParts > 1) {
+            // A chunk's sub-ranges came from several CTAs: the last CTA forms
+            // every chunk total (warp w: chunks w, w + 8, ...), in the order
+            // its scan will walk them.
+            for (int cc = warp; cc < C; cc += kDrawWarps) {
+                int s0, s1;
+                chunk_subranges(c.gt, cc, a.U, &s0, &s1);
+                const float tot = table_total(tb + s0, s1 - s0);
+                if (lane == 0) ct[cc] = tot;
+            }
+            __syncthreads();
+        }
         if (warp == 0) {
             // Chunk totals in order, then the sub-ranges of the chosen chunk.
             bool zero = false, fbw = false;
