@@ -1138,88 +1138,6 @@ __device__ void residual_subranges(const DrawCtx &c, int ch, int part, int U, fl
     }
 }
 
-// Residual weight of every sub-range of chunk `ch` into tbl, with the
-// chunk's target and draft blocks brought into shared memory by bulk copies
-// (cp.async.bulk, mbarrier completion, no multicast): kRsStages slots of
-// kRsStageUnits units of each vector, refilled by thread 0 once every warp
-// has passed the slot, so the copies of later stages are in flight while
-// the warps reduce the current one.  Warp w sums sub-range w of each stage
-// (lane l: unit l, then unit l + 32; the head joins sub-range 0 and the
-// tail the last one; then a fixed shuffle tree), the same order as
-// residual_subranges, so the table is identical.  Needs the draft vector in
-// the target's 16-byte phase and at least one body unit in the chunk.
-// Returns false if a copy did not complete within the wait bound (after
-// waiting, bounded, for the copies still in flight).
-constexpr int kRsStageUnits = kDrawWarps * kSubUnits;   // 512 units = 8 KB of each vector
-constexpr int kRsStages = 4;
-constexpr int kRsRingBytes = kRsStages * 2 * kRsStageUnits * 16;   // 64 KB
-constexpr uint64_t kRsWaitNs = 1000000000ull;
-
-// Bulk copies of stage st of a chunk's body units [u0, u1): the target and
-// the draft block into their halves of ring slot st % kRsStages.
-__device__ __forceinline__ void rs_issue(const char *tbody, const char *dbody, int u0, int u1,
-                                         int st, uint4 *ring, uint64_t *full) {
-    const int slot = st % kRsStages;
-    const int b0 = u0 + st * kRsStageUnits;
-    const uint32_t n = static_cast<uint32_t>(min(kRsStageUnits, u1 - b0));
-    uint4 *dst = ring + static_cast<size_t>(slot) * 2 * kRsStageUnits;
-    mbar_arrive_expect_tx(&full[slot], 2u * n * 16u);
-    bulk_g2s(dst, tbody + static_cast<long long>(b0) * 16, n * 16u, &full[slot]);
-    bulk_g2s(dst + kRsStageUnits, dbody + static_cast<long long>(b0) * 16, n * 16u, &full[slot]);
-}
-
-template <int ESIZE>
-__device__ __forceinline__ bool residual_subranges_ring(const DrawCtx &c, int ch, int U, float *tbl,
-                                        uint4 *ring, uint64_t *full) {
-    constexpr int kPer = 16 / ESIZE;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int u0 = ch * U;
-    const int u1 = max(u0, min(u0 + U, c.gt.n16));
-    const int nstage = (u1 - u0 + kRsStageUnits - 1) / kRsStageUnits;
-    const int slast = c.gt.n16 > 0 ? (c.gt.n16 - 1) / kSubUnits : 0;
-    const uint32_t pw = neg_inf_word<ESIZE>();
-    const uint4 pad = make_uint4(pw, pw, pw, pw);
-    if (tid == 0)
-        for (int st = 0; st < min(nstage, kRsStages); ++st)
-            rs_issue(c.gt.body, c.gd.body, u0, u1, st, ring, full);
-    bool ok = true;
-    int st = 0;
-    for (; st < nstage; ++st) {
-        const int slot = st % kRsStages;
-        const uint32_t par = (st / kRsStages) & 1u;
-        ok = mbar_wait(&full[slot], par, kRsWaitNs);
-        if (!__syncthreads_and(ok)) { ok = false; break; }
-        const int b0 = u0 + st * kRsStageUnits;
-        const int n = min(kRsStageUnits, u1 - b0);
-        const uint4 *rt = ring + static_cast<size_t>(slot) * 2 * kRsStageUnits;
-        const uint4 *rd = rt + kRsStageUnits;
-        const int l0 = warp * kSubUnits + lane, l1 = l0 + 32;
-        float acc = 0.f;
-        acc += body_sum<ESIZE, kDrawResidual>(c, l0 < n ? rt[l0] : pad, l0 < n ? rd[l0] : pad);
-        acc += body_sum<ESIZE, kDrawResidual>(c, l1 < n ? rt[l1] : pad, l1 < n ? rd[l1] : pad);
-        const int s = b0 / kSubUnits + warp;   // this warp's sub-range
-        if (lane == 0) {
-            if (s == 0 && c.gt.head > 0) acc += partial_sum<ESIZE, kDrawResidual>(c, 0, c.gt.head);
-            if (c.gt.tail > 0 && s == slast)
-                acc += partial_sum<ESIZE, kDrawResidual>(c, c.gt.head + c.gt.n16 * kPer,
-                                                         c.gt.tail);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (lane == 0 && s * kSubUnits < u1) tbl[s] = acc;
-        __syncthreads();   // every warp is past this slot
-        if (tid == 0 && st + kRsStages < nstage)
-            rs_issue(c.gt.body, c.gd.body, u0, u1, st + kRsStages, ring, full);
-    }
-    if (!ok && tid == 0) {
-        // Wait (bounded) for every copy still in flight, so that none lands
-        // in shared memory after the block exits.
-        for (int q = st; q < min(nstage, st + kRsStages); ++q)
-            mbar_wait(&full[q % kRsStages], (q / kRsStages) & 1u, kRsWaitNs / 4);
-    }
-    return ok;
-}
-
 // Sum of n table entries by one warp: rounds of 32 entries in order, a
 // fixed tree inside each round.  table_find walks the entries in the same
 // rounds, so a target below this total always finds its entry.
@@ -1521,8 +1439,6 @@ __global__ void __launch_bounds__(kDrawThreads) accept_kernel(VerifyArgs a) {
 // ---------------------------------------------------------------------------
 template <int ESIZE>
 __global__ void __launch_bounds__(kDrawThreads, 3) resample_kernel(VerifyArgs a) {
-    extern __shared__ __align__(128) uint4 rs_ring[];   // kRsRingBytes
-    __shared__ uint64_t rs_full[kRsStages];
     __shared__ DrawSmem ds;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     griddep_wait();
@@ -1572,21 +1488,7 @@ __global__ void __launch_bounds__(kDrawThreads, 3) resample_kernel(VerifyArgs a)
         set_chunk(chunk);
         float *tb = a.rtbl + static_cast<long long>(b) * a.nsub;
         float *ct = a.ctot + static_cast<long long>(b) * C;
-        const bool ring = kResidParts == 1 && c.aligned &&
-                          min(chunk * a.U + a.U, c.gt.n16) > chunk * a.U;
-        if (ring) {
-            if (tid == 0) {
-                for (int q = 0; q < kRsStages; ++q) mbar_init(&rs_full[q], 1);
-                fence_mbar_init();
-            }
-            __syncthreads();
-            if (!residual_subranges_ring<ESIZE>(c, chunk, a.U, tb, rs_ring, rs_full)) {
-                if (tid == 0 && a.status) atomicOr(a.status, SV_NOTE_TIMEOUT);
-                return;
-            }
-        } else {
-            residual_subranges<ESIZE>(c, chunk, part, a.U, tb);
-        }
+        residual_subranges<ESIZE>(c, chunk, part, a.U, tb);
         __syncthreads();
         if (kResidParts == 1 && warp == 0) {
             // This chunk's total, formed as the last CTA's scan will walk it.
@@ -1773,24 +1675,6 @@ static int stream_grid(int esize, long long max_items) {
     return static_cast<int>(max_items < n ? max_items : n);
 }
 
-// The resample kernel's bulk-copy ring needs more than the default 48 KB of
-// dynamic shared memory: opt in once per (dtype, device).  Threads that race
-// on an unset entry set the same attribute.
-static bool resample_smem_ready(int esize) {
-    static std::atomic<bool> done[2][64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return false;
-    std::atomic<bool> &d = done[esize == 4 ? 1 : 0][dev & 63];
-    if (d.load(std::memory_order_acquire)) return true;
-    const void *fn = esize == 4 ? reinterpret_cast<const void *>(&resample_kernel<4>)
-                                : reinterpret_cast<const void *>(&resample_kernel<2>);
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kRsRingBytes) !=
-        cudaSuccess)
-        return false;
-    d.store(true, std::memory_order_release);
-    return true;
-}
-
 static sv_status verify_impl(const void *zt, const void *zd, sv_dtype dtype, int B, int K, int V,
                              const int32_t *tokens, const int32_t *lengths, const float *temp,
                              uint64_t seed, int64_t row_base, int32_t *out_tokens,
@@ -1845,17 +1729,14 @@ static sv_status verify_impl(const void *zt, const void *zd, sv_dtype dtype, int
     if (e != cudaSuccess) return note_cuda(e);
     profile_mark_end(st);
     const unsigned draw_grid = static_cast<unsigned>(B) * static_cast<unsigned>(p.C) * kResidParts;
-    if (!resample_smem_ready(es)) return note_cuda(cudaGetLastError());
     if (es == 4) {
         e = launch_pdl(accept_kernel<4>, dim3(B), dim3(kDrawThreads), 0, st, a);
         if (e == cudaSuccess)
-            e = launch_pdl(resample_kernel<4>, dim3(draw_grid), dim3(kDrawThreads), kRsRingBytes,
-                           st, a);
+            e = launch_pdl(resample_kernel<4>, dim3(draw_grid), dim3(kDrawThreads), 0, st, a);
     } else {
         e = launch_pdl(accept_kernel<2>, dim3(B), dim3(kDrawThreads), 0, st, a);
         if (e == cudaSuccess)
-            e = launch_pdl(resample_kernel<2>, dim3(draw_grid), dim3(kDrawThreads), kRsRingBytes,
-                           st, a);
+            e = launch_pdl(resample_kernel<2>, dim3(draw_grid), dim3(kDrawThreads), 0, st, a);
     }
     if (e != cudaSuccess) return note_cuda(e);
     return note_cuda(cudaGetLastError());
