@@ -203,9 +203,9 @@ int sv_debug_sts_timeouts(void);
  * sv_verify_workspace_bytes -- device scratch that sv_verify needs for
  * (B, K, V, dtype): work counters, per-row state (length, first rejection
  * found so far, per-position completion counts), the position-major work
- * list, the per-chunk softmax partials, the residual draw table and the
- * resample work list: about B * V * elt / 256 + B * (2K+1) * V * elt / 8192
- * bytes (0.44 MB at B = 256, K = 8, V = 129280 bf16).  Returns 0 for
+ * list, the per-chunk softmax partials and the residual draw table: about
+ * B * V * elt / 256 + B * (2K+1) * V * elt / 8192 bytes (0.42 MB at
+ * B = 256, K = 8, V = 129280 bf16).  Returns 0 for
  * unsupported sizes.
  */
 size_t sv_verify_workspace_bytes(int B, int K, int V, sv_dtype dtype);

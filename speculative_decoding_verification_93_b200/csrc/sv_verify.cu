@@ -35,17 +35,17 @@
 //      runs the accept test of a position as soon as it is complete,
 //      lowering the row's first-rejection marker on a rejection.  Every
 //      mbarrier wait is bounded in wall time and reports SV_NOTE_TIMEOUT.
-//   3. accept_kernel (one CTA per row): settles j = first rejection (or L),
-//      merges the normalisers of positions 0..j, writes greedy rows, sets up
-//      each sampled row's final draw (for p-mass draws the chunk is chosen
-//      from the stream partials) and appends the resample work list.
-//   4. resample_kernel (one CTA per work entry): residual draws sum
-//      max(0, p_j - q_j) over their chunk by 64-unit sub-ranges, and each
-//      chunk CTA also forms its chunk's total in the order the scan will
-//      walk it; the last chunk CTA of the row (atomic counter, no waiting)
-//      picks the chunk from the chunk totals, the sub-range from that
-//      chunk's sub-ranges, and the token inside it.  p-mass draws locate
-//      the token inside the chosen chunk.  Only position j of a rejecting
+//   3. draw_kernel (one CTA per row and chunk), launched while the stream
+//      kernel runs: each CTA waits until its row is settled (the publisher
+//      sets a bit per accepted position; a rejection lowers the marker),
+//      then merges the normalisers of position j from the stream partials.
+//      Greedy rows: the argmax.  p-mass draws: the row's lead CTA picks the
+//      chunk from the partials' masses and locates the token inside it.
+//      Residual draws: every chunk CTA sums max(0, p_j - q_j) over its
+//      chunk by 64-unit sub-ranges; the last chunk CTA of the row (atomic
+//      count, no waiting) stages the row's sub-range table, forms the chunk
+//      totals in the order its scan walks them, and picks the chunk, the
+//      sub-range and the token inside it.  Only position j of a rejecting
 //      row is read a second time.
 #include <climits>
 #include <cstdint>
@@ -82,19 +82,17 @@ struct VerifyArgs {
     int32_t *out_accept;       // [B]
     int32_t *status;           // nullable
     float *dbg;                // nullable [B, S, 2]
-    int *ctr;                  // [0] next item, [1] total items, [2] resample work entries
+    int *ctr;                  // [0] next item, [1] total items, [2] a wait ran out
     int *rcnt;                 // [B]  chunks of the residual draw done
     int *leff;                 // [B]  verify length of a valid row, -1 for an invalid one
     int *row_j;                // [B]  first rejection found so far (starts at L)
     int *pcnt;                 // [B, K+1] item partials published per (row, position)
+    unsigned long long *dec;   // [B]  positions accepted (bit i)
     int *lvl_off;              // [K+2] first item of each position level
     int *lvl_row;              // [K+1, B+1] per-level exclusive prefix of row item counts
     float4 *part;              // [B, S, C]: (m, s, argmax bits, 0)
     float *rtbl;               // [B, nsub] residual mass per sub-range
-    float *ctot;               // [B, C] residual mass per chunk (its sub-ranges, in scan order)
     int nsub;                  // sub-ranges per row
-    int *work;                 // [B * C] (row * C + chunk) of the resample CTAs with work
-    struct DrawRecord *rec;    // [B] accept result and draw set-up
 };
 
 template <int ESIZE>
@@ -169,6 +167,7 @@ __global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(VerifyArgs a
         a.leff[b] = Lb;
         a.row_j[b] = Lb;
         a.rcnt[b] = 0;
+        a.dec[b] = 0ull;
         if (b < kPrologueSmemRows)
             s_row[b] = Lb < 0 ? -1 : (Lb | ((draft && a.temp[b] > 0.f) ? (1 << 30) : 0));
     }
@@ -324,8 +323,18 @@ __device__ void decide_position(const VerifyArgs &a, int b, int i, int x, float 
             else if (lq == kNegInf) acc = true;
             else acc = (lp >= lq) || (u < exp2f(lp - lq));
         }
+        // A rejection lowers the row's marker, an acceptance sets the
+        // position's bit: the draw kernel settles a row from the two.
         if (!acc) atomicMin(&a.row_j[b], i);
+        else red_or_relaxed(&a.dec[b], 1ull << i);
     }
+}
+
+// A wait that ran out: raise the status note, and tell the draw CTAs that
+// rows may never settle.
+__device__ __forceinline__ void report_timeout(const VerifyArgs &a) {
+    if (a.status) atomicOr(a.status, SV_NOTE_TIMEOUT);
+    atomicExch(&a.ctr[2], 1);
 }
 
 // Producer: fetch items (global atomic counter, prefetched one item ahead),
@@ -425,7 +434,7 @@ __device__ void producer(const VerifyArgs &a, StreamSmem &sm, uint4 *ring, int t
         // Unwind: report, then wait (bounded) for the copies still in flight
         // so that none lands in shared memory after the block exits.
         vstore(sm.abort, 1);
-        if (a.status) atomicOr(a.status, SV_NOTE_TIMEOUT);
+        report_timeout(a);
         const uint32_t n = it < kStages ? it : kStages;
         for (uint32_t i = 0; i < n; ++i) {
             const uint32_t t = it - 1 - i;
@@ -452,7 +461,7 @@ __device__ void consumers(const VerifyArgs &a, StreamSmem &sm, const uint4 *ring
         const uint32_t ph = (it / kStages) & 1u;
         if (!mbar_wait(&sm.full[st], ph, kWaitLimitNs) || vload(sm.abort)) {
             vstore(sm.abort, 1);
-            if (a.status && tid == 0) atomicOr(a.status, SV_NOTE_TIMEOUT);
+            if (tid == 0) report_timeout(a);
             break;
         }
         const StageDesc d = sm.desc[st];
@@ -541,7 +550,7 @@ __device__ void consumers(const VerifyArgs &a, StreamSmem &sm, const uint4 *ring
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) {
             vstore(sm.abort, 1);
-            if (a.status && lane == 0) atomicOr(a.status, SV_NOTE_TIMEOUT);
+            if (lane == 0) report_timeout(a);
             break;
         }
     }
@@ -569,7 +578,7 @@ __device__ void publisher(const VerifyArgs &a, StreamSmem &sm) {
         const uint32_t slot_i = iseq % kItemSlots, use = iseq / kItemSlots;
         if (!mbar_wait(&sm.ifull[slot_i], use & 1u, kWaitLimitNs) || vload(sm.abort)) {
             vstore(sm.abort, 1);
-            if (a.status && lane == 0) atomicOr(a.status, SV_NOTE_TIMEOUT);
+            if (lane == 0) report_timeout(a);
             break;
         }
         const ItemMeta im = sm.imeta[slot_i];
@@ -648,6 +657,9 @@ __global__ void __launch_bounds__(kBlock, 3) stream_kernel(VerifyArgs a) {
     }
     __syncthreads();
     griddep_wait();
+    // The draw kernel may launch at once: its CTAs take SMs as this grid's
+    // CTAs leave, and each waits for its own row to settle.
+    griddep_launch_dependents();
     const int total = __ldcg(&a.ctr[1]);
     if (tid >= kConsumers + 32) {
         publisher<ESIZE>(a, sm);
@@ -658,18 +670,19 @@ __global__ void __launch_bounds__(kBlock, 3) stream_kernel(VerifyArgs a) {
         return;
     }
     consumers<ESIZE>(a, sm, ring);
-    // This CTA has no work left: the accept kernel may start launching.
-    griddep_launch_dependents();
 }
 
 // ---------------------------------------------------------------------------
-// 3. Draw kernel: one CTA per (row, chunk).  Accept test from the partials,
-//    then the final token by inverse CDF over chunks, then within a chunk.
+// 3. Draw kernel helpers: the final token by inverse CDF over chunks, then
+//    within a chunk (p-mass draws) or by sub-ranges (residual draws).
 // ---------------------------------------------------------------------------
 constexpr int kDrawThreads = 256;
 constexpr int kDrawWarps = kDrawThreads / 32;
 
+constexpr int kTblSmem = 1024;   // sub-range entries the last residual CTA stages in shared memory
+
 struct DrawSmem {
+    float tbl[kTblSmem];
     float m[kMaxSlots];
     float s[kMaxSlots];
     int arg[kMaxSlots];
@@ -683,6 +696,7 @@ struct DrawSmem {
     int lastpos;
     int ysel;
     int last;
+    int note;
 };
 
 enum DrawMode { kDrawP = 0, kDrawResidual = 1, kDrawOneHot = 2 };
@@ -1141,6 +1155,12 @@ __device__ void residual_subranges(const DrawCtx &c, int ch, int part, int U, fl
 // Sum of n table entries by one warp: rounds of 32 entries in order, a
 // fixed tree inside each round.  table_find walks the entries in the same
 // rounds, so a target below this total always finds its entry.
+template <bool SMEM>
+__device__ __forceinline__ float tbl_ld(const float *tb, int s) {
+    return SMEM ? tb[s] : __ldcg(tb + s);
+}
+
+template <bool SMEM>
 __device__ float table_total(const float *tb, int n) {
     constexpr int kRounds = 8;
     const int lane = threadIdx.x & 31;
@@ -1150,7 +1170,7 @@ __device__ float table_total(const float *tb, int n) {
 #pragma unroll
         for (int q = 0; q < kRounds; ++q) {
             const int s = base + q * 32 + lane;
-            v[q] = s < n ? __ldcg(tb + s) : 0.f;
+            v[q] = s < n ? tbl_ld<SMEM>(tb, s) : 0.f;
         }
 #pragma unroll
         for (int q = 0; q < kRounds; ++q) {
@@ -1167,6 +1187,7 @@ __device__ float table_total(const float *tb, int n) {
 // *d_out is t minus the sum before it.  If rounding leaves t at or past the
 // end, the last entry with weight is returned with *fb set and an infinite
 // target.
+template <bool SMEM>
 __device__ int table_find(const float *tb, int n, float t, float *d_out, bool *fb) {
     constexpr int kRounds = 8;
     const int lane = threadIdx.x & 31;
@@ -1177,7 +1198,7 @@ __device__ int table_find(const float *tb, int n, float t, float *d_out, bool *f
 #pragma unroll
         for (int q = 0; q < kRounds; ++q) {
             const int s = base + q * 32 + lane;
-            v[q] = s < n ? __ldcg(tb + s) : 0.f;
+            v[q] = s < n ? tbl_ld<SMEM>(tb, s) : 0.f;
         }
 #pragma unroll
         for (int q = 0; q < kRounds; ++q) {
@@ -1275,62 +1296,113 @@ __device__ int locate_in_subrange(const DrawCtx &c, float d, bool *fb) {
     return y;
 }
 
-// Per-row result of the accept test and the set-up of the final draw.
-struct __align__(16) DrawRecord {
-    int j;        // first rejected position, or L
-    int mode;     // kDrawDone (outputs written), kDrawP, kDrawResidual, kDrawOneHot
-    int csel;     // selected chunk (p-mass modes), -1 if none
-    int xj;       // rejected draft token (one-hot mode)
-    float d;      // target inside the selected chunk (p-mass modes)
-    float u;      // resample uniform
-    float k;      // log2(e) / T
-    float mt, ct, md, cd;
-    int note;     // status note bits to raise
-};
-constexpr int kDrawDone = -1;
+// Wait (bounded, with back-off) until row b is settled, and return its j:
+// positions 0..j-1 accepted (their bits set) and position j rejected
+// (row_j == j), or all L positions accepted and the bonus position's
+// partials complete.  A position is accepted or rejected, never both, and
+// bits and marker only move one way, so the two reads need no order.  The
+// acquire of position j's completion count makes its partials visible.
+// -1 if the wait ran out or a stream wait did.
+__device__ int wait_row_settled(const VerifyArgs &a, int b, int L, bool draft) {
+    const uint64_t t0 = global_ns();
+    uint32_t backoff = 32;
+    while (true) {
+        const unsigned long long M = ld_relaxed(&a.dec[b]);
+        const int j = min(ld_relaxed(&a.row_j[b]), L);
+        const unsigned long long want = j >= 64 ? ~0ull : ((1ull << j) - 1ull);
+        if ((M & want) == want) {
+            const int need = a.C * ((draft && j < L) ? 2 : 1);
+            if (ld_acquire(&a.pcnt[static_cast<long long>(b) * (a.K + 1) + j]) >= need) return j;
+        }
+        if (ld_relaxed(&a.ctr[2]) != 0 || global_ns() - t0 > kWaitLimitNs) return -1;
+        __nanosleep(backoff);
+        if (backoff < 1024) backoff <<= 1;
+    }
+}
 
 // ---------------------------------------------------------------------------
-// 3. Accept kernel: one CTA per row.  Merges the partials into the
-//    normalisers, runs the accept test with Philox uniforms, writes the
-//    outputs of greedy rows, and records the final draw of sampled rows
-//    (for p-mass draws the chunk is already chosen here).
+// 3. Draw kernel: one CTA per (row, chunk, part), rows fastest.  It
+//    launches while the stream kernel runs; a CTA starts once its row is
+//    settled (positions 0..j-1 accepted, j rejected, or all accepted and the
+//    bonus position complete) and merges the normalisers of position j from
+//    the stream partials: the same values, in the same order, in every CTA
+//    of the row.  Greedy rows: the row's lead CTA writes the argmax.  p-mass
+//    draws (the bonus position, or p_j without x_j for a greedy drafter):
+//    the lead CTA picks the chunk from the partials' masses and locates the
+//    token inside it.  Residual draws: every chunk CTA sums max(0, p_j -
+//    q_j) over its chunk by 64-unit sub-ranges; the last one (atomic count,
+//    no waiting) stages the row's sub-range table, forms the chunk totals in
+//    the order its scan walks them, and picks the chunk, the sub-range and
+//    the token.  Only position j of a rejecting row is read a second time.
 // ---------------------------------------------------------------------------
 template <int ESIZE>
-__global__ void __launch_bounds__(kDrawThreads) accept_kernel(VerifyArgs a) {
+__global__ void __launch_bounds__(kDrawThreads, 3) draw_kernel(VerifyArgs a) {
     __shared__ DrawSmem ds;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    griddep_wait();
-    griddep_launch_dependents();   // resample CTAs wait for this grid anyway
-    const int b = blockIdx.x;
-    const int K = a.K, S = a.S, C = a.C;
-    DrawRecord *rec = a.rec + b;
-    const int L = __ldg(&a.leff[b]);
-    if (L < 0) {                   // invalid row, already marked
-        if (tid == 0) rec->mode = kDrawDone;
-        return;
-    }
+    // This grid launches while the stream kernel still runs (its CTAs take
+    // SMs as the stream kernel's leave), and each CTA waits for its own row
+    // instead of the whole stream.  The last CTA waits for the stream grid,
+    // so that this grid never completes before it.  The prologue's writes
+    // are visible: every stream CTA passed its own wait for the prologue
+    // before letting this grid launch.
+    if (blockIdx.x == gridDim.x - 1) griddep_wait();
+    const int K = a.K, C = a.C;
+    const int b = static_cast<int>(blockIdx.x % static_cast<unsigned>(a.B));
+    const int cp = static_cast<int>(blockIdx.x / static_cast<unsigned>(a.B));
+    const int chunk = cp / kResidParts, part = cp - chunk * kResidParts;
+    const int L = __ldcg(&a.leff[b]);
     const float T = __ldg(&a.temp[b]);
+    if (L < 0) return;   // invalid row: the prologue wrote its outputs
     const bool greedy = !(T > 0.f);
     const bool has_draft = (a.zd != nullptr) && !greedy;
     const float k = greedy ? 0.f : kLog2e / T;
     const uint64_t row = static_cast<uint64_t>(a.row_base) + static_cast<uint64_t>(b);
-    // The stream kernel decided every position up to the first rejection.
-    const int j = min(__ldg(&a.row_j[b]), L);
-    // Normalisers of the positions that were read in full: target 0..j and
-    // draft 0..min(j, L-1); warp w takes slots w, w+8, ...
-    const int ntgt = j + 1;
-    const int nslots = ntgt + (has_draft ? min(j + 1, L) : 0);
-    for (int q = warp; q < nslots; q += kDrawWarps) {
-        const int slot = q < ntgt ? q : (K + 1 + (q - ntgt));
+    // The row's lead CTA (spread over the grid by row) takes greedy rows and
+    // p-mass draws alone; only a row with a draft can need the others.
+    const bool lead = cp == b % (C * kResidParts);
+    if (!lead && !has_draft) return;
+    if (tid == 0) {
+        const int jw = wait_row_settled(a, b, L, has_draft);
+        if (jw < 0 && a.status) atomicOr(a.status, SV_NOTE_TIMEOUT);
+        // The normaliser output reads positions 0..j-1 as well: acquire
+        // their completion counts (complete, since they were accepted).
+        if (lead && a.dbg != nullptr)
+            for (int i = 0; i < jw; ++i) (void)ld_acquire(&a.pcnt[static_cast<long long>(b) * (K + 1) + i]);
+        ds.j = jw;
+    }
+    __syncthreads();
+    const int j = ds.j;   // first rejection, or L
+    if (j < 0) return;    // a wait ran out: outputs undefined, status raised
+    const bool resid = (j < L) && has_draft;
+    if (!resid && !lead) return;
+
+    // Normalisers of position j (target; draft too for a residual draw).
+    // The row's lead CTA, when normalisers are requested, takes every
+    // position that was read in full: target 0..j, draft 0..min(j, L-1).
+    // Warp w takes slots w, w + 8, ...
+    const bool all = lead && a.dbg != nullptr;
+    const int ntgt = all ? j + 1 : 1;
+    const int ndft = !has_draft ? 0 : (all ? min(j + 1, L) : (resid ? 1 : 0));
+    const int first = all ? 0 : j;
+    for (int q = warp; q < ntgt + ndft; q += kDrawWarps) {
+        const int slot = q < ntgt ? first + q : K + 1 + first + (q - ntgt);
+        const long long pb = (static_cast<long long>(b) * a.S + slot) * C;
         float m = kNegInf, sm = 0.f;
         int idx = INT_MAX;
-        for (int cc = lane; cc < C; cc += 32) {
-            const float4 p = __ldcg(&a.part[(static_cast<long long>(b) * S + slot) * C + cc]);
-            if (greedy) {
-                const int i2 = __float_as_int(p.z);
-                if (p.x > m || (p.x == m && i2 < idx)) { m = p.x; idx = i2; }
-            } else {
-                lse_merge(m, sm, p.x, p.y, k);
+        float4 pv[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {   // C <= kMaxChunks = 64: two chunks per lane
+            const int cc = lane + 32 * h;
+            pv[h] = make_float4(kNegInf, 0.f, 0.f, 0.f);
+            if (cc < C) {
+                const float4 p = __ldcg(&a.part[pb + cc]);
+                pv[h] = p;
+                if (greedy) {
+                    const int i2 = __float_as_int(p.z);
+                    if (p.x > m || (p.x == m && i2 < idx)) { m = p.x; idx = i2; }
+                } else {
+                    lse_merge(m, sm, p.x, p.y, k);
+                }
             }
         }
 #pragma unroll
@@ -1344,14 +1416,23 @@ __global__ void __launch_bounds__(kDrawThreads) accept_kernel(VerifyArgs a) {
                 lse_merge(m, sm, m2, s2, k);
             }
         }
+        if (slot == j && !greedy && !resid) {
+            // p-mass draws: the mass of p_j per chunk, in units of
+            // 2^((z - m_j) k), straight from the partials.
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int cc = lane + 32 * h;
+                if (cc < C) ds.cm[cc] = (pv[h].x != kNegInf) ? pv[h].y * ex2((pv[h].x - m) * k) : 0.f;
+            }
+        }
         if (lane == 0) {
             if (idx == INT_MAX) idx = 0;   // every logit -inf: documented as invalid input
             ds.m[slot] = m;
             ds.s[slot] = greedy ? 1.f : sm;
             ds.arg[slot] = idx;
-            if (a.dbg) {
-                a.dbg[(static_cast<long long>(b) * S + slot) * 2 + 0] = m;
-                a.dbg[(static_cast<long long>(b) * S + slot) * 2 + 1] = greedy ? 1.f : sm;
+            if (all) {
+                a.dbg[(static_cast<long long>(b) * a.S + slot) * 2 + 0] = m;
+                a.dbg[(static_cast<long long>(b) * a.S + slot) * 2 + 1] = greedy ? 1.f : sm;
             }
         }
     }
@@ -1365,107 +1446,60 @@ __global__ void __launch_bounds__(kDrawThreads) accept_kernel(VerifyArgs a) {
             else if (t == j) v = y;
             a.out_tokens[static_cast<long long>(b) * (K + 1) + t] = v;
         }
-        if (tid == 0) { a.out_accept[b] = j; rec->mode = kDrawDone; }
+        if (tid == 0) a.out_accept[b] = j;
         return;
     }
 
-    // Sampled row: set up the final draw at position j.
-    const bool resid = (j < L) && has_draft;
+    // Sampled row: the final draw at position j.
     const float mt = ds.m[j];
     const float u = uniform24(a.seed, row, static_cast<uint32_t>(j), 1u);
     const int xj = (j < L) ? a.tokens[static_cast<long long>(b) * K + j] : -1;
     int mode = (j == L) ? kDrawP : (resid ? kDrawResidual : kDrawOneHot);
     int note = 0;
+    int csel = -1;
+    float d = 0.f;
     if (!resid) {
-        // p_j (bonus) or p_j without x_j (greedy drafter): chunk masses come
-        // straight from the stream partials.
-        chunk_masses(a, b, j, mt, k, ds.cm);
-        __syncthreads();
-        if (tid == 0 && mode == kDrawOneHot) {
-            const VecGeom g = vec_geom<ESIZE>(vec_ptr<ESIZE>(a, b, j), a.V);
-            const int cx = chunk_of_element<ESIZE>(g, xj, a.U, C);
-            const float wx = ex2((ld_elem<ESIZE>(g.base, xj) - mt) * k);
-            ds.cm[cx] = fmaxf(ds.cm[cx] - wx, 0.f);
-        }
-        __syncthreads();
+        // p_j (bonus) or p_j without x_j (greedy drafter): pick the chunk
+        // from the partials' masses, then locate the token inside it.
         if (tid == 0) {
-            float d = 0.f;
-            int cs = select_chunk(ds.cm, C, u, &d);
+            if (mode == kDrawOneHot) {
+                const VecGeom g = vec_geom<ESIZE>(vec_ptr<ESIZE>(a, b, j), a.V);
+                const int cx = chunk_of_element<ESIZE>(g, xj, a.U, C);
+                const float wx = ex2((ld_elem<ESIZE>(g.base, xj) - mt) * k);
+                ds.cm[cx] = fmaxf(ds.cm[cx] - wx, 0.f);
+            }
+            float dd = 0.f;
+            int cs = select_chunk(ds.cm, C, u, &dd);
             if (cs < 0) {
                 // p_j one-hot at the rejected x_j (rounding): draw from p_j.
                 mode = kDrawP;
                 note = SV_NOTE_ZERO_RESIDUAL;
                 chunk_masses_serial(a, b, j, mt, k, ds.cm);
-                cs = select_chunk(ds.cm, C, u, &d);
+                cs = select_chunk(ds.cm, C, u, &dd);
             }
             ds.gsel = cs;
-            ds.dsel = d;
+            ds.dsel = dd;
             ds.lastpos = mode;
+            ds.note = note;
         }
         __syncthreads();
+        csel = ds.gsel;
+        d = ds.dsel;
+        mode = ds.lastpos;
+        note = ds.note;
     }
-    if (tid == 0) {
-        DrawRecord r;
-        r.j = j;
-        r.mode = resid ? kDrawResidual : ds.lastpos;
-        r.csel = resid ? -1 : ds.gsel;
-        r.xj = xj;
-        r.d = resid ? 0.f : ds.dsel;
-        r.u = u;
-        r.k = k;
-        r.mt = mt;
-        r.ct = resid ? log2f(ds.s[j]) : 0.f;
-        r.md = resid ? ds.m[K + 1 + j] : 0.f;
-        r.cd = resid ? log2f(ds.s[K + 1 + j]) : 0.f;
-        r.note = note;
-        *rec = r;
-        // Resample work: every chunk of a residual draw, the selected chunk
-        // of a p-mass draw.
-        if (resid) {
-            const int base = atomicAdd(&a.ctr[2], C * kResidParts);
-            for (int q = 0; q < C * kResidParts; ++q) a.work[base + q] = b * C * kResidParts + q;
-        } else {
-            a.work[atomicAdd(&a.ctr[2], 1)] = (b * C + (ds.gsel < 0 ? 0 : ds.gsel)) * kResidParts;
-        }
-    }
-}
-
-// ---------------------------------------------------------------------------
-// 4. Resample kernel: one CTA per (row, chunk).  p-mass draws: the CTA of
-//    the selected chunk locates the token inside it.  Residual draws: every
-//    chunk CTA sums max(0, p_j - q_j) over its chunk by segments; the last
-//    one (atomic counter, no waiting) selects the chunk and the segment from
-//    those sums and locates the token.
-// ---------------------------------------------------------------------------
-template <int ESIZE>
-__global__ void __launch_bounds__(kDrawThreads, 3) resample_kernel(VerifyArgs a) {
-    __shared__ DrawSmem ds;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    griddep_wait();
-    // CTA w takes work entry w; the entries of every row with a draw were
-    // appended by the accept kernel, so all the work sits in the first CTAs.
-    if (static_cast<int>(blockIdx.x) >= __ldcg(&a.ctr[2])) return;
-    const int entry = __ldcg(&a.work[blockIdx.x]);
-    const int part = entry % kResidParts;
-    const int b = entry / kResidParts / a.C;
-    const int chunk = entry / kResidParts - b * a.C;
-    const int K = a.K, C = a.C;
-    const DrawRecord r = a.rec[b];   // written by the previous launch
-    if (r.mode == kDrawDone) return;
-    const bool resid = r.mode == kDrawResidual;
-    const int j = r.j;
 
     DrawCtx c;
-    c.k = r.k;
-    c.mode = r.mode;
+    c.k = k;
+    c.mode = mode;
     c.gt = vec_geom<ESIZE>(vec_ptr<ESIZE>(a, b, j), a.V);
-    c.mt = r.mt;
-    c.ct = r.ct;
-    c.xj = r.xj;
+    c.mt = mt;
+    c.ct = resid ? log2f(ds.s[j]) : 0.f;
+    c.xj = xj;
     if (resid) {
         c.gd = vec_geom<ESIZE>(vec_ptr<ESIZE>(a, b, K + 1 + j), a.V);
-        c.md = r.md;
-        c.cd = r.cd;
+        c.md = ds.m[K + 1 + j];
+        c.cd = log2f(ds.s[K + 1 + j]);
     } else {
         c.gd = c.gt; c.md = 0.f; c.cd = 0.f;
     }
@@ -1476,9 +1510,6 @@ __global__ void __launch_bounds__(kDrawThreads, 3) resample_kernel(VerifyArgs a)
         c.has_head = (cc == 0);
         c.has_tail = (cc == C - 1);
     };
-    int note = r.note;
-    int csel = r.csel;
-    float d = r.d;
     int y = -1;
     bool fb = false;
     if (resid) {
@@ -1487,54 +1518,49 @@ __global__ void __launch_bounds__(kDrawThreads, 3) resample_kernel(VerifyArgs a)
         // row's table and the token inside it.
         set_chunk(chunk);
         float *tb = a.rtbl + static_cast<long long>(b) * a.nsub;
-        float *ct = a.ctot + static_cast<long long>(b) * C;
         residual_subranges<ESIZE>(c, chunk, part, a.U, tb);
         __syncthreads();
-        if (kResidParts == 1 && warp == 0) {
-            // This chunk's total, formed as the last CTA's scan will walk it.
-            int s0, s1;
-            chunk_subranges(c.gt, chunk, a.U, &s0, &s1);
-            const float tot = table_total(tb + s0, s1 - s0);
-            if (lane == 0) ct[chunk] = tot;
-        }
         if (tid == 0) {
-            __threadfence();
-            const int done = atomicAdd(&a.rcnt[b], 1) + 1;
-            __threadfence();
+            // Release: this CTA's table entries (ordered before this thread
+            // by the barrier) are visible before the count; acquire: the
+            // last CTA sees every entry counted before it.
+            const int done = atom_add_acq_rel(&a.rcnt[b], 1) + 1;
             ds.last = (done == C * kResidParts);
         }
         __syncthreads();
         if (!ds.last) return;
-        if (kResidParts > 1) {
-            // A chunk's sub-ranges came from several CTAs: the last CTA forms
-            // every chunk total (warp w: chunks w, w + 8, ...), in the order
-            // its scan will walk them.
-            for (int cc = warp; cc < C; cc += kDrawWarps) {
-                int s0, s1;
-                chunk_subranges(c.gt, cc, a.U, &s0, &s1);
-                const float tot = table_total(tb + s0, s1 - s0);
-                if (lane == 0) ct[cc] = tot;
-            }
+        // The row's whole table in one parallel round trip (shared memory
+        // when it fits), then every step of the pick reads it from there.
+        const int nsub = max(1, (c.gt.n16 + kSubUnits - 1) / kSubUnits);
+        const bool staged = nsub <= kTblSmem;
+        if (staged) {
+            for (int q = tid; q < nsub; q += kDrawThreads) ds.tbl[q] = __ldcg(tb + q);
             __syncthreads();
         }
         if (warp == 0) {
-            // Chunk totals in order, then the sub-ranges of the chosen chunk.
+            // Chunk totals, each formed as the scan below walks it, summed in
+            // chunk order; then the sub-ranges of the chosen chunk.
             bool zero = false, fbw = false;
-            const int nsub = max(1, (c.gt.n16 + kSubUnits - 1) / kSubUnits);
-            const float w0 = lane < C ? __ldcg(ct + lane) : 0.f;
-            const float w1 = lane + 32 < C ? __ldcg(ct + lane + 32) : 0.f;
             float R = 0.f;
-            for (int q = 0; q < C; ++q) R += __shfl_sync(0xffffffffu, q < 32 ? w0 : w1, q & 31);
+            for (int q = 0; q < C; ++q) {
+                int s0, s1;
+                chunk_subranges(c.gt, q, a.U, &s0, &s1);
+                const float tot = staged ? table_total<true>(ds.tbl + s0, s1 - s0)
+                                         : table_total<false>(tb + s0, s1 - s0);
+                if (lane == 0) ds.cm[q] = tot;
+                R += tot;
+            }
+            __syncwarp();
             int sel = -1;
             float dsel = 0.f;
             if (!(R > 0.f)) {
                 zero = true;
             } else {
-                const float t = r.u * R;
+                const float t = u * R;
                 float cum = 0.f, tc = 0.f;
                 int cs = -1, clast = 0;
                 for (int q = 0; q < C; ++q) {
-                    const float w = __shfl_sync(0xffffffffu, q < 32 ? w0 : w1, q & 31);
+                    const float w = ds.cm[q];
                     if (w > 0.f) clast = q;
                     if (cs < 0 && cum + w > t) { cs = q; tc = t - cum; }
                     if (cs < 0) cum += w;
@@ -1542,7 +1568,8 @@ __global__ void __launch_bounds__(kDrawThreads, 3) resample_kernel(VerifyArgs a)
                 if (cs < 0) { cs = clast; tc = __int_as_float(0x7f800000); fbw = true; }
                 int s0, s1;
                 chunk_subranges(c.gt, cs, a.U, &s0, &s1);
-                sel = s0 + table_find(tb + s0, s1 - s0, tc, &dsel, &fbw);
+                sel = s0 + (staged ? table_find<true>(ds.tbl + s0, s1 - s0, tc, &dsel, &fbw)
+                                   : table_find<false>(tb + s0, s1 - s0, tc, &dsel, &fbw));
             }
             int yw = -1;
             if (!zero && sel >= 0) {
@@ -1569,8 +1596,8 @@ __global__ void __launch_bounds__(kDrawThreads, 3) resample_kernel(VerifyArgs a)
             if (tid == 0) {
                 float dd = 0.f;
                 note |= SV_NOTE_ZERO_RESIDUAL;
-                chunk_masses_serial(a, b, j, r.mt, r.k, ds.cm);
-                ds.gsel = select_chunk(ds.cm, C, r.u, &dd);
+                chunk_masses_serial(a, b, j, mt, k, ds.cm);
+                ds.gsel = select_chunk(ds.cm, C, u, &dd);
                 ds.dsel = dd;
             }
             __syncthreads();
@@ -1609,9 +1636,7 @@ template <int ESIZE> static const void *stream_kernel_ptr() {
 struct Plan {
     int C, U, S;
     int nsub;
-    size_t off_rcnt, off_leff, off_rowj, off_pcnt, off_lvloff, off_lvlrow, off_part, off_rtbl, off_ctot,
-        off_work,
-        off_rec, bytes;
+    size_t off_rcnt, off_leff, off_rowj, off_pcnt, off_dec, off_lvloff, off_lvlrow, off_part, off_rtbl, bytes;
 };
 
 static bool make_plan(int B, int K, int V, sv_dtype dtype, Plan *p) {
@@ -1636,15 +1661,13 @@ static bool make_plan(int B, int K, int V, sv_dtype dtype, Plan *p) {
     p->off_leff = off;   off = align16(off + iB);
     p->off_rowj = off;   off = align16(off + iB);
     p->off_pcnt = off;   off = align16(off + iB * (K + 1));
+    p->off_dec = off;    off = align16(off + sizeof(unsigned long long) * static_cast<size_t>(B));
     p->off_lvloff = off; off = align16(off + sizeof(int) * static_cast<size_t>(K + 2));
     p->off_lvlrow = off; off = align16(off + sizeof(int) * static_cast<size_t>(K + 1) * (B + 1));
     p->off_part = off;   off = align16(off + sizeof(float4) * static_cast<size_t>(items));
     p->nsub = static_cast<int>((n16 + kSubUnits - 1) / kSubUnits);
     if (p->nsub < 1) p->nsub = 1;
     p->off_rtbl = off;   off = align16(off + sizeof(float) * static_cast<size_t>(B) * p->nsub);
-    p->off_ctot = off;   off = align16(off + sizeof(float) * static_cast<size_t>(B) * C);
-    p->off_work = off;   off = align16(off + sizeof(int) * static_cast<size_t>(B) * C * kResidParts);
-    p->off_rec = off;    off = align16(off + sizeof(DrawRecord) * static_cast<size_t>(B));
     p->bytes = off;
     return true;
 }
@@ -1705,14 +1728,12 @@ static sv_status verify_impl(const void *zt, const void *zd, sv_dtype dtype, int
     a.leff = reinterpret_cast<int *>(w + p.off_leff);
     a.row_j = reinterpret_cast<int *>(w + p.off_rowj);
     a.pcnt = reinterpret_cast<int *>(w + p.off_pcnt);
+    a.dec = reinterpret_cast<unsigned long long *>(w + p.off_dec);
     a.lvl_off = reinterpret_cast<int *>(w + p.off_lvloff);
     a.lvl_row = reinterpret_cast<int *>(w + p.off_lvlrow);
     a.part = reinterpret_cast<float4 *>(w + p.off_part);
     a.rtbl = reinterpret_cast<float *>(w + p.off_rtbl);
-    a.ctot = reinterpret_cast<float *>(w + p.off_ctot);
     a.nsub = p.nsub;
-    a.work = reinterpret_cast<int *>(w + p.off_work);
-    a.rec = reinterpret_cast<DrawRecord *>(w + p.off_rec);
 
     const int grid = stream_grid(es, static_cast<long long>(B) * p.S * p.C);
     if (grid <= 0) return note_cuda(cudaGetLastError());
@@ -1729,15 +1750,8 @@ static sv_status verify_impl(const void *zt, const void *zd, sv_dtype dtype, int
     if (e != cudaSuccess) return note_cuda(e);
     profile_mark_end(st);
     const unsigned draw_grid = static_cast<unsigned>(B) * static_cast<unsigned>(p.C) * kResidParts;
-    if (es == 4) {
-        e = launch_pdl(accept_kernel<4>, dim3(B), dim3(kDrawThreads), 0, st, a);
-        if (e == cudaSuccess)
-            e = launch_pdl(resample_kernel<4>, dim3(draw_grid), dim3(kDrawThreads), 0, st, a);
-    } else {
-        e = launch_pdl(accept_kernel<2>, dim3(B), dim3(kDrawThreads), 0, st, a);
-        if (e == cudaSuccess)
-            e = launch_pdl(resample_kernel<2>, dim3(draw_grid), dim3(kDrawThreads), 0, st, a);
-    }
+    e = (es == 4) ? launch_pdl(draw_kernel<4>, dim3(draw_grid), dim3(kDrawThreads), 0, st, a)
+                  : launch_pdl(draw_kernel<2>, dim3(draw_grid), dim3(kDrawThreads), 0, st, a);
     if (e != cudaSuccess) return note_cuda(e);
     return note_cuda(cudaGetLastError());
 }
@@ -1776,7 +1790,7 @@ extern "C" sv_status sv_verify_debug(const void *target_logits, const void *draf
                            workspace_bytes, status, stats_out, stream);
 }
 
-extern "C" int sv_verify_launches(void) { return 4; }
+extern "C" int sv_verify_launches(void) { return 3; }
 
 // ---------------------------------------------------------------------------
 // Allocation-free variant: the scratch lives in a fixed device array that

@@ -32,7 +32,7 @@ def test_status_strings_and_version():
     assert sv.sv_status_string(4) == "SV_ERR_WORKSPACE"
     assert sv.sv_status_string(99) == "SV_UNKNOWN"
     assert sv.lib().sv_version() >= 1
-    assert sv.sv_verify_launches() == 4
+    assert sv.sv_verify_launches() == 3
 
 
 def test_workspace_bytes():
