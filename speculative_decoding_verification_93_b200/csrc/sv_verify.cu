@@ -73,6 +73,7 @@ struct VerifyArgs {
     const char *zt;            // [B, K+1, V]
     const char *zd;            // [B, K, V] or nullptr (greedy drafter)
     int B, K, V, S, C, U;      // S = 2K+1 slots per row, C chunks per vector, U units per chunk
+    int P;                     // draw CTAs per chunk of a residual draw (1 or 2)
     const int32_t *tokens;     // [B, K]
     const int32_t *lengths;    // [B]
     const float *temp;         // [B]
@@ -1065,7 +1066,8 @@ __device__ __forceinline__ void chunk_masses(const VerifyArgs &a, int b, int j, 
 // ---------------------------------------------------------------------------
 constexpr int kSubUnits = 64;   // units per sub-range; chunk sizes are multiples of it
 constexpr int kRunUnits = 3;    // local units per lane in a located sub-range (66 / 32)
-constexpr int kResidParts = 1;  // resample CTAs per chunk of a residual draw
+constexpr int kResidLaneUnits = 8;   // units per lane per block of the residual sums (even)
+static_assert(kResidLaneUnits % 2 == 0, "a sub-range is two units per lane");
 
 // Draw weight of `count` (< one unit) elements from element `first`,
 // loaded directly (vector head or tail).
@@ -1085,39 +1087,43 @@ __device__ __forceinline__ float partial_sum(const DrawCtx &c, int first, int co
 }
 
 // Residual weight of every sub-range of part `part` of chunk `ch` into tbl.
-// Warp w takes the 256-unit blocks w, w + 8, ... of the part with eight units per lane in
-// flight; unit base + lane + 32 q lies in sub-range base / 64 + q / 2.  The
-// head joins sub-range 0 and the tail the last one.  Each sum has a fixed
-// order.
+// Warp w takes the blocks w, w + 8, ... of 32 NQ units (NQ units per lane
+// in flight, loaded without L1 allocation: the pass touches them once) of
+// the part; unit base + lane + 32 q lies in sub-range base / 64 + q / 2.
+// The head joins sub-range 0 and the tail the last one.  Each sum has a
+// fixed order.
 template <int ESIZE>
-__device__ void residual_subranges(const DrawCtx &c, int ch, int part, int U, float *tbl) {
+__device__ void residual_subranges(const DrawCtx &c, int ch, int part, int P, int U, float *tbl) {
     constexpr int kPer = 16 / ESIZE;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int PU = (U / kResidParts + kSubUnits - 1) / kSubUnits * kSubUnits;   // units per part
+    const int PU = (U / P + kSubUnits - 1) / kSubUnits * kSubUnits;   // units per part
     const int u0 = ch * U + part * PU;
     const int u1 = max(u0, min(min(u0 + PU, (ch + 1) * U), c.gt.n16));
     const int slast = c.gt.n16 > 0 ? (c.gt.n16 - 1) / kSubUnits : 0;
     const uint32_t pw = neg_inf_word<ESIZE>();
     const uint4 pad = make_uint4(pw, pw, pw, pw);
-    int nblk = (u1 - u0 + 255) / 256;
+    constexpr int NQ = kResidLaneUnits, NS = NQ / 2;   // units per lane, sub-ranges per block
+    int nblk = (u1 - u0 + 32 * NQ - 1) / (32 * NQ);
     if (c.gt.n16 == 0 && ch == 0 && part == 0) nblk = 1;   // head and tail only
     for (int blk = warp; blk < nblk; blk += kDrawWarps) {
-        const int base = u0 + blk * 256;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        if (c.aligned) {
-            uint4 t[8], d[8];
+        const int base = u0 + blk * 32 * NQ;
+        float acc[NS];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
+        for (int r = 0; r < NS; ++r) acc[r] = 0.f;
+        if (c.aligned) {
+            uint4 t[NQ], d[NQ];
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
                 const int u = base + lane + 32 * q;
                 const long long off = static_cast<long long>(u) * 16;
-                t[q] = u < u1 ? ld_reuse(c.gt.body + off) : pad;
-                d[q] = u < u1 ? ld_reuse(c.gd.body + off) : pad;
+                t[q] = u < u1 ? ld_stream(c.gt.body + off) : pad;
+                d[q] = u < u1 ? ld_stream(c.gd.body + off) : pad;
             }
 #pragma unroll
-            for (int q = 0; q < 8; ++q) acc[q >> 1] += body_sum<ESIZE, kDrawResidual>(c, t[q], d[q]);
+            for (int q = 0; q < NQ; ++q) acc[q >> 1] += body_sum<ESIZE, kDrawResidual>(c, t[q], d[q]);
         } else {
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
+            for (int q = 0; q < NQ; ++q) {
                 const int u = base + lane + 32 * q;
                 if (u < u1) {
                     UnitData ud;
@@ -1134,17 +1140,17 @@ __device__ void residual_subranges(const DrawCtx &c, int ch, int part, int U, fl
         const int s0 = base / kSubUnits;
         if (lane == 0) {
             if (s0 == 0 && c.gt.head > 0) acc[0] += partial_sum<ESIZE, kDrawResidual>(c, 0, c.gt.head);
-            if (c.gt.tail > 0 && slast >= s0 && slast < s0 + 4)
+            if (c.gt.tail > 0 && slast >= s0 && slast < s0 + NS)
                 acc[slast - s0] += partial_sum<ESIZE, kDrawResidual>(
                     c, c.gt.head + c.gt.n16 * kPer, c.gt.tail);
         }
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+        for (int r = 0; r < NS; ++r)
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], o);
         if (lane == 0) {
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
+            for (int r = 0; r < NS; ++r) {
                 const int s = s0 + r;
                 if (s * kSubUnits < u1 || (c.gt.n16 == 0 && s == 0)) tbl[s] = acc[r];
             }
@@ -1349,7 +1355,7 @@ __global__ void __launch_bounds__(kDrawThreads, 3) draw_kernel(VerifyArgs a) {
     const int K = a.K, C = a.C;
     const int b = static_cast<int>(blockIdx.x % static_cast<unsigned>(a.B));
     const int cp = static_cast<int>(blockIdx.x / static_cast<unsigned>(a.B));
-    const int chunk = cp / kResidParts, part = cp - chunk * kResidParts;
+    const int chunk = cp / a.P, part = cp - chunk * a.P;
     const int L = __ldcg(&a.leff[b]);
     const float T = __ldg(&a.temp[b]);
     if (L < 0) return;   // invalid row: the prologue wrote its outputs
@@ -1359,7 +1365,7 @@ __global__ void __launch_bounds__(kDrawThreads, 3) draw_kernel(VerifyArgs a) {
     const uint64_t row = static_cast<uint64_t>(a.row_base) + static_cast<uint64_t>(b);
     // The row's lead CTA (spread over the grid by row) takes greedy rows and
     // p-mass draws alone; only a row with a draft can need the others.
-    const bool lead = cp == b % (C * kResidParts);
+    const bool lead = cp == b % (C * a.P);
     if (!lead && !has_draft) return;
     if (tid == 0) {
         const int jw = wait_row_settled(a, b, L, has_draft);
@@ -1518,14 +1524,14 @@ __global__ void __launch_bounds__(kDrawThreads, 3) draw_kernel(VerifyArgs a) {
         // row's table and the token inside it.
         set_chunk(chunk);
         float *tb = a.rtbl + static_cast<long long>(b) * a.nsub;
-        residual_subranges<ESIZE>(c, chunk, part, a.U, tb);
+        residual_subranges<ESIZE>(c, chunk, part, a.P, a.U, tb);
         __syncthreads();
         if (tid == 0) {
             // Release: this CTA's table entries (ordered before this thread
             // by the barrier) are visible before the count; acquire: the
             // last CTA sees every entry counted before it.
             const int done = atom_add_acq_rel(&a.rcnt[b], 1) + 1;
-            ds.last = (done == C * kResidParts);
+            ds.last = (done == C * a.P);
         }
         __syncthreads();
         if (!ds.last) return;
@@ -1737,6 +1743,12 @@ static sv_status verify_impl(const void *zt, const void *zd, sv_dtype dtype, int
 
     const int grid = stream_grid(es, static_cast<long long>(B) * p.S * p.C);
     if (grid <= 0) return note_cuda(cudaGetLastError());
+    // Residual chunks are split over two draw CTAs when the rows' chunk CTAs
+    // would fill at most two rounds of the SMs' slots (three per SM, like
+    // the stream kernel's); with more rows one CTA per chunk keeps the
+    // per-row count round trips fewer.
+    const int slots = stream_grid(es, LLONG_MAX);
+    a.P = (static_cast<long long>(B) * p.C <= 2LL * slots) ? 2 : 1;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // Every launch below may overlap the tail of the one before it
     // (programmatic dependent launch); each kernel waits for its
@@ -1749,7 +1761,7 @@ static sv_status verify_impl(const void *zt, const void *zd, sv_dtype dtype, int
                   : launch_pdl(stream_kernel<2>, dim3(grid), dim3(kBlock), kRingBytes, st, a);
     if (e != cudaSuccess) return note_cuda(e);
     profile_mark_end(st);
-    const unsigned draw_grid = static_cast<unsigned>(B) * static_cast<unsigned>(p.C) * kResidParts;
+    const unsigned draw_grid = static_cast<unsigned>(B) * static_cast<unsigned>(p.C) * a.P;
     e = (es == 4) ? launch_pdl(draw_kernel<4>, dim3(draw_grid), dim3(kDrawThreads), 0, st, a)
                   : launch_pdl(draw_kernel<2>, dim3(draw_grid), dim3(kDrawThreads), 0, st, a);
     if (e != cudaSuccess) return note_cuda(e);
