@@ -1171,19 +1171,32 @@ __device__ float table_total(const float *tb, int n) {
     constexpr int kRounds = 8;
     const int lane = threadIdx.x & 31;
     float R = 0.f;
-    float v[kRounds];
-    for (int base = 0; base < n; base += 32 * kRounds) {
-#pragma unroll
-        for (int q = 0; q < kRounds; ++q) {
-            const int s = base + q * 32 + lane;
-            v[q] = s < n ? tbl_ld<SMEM>(tb, s) : 0.f;
-        }
-#pragma unroll
-        for (int q = 0; q < kRounds; ++q) {
-            float r = v[q];
+    if constexpr (SMEM) {
+        // The same rounds in the same order, one at a time: a staged table
+        // needs no loads in flight, and the loop keeps this once-per-row
+        // code small.
+#pragma unroll 1
+        for (int r0 = 0; r0 < n; r0 += 32) {
+            float r = r0 + lane < n ? tb[r0 + lane] : 0.f;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
             R += r;
+        }
+    } else {
+        float v[kRounds];
+        for (int base = 0; base < n; base += 32 * kRounds) {
+#pragma unroll
+            for (int q = 0; q < kRounds; ++q) {
+                const int s = base + q * 32 + lane;
+                v[q] = s < n ? tbl_ld<SMEM>(tb, s) : 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < kRounds; ++q) {
+                float r = v[q];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+                R += r;
+            }
         }
     }
     return R;
@@ -1199,33 +1212,42 @@ __device__ int table_find(const float *tb, int n, float t, float *d_out, bool *f
     const int lane = threadIdx.x & 31;
     int sel = -1, lastpos = -1;
     float dsel = 0.f, cum = 0.f;
-    float v[kRounds];
-    for (int base = 0; base < n && sel < 0; base += 32 * kRounds) {
+    auto round = [&](int r0, float v) {   // one round of 32 entries from r0
+        if (v > 0.f) lastpos = r0 + lane;
+        float incl = v;
 #pragma unroll
-        for (int q = 0; q < kRounds; ++q) {
-            const int s = base + q * 32 + lane;
-            v[q] = s < n ? tbl_ld<SMEM>(tb, s) : 0.f;
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
         }
+        const unsigned hit = __ballot_sync(0xffffffffu, v > 0.f && cum + incl > t);
+        if (hit) {
+            const int l = __ffs(hit) - 1;
+            sel = r0 + l;
+            dsel = t - (cum + __shfl_sync(0xffffffffu, incl - v, l));
+        } else {
+            float r = v;
 #pragma unroll
-        for (int q = 0; q < kRounds; ++q) {
-            if (sel >= 0) break;
-            if (v[q] > 0.f) lastpos = base + q * 32 + lane;
-            float incl = v[q];
+            for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+            cum += r;
+        }
+    };
+    if constexpr (SMEM) {
+        // Staged table: the rounds one at a time (same order), small code.
+#pragma unroll 1
+        for (int r0 = 0; r0 < n && sel < 0; r0 += 32) round(r0, r0 + lane < n ? tb[r0 + lane] : 0.f);
+    } else {
+        float v[kRounds];
+        for (int base = 0; base < n && sel < 0; base += 32 * kRounds) {
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
+            for (int q = 0; q < kRounds; ++q) {
+                const int s = base + q * 32 + lane;
+                v[q] = s < n ? tbl_ld<SMEM>(tb, s) : 0.f;
             }
-            const unsigned hit = __ballot_sync(0xffffffffu, v[q] > 0.f && cum + incl > t);
-            if (hit) {
-                const int l = __ffs(hit) - 1;
-                sel = base + q * 32 + l;
-                dsel = t - (cum + __shfl_sync(0xffffffffu, incl - v[q], l));
-            } else {
-                float r = v[q];
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
-                cum += r;
+            for (int q = 0; q < kRounds; ++q) {
+                if (sel >= 0) break;
+                round(base + q * 32, v[q]);
             }
         }
     }
@@ -1253,26 +1275,33 @@ __device__ __forceinline__ void chunk_subranges(const VecGeom &g, int ch, int U,
 // rounding leaves d at or past the total, the last element with positive
 // weight is returned and *fb is set; -1 if there is none.
 template <int ESIZE, int MODE>
-__device__ int locate_in_subrange(const DrawCtx &c, float d, bool *fb) {
+__device__ int locate_in_subrange(const DrawCtx &c, float d, bool *fb, float *wbuf) {
     constexpr int kPer = 16 / ESIZE;
+    static_assert(kRunUnits == 3, "three units per lane");
     const int lane = threadIdx.x & 31;
     const int NU = c.nbody + 2;
     const int l0 = min(lane * kRunUnits, NU);
     const int l1 = min(l0 + kRunUnits, NU);
-    UnitData ud[kRunUnits];
-#pragma unroll
-    for (int q = 0; q < kRunUnits; ++q)
-        ud[q] = (l0 + q < l1) ? load_unit<ESIZE, MODE>(c, l0 + q) : empty_unit();
+    // The three loads go out together; the weights are then formed by a loop
+    // over the units that is not unrolled.  This code runs once per row, as
+    // the last step of the draw, when its instructions are no longer cached:
+    // its size, not its arithmetic, sets how long it takes.
+    const UnitData v0 = (l0 < l1) ? load_unit<ESIZE, MODE>(c, l0) : empty_unit();
+    const UnitData v1 = (l0 + 1 < l1) ? load_unit<ESIZE, MODE>(c, l0 + 1) : empty_unit();
+    const UnitData v2 = (l0 + 2 < l1) ? load_unit<ESIZE, MODE>(c, l0 + 2) : empty_unit();
     float mine = 0.f;
     int lastpos = -1;
-#pragma unroll
-    for (int q = 0; q < kRunUnits; ++q)
+#pragma unroll 1
+    for (int q = 0; q < kRunUnits; ++q) {
+        const UnitData u = q == 0 ? v0 : (q == 1 ? v1 : v2);
 #pragma unroll
         for (int e = 0; e < kPer; ++e) {
-            const float w = elem_weight<ESIZE, MODE>(c, ud[q], e);
-            if (w > 0.f) lastpos = ud[q].first + e;
+            const float w = elem_weight<ESIZE, MODE>(c, u, e);
+            if (w > 0.f) lastpos = u.first + e;
             mine += w;
+            wbuf[(q * kPer + e) * 32 + lane] = w;   // for the second pass below
         }
+    }
     float incl = mine;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -1284,15 +1313,17 @@ __device__ int locate_in_subrange(const DrawCtx &c, float d, bool *fb) {
     int y = -1;
     const unsigned hit = __ballot_sync(0xffffffffu, incl > d);
     if (hit && lane == __ffs(hit) - 1) {
+        // The same weights, in the same order, from shared memory.
         float cum = excl;
-#pragma unroll
-        for (int q = 0; q < kRunUnits; ++q)
-#pragma unroll
-            for (int e = 0; e < kPer; ++e) {
-                const float w = elem_weight<ESIZE, MODE>(c, ud[q], e);
-                if (y < 0 && w > 0.f && cum + w > d) y = ud[q].first + e;
-                cum += w;
+#pragma unroll 1
+        for (int k = 0; k < kRunUnits * kPer; ++k) {
+            const float w = wbuf[k * 32 + lane];
+            if (y < 0 && w > 0.f && cum + w > d) {
+                const int q = k / kPer;
+                y = (q == 0 ? v0.first : (q == 1 ? v1.first : v2.first)) + (k - q * kPer);
             }
+            cum += w;
+        }
     }
     y = __reduce_max_sync(0xffffffffu, y);
     if (y < 0) {
@@ -1584,7 +1615,7 @@ __global__ void __launch_bounds__(kDrawThreads, 3) draw_kernel(VerifyArgs a) {
                 cs.nbody = max(0, min(kSubUnits, c.gt.n16 - cs.ubody0));
                 cs.has_head = (sel == 0) && c.gt.head > 0;
                 cs.has_tail = (sel == nsub - 1) && c.gt.tail > 0;
-                yw = locate_in_subrange<ESIZE, kDrawResidual>(cs, dsel, &fbw);
+                yw = locate_in_subrange<ESIZE, kDrawResidual>(cs, dsel, &fbw, ds.tbl);
             }
             if (lane == 0) {
                 ds.ysel = yw;
