@@ -123,6 +123,21 @@ def test_ragged_slices_match_oracle(V, dtype, K, B, nshards):
     assert total["tie_mismatches"] <= max(2, total["rows"] // 50)
 
 
+@pytest.mark.parametrize("B,V,dtype,nshards", [(1025, 1000, torch.bfloat16, 2),
+                                              (2100, 517, torch.float32, 3)])
+def test_many_rows(B, V, dtype, nshards):
+    """Thousands of rows (grids of tens of thousands of stats CTAs, most of
+    them for slots no row reads) against the oracle."""
+    b = _cuda(workloads.random_small(B, 3, V, dtype=dtype, seed=B + V, temps=(0.0, 0.6, 1.0, 2.5)))
+    g = vp_emulated(b.zt, b.zd, b.tokens, b.lengths, b.temperature, 11, nshards)
+    ln = b.lengths.cpu().numpy()
+    o = oracle_verify(b.zt, b.zd, b.tokens, ln, b.temperature, 11)
+    check_structure(g, b.tokens.cpu().numpy(), ln)
+    r = compare(g, o)
+    assert g["status"] & ~(sv.SV_NOTE_CDF_FALLBACK | sv.SV_NOTE_ZERO_RESIDUAL) == 0
+    assert r["tie_mismatches"] <= max(2, r["rows"] // 50)
+
+
 @pytest.mark.parametrize("V,dtype,nshards", [(1000, torch.float32, 3),
                                              (129280, torch.bfloat16, 8),
                                              (20011, torch.float32, 5)])
