@@ -5,7 +5,9 @@
 
 One step = one pass of the whole hot path over one batch: the schedule
 (prefix survival -> verify lengths) and the verification (softmax statistics,
-accept test, correction/bonus draw), through the library's C ABI.  The
+accept test, correction/bonus draw), through the library's C ABI
+(sv_schedule_verify: the schedule runs in the verification's first kernel;
+workloads with fixed lengths call sv_verify).  The
 default workload is the 256-row, 8-draft, 129280-token bf16 batch (per-row
 temperature from {0, 0.6, 1.0}, lengths from the schedule with
 conf ~ Beta(8,2), tau = 0.3).  Inputs are synthetic and seeded.  Workloads
@@ -394,9 +396,11 @@ def run_ours(args, rank, world, local_rank):
 
     def step(i, zt, zd, tokens, temp, conf, ln):
         if fixed is None:
-            sv.sv_schedule(conf, batch.tau, ln)
-        sv.sv_verify(zt, zd, tokens, ln, temp, args.seed + i, out_tok, out_acc, ws,
-                     status=status, row_base=row_base)
+            sv.sv_schedule_verify(zt, zd, tokens, conf, batch.tau, ln, temp, args.seed + i, out_tok,
+                                  out_acc, ws, status=status, row_base=row_base)
+        else:
+            sv.sv_verify(zt, zd, tokens, ln, temp, args.seed + i, out_tok, out_acc, ws,
+                         status=status, row_base=row_base)
 
     ln_buf = lengths if fixed is None else fixed
     for i in range(args.warmup):
@@ -659,8 +663,7 @@ def run_ours(args, rank, world, local_rank):
                "dtype": "f32", "data": "synthetic",
                "config": dict(workload_config(batch, lengths_np, esize),
                               parallelism=f"dp{world} (row shards, no collective)"),
-               "e2e": e2e, "gpu_launches": args.steps * (sv.sv_verify_launches()
-                                                         + (1 if fixed is None else 0)),
+               "e2e": e2e, "gpu_launches": args.steps * sv.sv_verify_launches(),
                "roofline": roofline, "cpu_baseline": cpu, "parity": parity, "clocks": clk,
                "schedule": sched,
                "admission": admit,

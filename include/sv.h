@@ -285,6 +285,32 @@ sv_status sv_verify(const void *target_logits, const void *draft_logits, sv_dtyp
                     void *stream);
 
 /*
+ * sv_schedule_verify -- sv_schedule followed by sv_verify, in one call and
+ * without the schedule launch: the verification prologue computes each
+ * row's length from its confidences with the same function as sv_schedule
+ * (same formula, same fp32 order), writes it to `lengths`, and verifies
+ * with it.  Lengths and outputs are identical, bit for bit, to calling
+ * sv_schedule(conf, B, K, load, lengths) and then sv_verify with `lengths`.
+ *
+ * Defined by: the passages cited at sv_schedule and sv_verify.
+ *
+ *   conf      device, float32 [B, K], read only (as sv_schedule).
+ *   load      threshold tau (as sv_schedule).
+ *   lengths   device, int32 [B], written: the scheduled verify lengths.
+ *   Every other argument is that of sv_verify.
+ * Returns SV_OK, SV_ERR_ARG (a null pointer, including conf or lengths),
+ * SV_ERR_DTYPE, SV_ERR_SHAPE, SV_ERR_WORKSPACE or SV_ERR_CUDA; the workspace
+ * is sv_verify_workspace_bytes(B, K, V, dtype).
+ */
+sv_status sv_schedule_verify(const void *target_logits, const void *draft_logits, sv_dtype dtype,
+                             int B, int K, int V, const int32_t *draft_tokens,
+                             const float *conf, float load, int32_t *lengths,
+                             const float *temperature, uint64_t seed, int64_t row_base,
+                             int32_t *out_tokens, int32_t *out_accept_len,
+                             void *workspace, size_t workspace_bytes, int32_t *status,
+                             void *stream);
+
+/*
  * sv_verify_debug -- sv_verify plus an export of the softmax normalisers it
  * computed: stats_out (device float32 [B, 2K+1, 2]) receives, for every
  * vector the call read, (m, Sigma) with m = max_v z_v and

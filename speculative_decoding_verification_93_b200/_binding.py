@@ -59,6 +59,8 @@ def lib():
     L.sv_verify_workspace_bytes.restype = sz
     L.sv_verify.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, u64, i64, vp, vp, vp, sz, vp,
                             vp]
+    L.sv_schedule_verify.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, ctypes.c_float, vp, vp,
+                                     u64, i64, vp, vp, vp, sz, vp, vp]
     L.sv_verify_debug.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, u64, i64, vp, vp, vp,
                                   sz, vp, vp, vp]
     L.sv_verify_noalloc.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, u64, i64, vp, vp, vp,
@@ -242,6 +244,22 @@ def sv_verify(target_logits, draft_logits, draft_tokens, lengths, temperature, s
         _ptr(temperature), ctypes.c_uint64(seed & (2**64 - 1)), int(row_base), _ptr(out_tokens),
         _ptr(out_accept_len), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _ptr(status), _stream(stream, target_logits)))
+
+
+def sv_schedule_verify(target_logits, draft_logits, draft_tokens, conf, load: float, lengths,
+                       temperature, seed: int, out_tokens, out_accept_len, workspace, status=None,
+                       row_base: int = 0, stream=None) -> None:
+    """sv_schedule then sv_verify in one call: `lengths` receives the
+    scheduled lengths (see include/sv.h)."""
+    B, K, V, dt = _verify_args(target_logits, draft_logits, draft_tokens, lengths, temperature)
+    _need(conf, torch.float32, "conf")
+    if tuple(conf.shape) != (B, K):
+        raise TypeError("conf must be a [B, K] float32 tensor")
+    _check("sv_schedule_verify", lib().sv_schedule_verify(
+        _ptr(target_logits), _ptr(draft_logits), dt, B, K, V, _ptr(draft_tokens), _ptr(conf),
+        float(load), _ptr(lengths), _ptr(temperature), ctypes.c_uint64(seed & (2**64 - 1)),
+        int(row_base), _ptr(out_tokens), _ptr(out_accept_len), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream, target_logits)))
 
 
 def sv_verify_debug(target_logits, draft_logits, draft_tokens, lengths, temperature, seed: int,

@@ -33,18 +33,8 @@ __global__ void schedule_kernel(const float *__restrict__ conf, int B, int K, fl
                                 int32_t *__restrict__ lengths) {
     griddep_wait();                 // the previous step may still read `lengths`
     griddep_launch_dependents();    // the verification prologue may launch now
-    for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < B; b += gridDim.x * blockDim.x) {
-        const float *c = conf + static_cast<long long>(b) * K;
-        float S = 1.f;
-        int L = 0;
-        for (int i = 1; i <= K; ++i) {
-            float ci = __ldg(c + (i - 1));
-            ci = isnan(ci) ? 0.f : fminf(fmaxf(ci, 0.f), 1.f);
-            S = S * ci;
-            if (S >= tau) L = i;
-        }
-        lengths[b] = L;
-    }
+    for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < B; b += gridDim.x * blockDim.x)
+        lengths[b] = schedule_length(conf + static_cast<long long>(b) * K, K, tau);
 }
 
 // ---------------------------------------------------------------------------

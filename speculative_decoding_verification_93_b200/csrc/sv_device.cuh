@@ -361,6 +361,23 @@ __device__ __forceinline__ int atom_add_acq_rel(int *p, int v) {
     return old;
 }
 
+// Verify length of one row from its K confidences: S_i = prod_{j<=i}
+// clamp(c_{j-1}, 0, 1) (NaN counts as 0), left to right in fp32, and
+// L = max{i in 0..K : S_i >= tau} with S_0 = 1.  The schedule kernel and the
+// fused schedule-and-verify prologue both call this, so their lengths agree
+// bit for bit.
+__device__ __forceinline__ int schedule_length(const float *__restrict__ c, int K, float tau) {
+    float S = 1.f;
+    int L = 0;
+    for (int i = 1; i <= K; ++i) {
+        float ci = __ldg(c + (i - 1));
+        ci = isnan(ci) ? 0.f : fminf(fmaxf(ci, 0.f), 1.f);
+        S = S * ci;
+        if (S >= tau) L = i;
+    }
+    return L;
+}
+
 // Relaxed load of a flag that other CTAs update (a stale value only makes
 // the caller do redundant work).
 __device__ __forceinline__ int ld_relaxed(const int *p) {

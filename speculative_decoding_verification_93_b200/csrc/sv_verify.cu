@@ -83,6 +83,9 @@ struct VerifyArgs {
     int32_t *out_accept;       // [B]
     int32_t *status;           // nullable
     float *dbg;                // nullable [B, S, 2]
+    const float *conf;         // [B, K] confidences, or null: lengths given
+    float tau;                 // schedule threshold when conf is set
+    int32_t *lengths_out;      // [B] scheduled lengths, written when conf is set
     int *ctr;                  // [0] next item, [1] total items, [2] a wait ran out
     int *rcnt;                 // [B]  chunks of the residual draw done
     int *leff;                 // [B]  verify length of a valid row, -1 for an invalid one
@@ -104,8 +107,7 @@ __device__ __forceinline__ const char *vec_ptr(const VerifyArgs &a, int b, int s
 }
 
 // Row data checks: status bits, 0 if the row is valid.
-__device__ __forceinline__ int row_errors(const VerifyArgs &a, int b) {
-    const int L = a.lengths[b];
+__device__ __forceinline__ int row_errors(const VerifyArgs &a, int b, int L) {
     const float T = a.temp[b];
     int bits = 0;
     if (L < 0 || L > a.K) bits |= SV_ROW_BAD_LENGTH;
@@ -155,7 +157,12 @@ __global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(VerifyArgs a
     const bool draft = a.zd != nullptr;
     // Rows: validity, effective length, first-rejection marker, counters.
     for (int b = tid; b < a.B; b += kPrologueThreads) {
-        const int bits = row_errors(a, b);
+        // The row's length: given, or scheduled here from its confidences
+        // (the schedule kernel's own function, so the lengths agree).
+        const int L0 = a.conf ? schedule_length(a.conf + static_cast<long long>(b) * a.K, a.K, a.tau)
+                              : a.lengths[b];
+        if (a.conf) a.lengths_out[b] = L0;
+        const int bits = row_errors(a, b, L0);
         int Lb = -1;
         if (bits) {
             a.out_accept[b] = -1;
@@ -163,7 +170,7 @@ __global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(VerifyArgs a
                 a.out_tokens[static_cast<long long>(b) * K1 + i] = -1;
             if (a.status) atomicOr(a.status, bits);
         } else {
-            Lb = a.lengths[b];
+            Lb = L0;
         }
         a.leff[b] = Lb;
         a.row_j[b] = Lb;
@@ -1739,9 +1746,10 @@ static sv_status verify_impl(const void *zt, const void *zd, sv_dtype dtype, int
                              const int32_t *tokens, const int32_t *lengths, const float *temp,
                              uint64_t seed, int64_t row_base, int32_t *out_tokens,
                              int32_t *out_accept, void *ws, size_t ws_bytes, int32_t *status,
-                             float *dbg, void *stream) {
-    if (!zt || !tokens || !lengths || !temp || !out_tokens || !out_accept || !ws)
-        return SV_ERR_ARG;
+                             float *dbg, void *stream, const float *conf = nullptr,
+                             float tau = 0.f, int32_t *lengths_out = nullptr) {
+    if (!zt || !tokens || !temp || !out_tokens || !out_accept || !ws) return SV_ERR_ARG;
+    if (conf ? !lengths_out : !lengths) return SV_ERR_ARG;
     if (dtype != SV_F32 && dtype != SV_BF16) return SV_ERR_DTYPE;
     Plan p;
     if (!make_plan(B, K, V, dtype, &p)) return SV_ERR_SHAPE;
@@ -1757,6 +1765,7 @@ static sv_status verify_impl(const void *zt, const void *zd, sv_dtype dtype, int
     a.zd = static_cast<const char *>(zd);
     a.B = B; a.K = K; a.V = V; a.S = p.S; a.C = p.C; a.U = p.U;
     a.tokens = tokens; a.lengths = lengths; a.temp = temp;
+    a.conf = conf; a.tau = tau; a.lengths_out = lengths_out;
     a.seed = seed; a.row_base = row_base;
     a.out_tokens = out_tokens; a.out_accept = out_accept; a.status = status; a.dbg = dbg;
     char *w = static_cast<char *>(ws);
@@ -1817,6 +1826,20 @@ extern "C" sv_status sv_verify(const void *target_logits, const void *draft_logi
     return sv::verify_impl(target_logits, draft_logits, dtype, B, K, V, draft_tokens, lengths,
                            temperature, seed, row_base, out_tokens, out_accept_len, workspace,
                            workspace_bytes, status, nullptr, stream);
+}
+
+extern "C" sv_status sv_schedule_verify(const void *target_logits, const void *draft_logits,
+                                        sv_dtype dtype, int B, int K, int V,
+                                        const int32_t *draft_tokens, const float *conf, float load,
+                                        int32_t *lengths, const float *temperature, uint64_t seed,
+                                        int64_t row_base, int32_t *out_tokens,
+                                        int32_t *out_accept_len, void *workspace,
+                                        size_t workspace_bytes, int32_t *status, void *stream) {
+    sv::NvtxRange nvtx_range("sv_schedule_verify");
+    if (!conf || !lengths) return SV_ERR_ARG;
+    return sv::verify_impl(target_logits, draft_logits, dtype, B, K, V, draft_tokens, nullptr,
+                           temperature, seed, row_base, out_tokens, out_accept_len, workspace,
+                           workspace_bytes, status, nullptr, stream, conf, load, lengths);
 }
 
 extern "C" sv_status sv_verify_debug(const void *target_logits, const void *draft_logits,

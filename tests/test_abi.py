@@ -212,3 +212,23 @@ def test_binding_argtypes_match_header():
             assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
             checked += 1
     assert checked >= 20
+
+
+def test_schedule_verify_arguments_rejected_on_host():
+    L = sv.lib()
+    v = ctypes.c_void_p
+    p = v(1 << 20)
+    ws = v(1 << 24)
+    n = sv.sv_verify_workspace_bytes(4, 4, 1000, sv.SV_BF16)
+
+    def call(zt=p, tok=p, conf=p, ln=p, temp=p, ot=p, oa=p, w=ws, wsb=1 << 40, dtype=sv.SV_BF16,
+             B=4, K=4, V=1000, row_base=0):
+        return L.sv_schedule_verify(zt, None, dtype, B, K, V, tok, conf, ctypes.c_float(0.3), ln,
+                                    temp, ctypes.c_uint64(0), row_base, ot, oa, w, wsb, None, None)
+    for kw in ("zt", "tok", "conf", "ln", "temp", "ot", "oa", "w"):
+        assert call(**{kw: None}) == 1, kw
+    assert call(dtype=4) == 3
+    assert call(K=0) == 2 and call(B=0) == 2 and call(V=(1 << 20) + 1) == 2
+    assert call(row_base=-1) == 1
+    assert call(w=v((1 << 24) + 8)) == 1
+    assert call(wsb=n - 1) == 4
